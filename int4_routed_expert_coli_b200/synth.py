@@ -1,0 +1,172 @@
+"""Seeded synthetic inputs for the routed-expert MoE layer.
+
+This module is the only code shared by the CUDA path and the CPU oracle's
+tests.  It draws random numbers and lays them out in the storage formats of
+the layer's inputs; it computes nothing of the layer itself (no routing, no
+dequantisation, no matmul, no activation).
+
+Formats (the layer's inputs, as the C-ABI header documents them):
+
+* expert matrices ``gate_q``/``up_q`` ``[I][H/2]`` and ``down_q`` ``[H][I/2]``
+  are uint8, two signed int4 codes per byte along the reduction dimension;
+  a uniformly random byte gives two independent codes uniform over [-8, 7].
+* scales ``gate_s``/``up_s`` ``[I][H/64]`` and ``down_s`` ``[H][I/64]`` are
+  bf16, drawn from U(0.005, 0.02) in fp32 and rounded to bf16 (RNE).
+* activations ``x`` ``[T][H]`` are bf16 drawn from N(0, 1).
+* router logits ``[T][E]`` are fp32; the router weight ``[E][H]`` is fp32
+  N(0, 0.02).
+
+The workloads follow the pages' GLM-5.2 numbers (256 routed experts, 8 + 1
+active per layer, about 19 MB per int4 expert: "zhichai.net/topic/178503686",
+section on MoE sparsity; "yunpan.plus/t/30351-1-1", memory-tier section).
+
+Zipf-skewed routing (``zipf_routing``) realises a chosen expert set through
+logits: chosen experts get 3 + |N(0,1)|, the rest min(N(0,1), 2.5), so any
+correct top-k over those logits returns exactly the drawn set.  The 71.6 %
+repeat probability is the pages' one-layer-ahead predictability figure
+("yunpan.plus/t/30351-1-1", memory-tier section), reused as a step-to-step
+repeat rate.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+GROUP = 64  # K elements per bf16 scale (the gs64 container)
+
+
+@dataclasses.dataclass
+class ExpertBank:
+    """All experts of one layer: ``n`` = routed + shared, shared last.
+
+    Each tensor's leading dim is the expert; one expert's matrix is a
+    contiguous slice, so per-expert device pointers are plain offsets.
+    """
+
+    hidden: int
+    inter: int
+    n: int
+    gate_q: torch.Tensor  # [n][I][H/2]  uint8
+    up_q: torch.Tensor    # [n][I][H/2]  uint8
+    down_q: torch.Tensor  # [n][H][I/2]  uint8
+    gate_s: torch.Tensor  # [n][I][H/64] bf16
+    up_s: torch.Tensor    # [n][I][H/64] bf16
+    down_s: torch.Tensor  # [n][H][I/64] bf16
+
+    def expert_numpy(self, e: int) -> dict:
+        """Copy expert ``e`` to host numpy arrays (scales as raw bf16 bits)."""
+        out = {}
+        for name in ("gate_q", "up_q", "down_q"):
+            out[name] = getattr(self, name)[e].cpu().numpy()
+        for name in ("gate_s", "up_s", "down_s"):
+            out[name] = getattr(self, name)[e].cpu().view(torch.int16).numpy().view(np.uint16)
+        return out
+
+    def nbytes_per_expert(self) -> int:
+        h, i = self.hidden, self.inter
+        return 3 * h * i // 2 + 3 * (h * i // GROUP) * 2
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def make_expert_bank(hidden: int, inter: int, n_experts: int, seed: int,
+                     device="cpu") -> ExpertBank:
+    """Random int4 gs64 experts: codes uniform over [-8, 7], scales U(.005,.02)."""
+    if hidden % (2 * GROUP) or inter % (2 * GROUP):
+        raise ValueError("hidden and inter must be multiples of 128")
+    g = _gen(seed, device)
+    kw = dict(dtype=torch.uint8, device=device)
+    gate_q = torch.empty(n_experts, inter, hidden // 2, **kw).random_(0, 256, generator=g)
+    up_q = torch.empty(n_experts, inter, hidden // 2, **kw).random_(0, 256, generator=g)
+    down_q = torch.empty(n_experts, hidden, inter // 2, **kw).random_(0, 256, generator=g)
+
+    def scales(rows, cols):
+        s = torch.empty(n_experts, rows, cols, dtype=torch.float32, device=device)
+        s.uniform_(0.005, 0.02, generator=g)
+        return s.to(torch.bfloat16)
+
+    gate_s = scales(inter, hidden // GROUP)
+    up_s = scales(inter, hidden // GROUP)
+    down_s = scales(hidden, inter // GROUP)
+    return ExpertBank(hidden, inter, n_experts, gate_q, up_q, down_q, gate_s, up_s, down_s)
+
+
+def make_activations(tokens: int, hidden: int, seed: int, device="cpu") -> torch.Tensor:
+    """x [T][H] bf16, N(0, 1)."""
+    g = _gen(seed, device)
+    return torch.randn(tokens, hidden, generator=g, device=device).to(torch.bfloat16)
+
+
+def make_router_weight(n_routed: int, hidden: int, seed: int, device="cpu") -> torch.Tensor:
+    """W_r [E][H] fp32, N(0, 0.02)."""
+    g = _gen(seed, device)
+    return torch.randn(n_routed, hidden, generator=g, device=device) * 0.02
+
+
+def make_logits_normal(tokens: int, n_routed: int, seed: int, device="cpu") -> torch.Tensor:
+    """Router logits [T][E] fp32, N(0, 1)."""
+    g = _gen(seed, device)
+    return torch.randn(tokens, n_routed, generator=g, device=device)
+
+
+def make_logits_uniform(tokens: int, n_routed: int, seed: int, device="cpu") -> torch.Tensor:
+    """Router logits [T][E] fp32, U[0, 1)."""
+    g = _gen(seed, device)
+    return torch.rand(tokens, n_routed, generator=g, device=device)
+
+
+def make_residual(tokens: int, hidden: int, seed: int, dtype=torch.float32,
+                  device="cpu") -> torch.Tensor:
+    g = _gen(seed, device)
+    return torch.randn(tokens, hidden, generator=g, device=device).to(dtype)
+
+
+def zipf_routing(tokens: int, n_routed: int, top_k: int, steps: int, seed: int,
+                 exponent: float = 1.1, repeat: float = 0.716):
+    """Zipf-skewed expert sets per step and logits that realise them.
+
+    Returns ``(sets, logits)``: ``sets[s]`` is an int array [T][k] of the drawn
+    experts (unordered), ``logits[s]`` a float32 array [T][E] whose top-k per
+    row is exactly that set.
+    """
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(n_routed)               # Zipf rank -> expert id
+    p = np.arange(1, n_routed + 1, dtype=np.float64) ** (-exponent)
+    p /= p.sum()
+
+    def draw(exclude):
+        while True:
+            e = int(perm[rng.choice(n_routed, p=p)])
+            if e not in exclude:
+                return e
+
+    sets, logits = [], []
+    prev = None
+    for s in range(steps):
+        cur = np.empty((tokens, top_k), dtype=np.int64)
+        for t in range(tokens):
+            picked: list[int] = []
+            for j in range(top_k):
+                if prev is not None and rng.random() < repeat:
+                    cand = int(prev[t, j])
+                    if cand not in picked:
+                        picked.append(cand)
+                        continue
+                excl = set(picked) | (set(prev[t].tolist()) if prev is not None else set())
+                if len(excl) >= n_routed:
+                    excl = set(picked)
+                picked.append(draw(excl))
+            cur[t] = picked
+        lg = np.minimum(rng.standard_normal((tokens, n_routed)), 2.5)
+        for t in range(tokens):
+            lg[t, cur[t]] = 3.0 + np.abs(rng.standard_normal(top_k))
+        sets.append(cur)
+        logits.append(lg.astype(np.float32))
+        prev = cur
+    return sets, logits
