@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of one routed int4 gs64 MoE layer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, same workload
+
+Default workload: GLM-5.2-shaped single-token decode (H 6144, I 2048, 256
+routed experts top-8 + 1 shared, about 19 MB per int4 gs64 expert, all 257
+experts resident in HBM), fresh seeded token and N(0,1) router logits every
+step.  A step is one full layer call through the C ABI (route, batch-union,
+gate/up, down, combine).  Inputs for every step sit in HBM before the timed
+region; L2 is flushed (a 256 MiB write) between timed steps and each step is
+timed alone with CUDA events on the launching stream.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own token
+stream (no data-path collective); the timed total is the max over ranks and
+`value` counts the tokens of all ranks ("scaling": "weak").
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_routed_expert_coli_b200 import synth  # noqa: E402
+
+GLM = dict(H=6144, I=2048, E=256, k=8, n_shared=1)
+WORKLOADS = {
+    # name: (tokens per step, routing kind, description)
+    "decode": (1, "normal", "GLM-5.2-shaped single-token decode: H 6144, I 2048, 256 routed "
+                            "experts top-8 + 1 shared, int4 gs64, T=1, logits N(0,1)"),
+    "verify4": (4, "zipf", "GLM-5.2-shaped speculative verify: T=4, Zipf-1.1 routing, "
+                           "71.6% step-to-step expert repeats"),
+    "batch32": (32, "zipf", "GLM-5.2-shaped small-batch decode: T=32, Zipf-1.1 routing, "
+                            "71.6% step-to-step expert repeats"),
+    "prefill": (4096, "uniform", "GLM-5.2-shaped prefill: T=4096, logits U[0,1)"),
+}
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def expert_bytes(H, I):
+    return 3 * H * I // 2 + 3 * (H * I // 64) * 2
+
+
+def gateup_bytes(H, I):
+    return 2 * (H * I // 2) + 2 * (H * I // 64) * 2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def make_inputs(name, steps, seed, device):
+    """Per-step activations and logits (lists of device tensors)."""
+    T, kind, _ = WORKLOADS[name]
+    xs, lgs = [], []
+    if kind == "zipf":
+        _, lg_np = synth.zipf_routing(T, GLM["E"], GLM["k"], steps=steps, seed=seed)
+    for s in range(steps):
+        xs.append(synth.make_activations(T, GLM["H"], seed=seed * 100003 + s, device=device))
+        if kind == "normal":
+            lgs.append(synth.make_logits_normal(T, GLM["E"], seed=seed * 100019 + s, device=device))
+        elif kind == "uniform":
+            lgs.append(synth.make_logits_uniform(T, GLM["E"], seed=seed * 100019 + s, device=device))
+        else:
+            lgs.append(torch.from_numpy(lg_np[s]).to(device))
+    return xs, lgs
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        sel = []
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            sel = ["--id=" + bus]
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            sel = ["-i", vis.split(",")[device_index]] if vis else ["-i", str(device_index)]
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = list(csv.reader(io.StringIO(self.file.read())))
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        load = [v for v in sm if v > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+def oracle_steps(bank, xs, lgs, n_threads):
+    """Oracle on the given steps (every token of every step); returns
+    (seconds, tokens)."""
+    import oracle
+    E, k, n_sh = GLM["E"], GLM["k"], GLM["n_shared"]
+    routes = [oracle.route(lg.float().cpu().numpy(), k) for lg in lgs]
+    needed = set(range(E, E + n_sh))
+    for idx, _ in routes:
+        needed |= set(idx.ravel().tolist())
+    ex = oracle.Experts([bank.expert_numpy(e) if e in needed else None for e in range(bank.n)])
+    xb = [x.view(torch.int16).cpu().numpy().view(np.uint16) for x in xs]
+    # all steps' tokens in one batch: the oracle is per token, so this is the
+    # same work as running the steps one after another, spread over threads
+    X = np.concatenate(xb, axis=0)
+    IDX = np.concatenate([r[0] for r in routes], axis=0)
+    W = np.concatenate([r[1] for r in routes], axis=0)
+    t0 = time.perf_counter()
+    oracle.layer(GLM["H"], GLM["I"], E, k, n_sh, ex, X, IDX, W, n_threads=n_threads)
+    return time.perf_counter() - t0, X.shape[0]
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle on the same workload: each step is one full layer step
+    of the workload (all its tokens), timed on the host cores."""
+    if rank != 0:
+        return
+    name = args.workload
+    T, _, desc = WORKLOADS[name]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    bank = synth.make_expert_bank(GLM["H"], GLM["I"], GLM["E"] + 1, seed=1, device=dev)
+    cores = os.cpu_count() or 1
+    n = args.warmup + args.steps
+    sample_tokens = min(T, 8)  # tokens per step the oracle computes (prefill: a sample)
+    xs, lgs = make_inputs(name, n, seed=7, device=dev)
+    xs = [x[:sample_tokens] for x in xs]
+    lgs = [lg[:sample_tokens] for lg in lgs]
+    sec = 0.0
+    toks = 0
+    for i in range(n):
+        s, t = oracle_steps(bank, [xs[i]], [lgs[i]], n_threads=cores)
+        if i >= args.warmup:
+            sec += s
+            toks += t
+    value = toks / sec
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": desc, "tokens_per_step": sample_tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {sample_tokens} token(s) each, "
+                                   f"all {GLM['k']}+{GLM['n_shared']} experts per token"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local):
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    name = args.workload
+    T, kind, desc = WORKLOADS[name]
+    H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    bank = synth.make_expert_bank(H, I, E + n_sh, seed=1, device=dev)
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=n_sh)
+    n = args.warmup + args.steps
+    xs, lgs = make_inputs(name, n, seed=1000 + rank, device=dev)
+    ws = layer.workspace(T, dev)
+    out = torch.empty(T, H, dtype=torch.float32, device=dev)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c.coli_moe_layer(layer.handle, T, xs[i], lgs[i], None, None, out, c.COLI_OUT_F32, idx,
+                         None, ws, stream)
+
+    for i in range(args.warmup):
+        step(i)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    if c.coli_moe_get_status(ws) != c.COLI_OK:
+        raise RuntimeError("device status after warm-up: " + c.status_string(c.coli_moe_get_status(ws)))
+
+    # unique routed experts per timed step (sets the algorithmic bytes)
+    uniq = []
+    for i in range(args.warmup, n):
+        uniq.append(len(set(torch.topk(lgs[i], k, dim=1).indices.flatten().tolist())))
+
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    c.coli_moe_profile_enable(True)
+    for j in range(args.steps):
+        ev[j][0].record(stream)
+        step(args.warmup + j)
+        ev[j][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    c.coli_moe_profile_enable(False)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    phase_ms, n_calls = c.coli_moe_profile_read()
+    total_ms = max_over_ranks(sum(ms_steps), world)
+    if c.coli_moe_get_status(ws) != c.COLI_OK:
+        raise RuntimeError("device status: " + c.status_string(c.coli_moe_get_status(ws)))
+
+    # ---- end to end through the C ABI with host buffers --------------------
+    x_host = torch.stack([x.cpu() for x in xs[args.warmup:]]).pin_memory()
+    lg_host = torch.stack([lg.cpu() for lg in lgs[args.warmup:]]).pin_memory()
+    out_host = torch.empty(args.steps, T, H, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    lg_dev = torch.empty(T, E, dtype=torch.float32, device=dev)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for j in range(args.steps):
+        ev2[j][0].record(stream)
+        x_dev.copy_(x_host[j], non_blocking=True)
+        lg_dev.copy_(lg_host[j], non_blocking=True)
+        c.coli_moe_layer(layer.handle, T, x_dev, lg_dev, None, None, out, c.COLI_OUT_F32, None,
+                         None, ws, stream)
+        out_host[j].copy_(out, non_blocking=True)
+        ev2[j][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) --------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        n_s = max(1, min(args.steps, 2 * cores // (k + n_sh) + 1, 16 if T == 1 else 2))
+        tok = min(T, 8)
+        sec, toks = oracle_steps(bank, [x[:tok] for x in xs[args.warmup:args.warmup + n_s]],
+                                 [lg[:tok] for lg in lgs[args.warmup:args.warmup + n_s]],
+                                 n_threads=cores)
+        cpu = {"value": toks / sec, "unit": "tokens/s",
+               "cores": min(cores, toks * (k + n_sh)), "kind": "oracle",
+               "sample": f"{n_s} steps x {tok} token(s), every routed + shared expert of each "
+                         f"token, double precision, {sec:.1f} s"}
+
+    if rank != 0:
+        return
+    P = peaks()
+    tokens = T * args.steps * world
+    value = tokens / (total_ms / 1e3)
+    n_uniq = statistics.mean(uniq)
+    step_bytes = (n_uniq + n_sh) * expert_bytes(H, I)
+    gu_ms = phase_ms[1] / max(n_calls, 1)
+    gu_bytes = (n_uniq + n_sh) * gateup_bytes(H, I)
+    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4xbf16/f16->f32", "data": "synthetic",
+        "config": {"workload": desc, "tokens_per_step": T, "hidden": H, "inter": I,
+                   "routed_experts": E, "top_k": k, "shared_experts": n_sh,
+                   "expert_bytes": expert_bytes(H, I), "unique_routed_experts_per_step": n_uniq,
+                   "l2": "flushed between timed steps (256 MiB write), steps timed alone",
+                   "parallelism": f"replicas x{world}"},
+        "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": achieved,
+                     "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
+                     "peak_source": P["src"], "traffic": None,
+                     "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms},
+        "phase_ms_per_step": {"prep": phase_ms[0] / max(n_calls, 1), "gateup": gu_ms,
+                              "down": phase_ms[2] / max(n_calls, 1),
+                              "combine": phase_ms[3] / max(n_calls, 1)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 4},
+        "gpu_launches": 7 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

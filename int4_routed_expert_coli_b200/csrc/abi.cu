@@ -1,0 +1,346 @@
+// Host side of the C ABI declared in include/coli_moe.h: argument checks,
+// workspace carving and kernel launches.  Every check runs before anything is
+// enqueued, so a call that returns an error has launched nothing.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "coli_internal.cuh"
+
+struct coli_moe {
+    int device;
+    int H, I, E, k, n_shared, prefill_min;
+    int num_sms;
+    coli::DevExpert* d_experts;  // device table, E + n_shared entries
+};
+
+namespace {
+
+using coli::kGroup;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+coli_status check_route_dims(int32_t T, int32_t E, int32_t k) {
+    if (T < 0) return COLI_ERR_INVALID_ARG;
+    if (E < 1 || E > coli::kMaxExperts || k < 1 || k > E || k > coli::kMaxTopK)
+        return COLI_ERR_SHAPE;
+    if ((int64_t)T * k > (int64_t)1 << 24) return COLI_ERR_SHAPE;
+    return COLI_OK;
+}
+
+coli_status from_cuda(cudaError_t e) { return e == cudaSuccess ? COLI_OK : COLI_ERR_CUDA; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+coli::WsLayout layout_for(const coli_moe* h, int64_t T) {
+    return coli::ws_layout(T, h->E, h->k, h->H, h->I, h->n_shared);
+}
+
+// Shared validation of the FFN-side arguments.
+coli_status check_ffn_common(const coli_moe* h, int32_t T, const void* x, const void* residual,
+                             const void* out, int out_dtype, const void* ws, size_t ws_bytes) {
+    if (!h || T < 0) return COLI_ERR_INVALID_ARG;
+    if (out_dtype != COLI_OUT_F32 && out_dtype != COLI_OUT_BF16) return COLI_ERR_INVALID_ARG;
+    if ((int64_t)T * h->k > (int64_t)1 << 24) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    if (!x || !out || !ws) return COLI_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)))
+        return COLI_ERR_ALIGN;
+    if (!aligned(ws, 256)) return COLI_ERR_ALIGN;
+    if (ws_bytes < layout_for(h, T).total) return COLI_ERR_WORKSPACE;
+    return COLI_OK;
+}
+
+coli::FfnArgs make_args(const coli_moe* h, int32_t T, const void* x, const float* w,
+                        const int32_t* offsets, const int32_t* pairs, const int32_t* active,
+                        const int32_t* n_active, const void* residual, void* out,
+                        coli_out_dtype od, void* ws) {
+    const coli::WsLayout L = layout_for(h, T);
+    coli::FfnArgs a;
+    a.experts = h->d_experts;
+    a.H = h->H;
+    a.I = h->I;
+    a.E = h->E;
+    a.k = h->k;
+    a.n_shared = h->n_shared;
+    a.T = T;
+    a.offsets = offsets;
+    a.pairs = pairs;
+    a.active = active;
+    a.n_active = n_active;
+    a.topk_w = w;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.xp = at<__nv_bfloat16>(ws, L.xp);
+    a.inv = at<int>(ws, L.inv);
+    a.hp = at<__half>(ws, L.hp);
+    a.y = at<float>(ws, L.y);
+    a.residual = residual;
+    a.out = out;
+    a.out_bf16 = od == COLI_OUT_BF16;
+    a.status = at<int>(ws, 0);
+    return a;
+}
+
+// Timing diagnostics: one set of 5 events per recorded call.
+struct ProfileState {
+    bool enabled = false;
+    std::vector<cudaEvent_t> events;  // 5 per call
+    int open_call = -1;               // index of the call being recorded
+};
+ProfileState g_prof;
+
+void profile_begin_call(cudaStream_t st) {
+    if (!g_prof.enabled) return;
+    const size_t base = g_prof.events.size();
+    for (int i = 0; i < 5; ++i) {
+        cudaEvent_t ev = nullptr;
+        if (cudaEventCreate(&ev) != cudaSuccess) {
+            g_prof.open_call = -1;
+            return;
+        }
+        g_prof.events.push_back(ev);
+    }
+    g_prof.open_call = (int)(base / 5);
+    cudaEventRecord(g_prof.events[base], st);
+}
+
+void profile_end_call() { g_prof.open_call = -1; }
+
+}  // namespace
+
+namespace coli {
+cudaEvent_t profile_event(int i) {
+    if (!g_prof.enabled || g_prof.open_call < 0 || i < 0 || i > 4) return nullptr;
+    return g_prof.events[(size_t)g_prof.open_call * 5 + i];
+}
+}  // namespace coli
+
+extern "C" {
+
+coli_status coli_moe_profile_enable(int32_t enable) {
+    g_prof.enabled = enable != 0;
+    g_prof.open_call = -1;
+    return COLI_OK;
+}
+
+coli_status coli_moe_profile_read(double* ms, int32_t* n_calls) {
+    if (!ms || !n_calls) return COLI_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i) ms[i] = 0.0;
+    const size_t calls = g_prof.events.size() / 5;
+    coli_status st = COLI_OK;
+    for (size_t c = 0; c < calls; ++c) {
+        cudaEvent_t* ev = &g_prof.events[c * 5];
+        if (cudaEventSynchronize(ev[4]) != cudaSuccess) st = COLI_ERR_CUDA;
+        for (int i = 0; i < 4; ++i) {
+            float t = 0.f;
+            if (cudaEventElapsedTime(&t, ev[i], ev[i + 1]) == cudaSuccess) ms[i] += t;
+            else st = COLI_ERR_CUDA;
+        }
+    }
+    for (cudaEvent_t ev : g_prof.events) cudaEventDestroy(ev);
+    g_prof.events.clear();
+    g_prof.open_call = -1;
+    *n_calls = (int32_t)calls;
+    return st;
+}
+
+coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
+    if (!out) return COLI_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!d || !d->experts) return COLI_ERR_INVALID_ARG;
+    if (d->group_size != kGroup) return COLI_ERR_SHAPE;
+    if (d->hidden <= 0 || d->inter <= 0 || d->hidden % 128 || d->inter % 128) return COLI_ERR_SHAPE;
+    if (d->n_routed < 1 || d->n_routed > coli::kMaxExperts) return COLI_ERR_SHAPE;
+    if (d->top_k < 1 || d->top_k > d->n_routed || d->top_k > coli::kMaxTopK) return COLI_ERR_SHAPE;
+    if (d->n_shared < 0 || d->n_shared > coli::kMaxShared) return COLI_ERR_SHAPE;
+    if (d->prefill_min_tokens < 0) return COLI_ERR_INVALID_ARG;
+    const int n = d->n_routed + d->n_shared;
+    for (int e = 0; e < n; ++e) {
+        const coli_expert& x = d->experts[e];
+        const void* ptrs[6] = {x.gate_q, x.up_q, x.down_q, x.gate_s, x.up_s, x.down_s};
+        for (const void* p : ptrs) {
+            if (!p) return COLI_ERR_INVALID_ARG;
+            if (!aligned(p, 16)) return COLI_ERR_ALIGN;
+        }
+    }
+    int dev = 0, major = 0, minor = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return COLI_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return COLI_ERR_CUDA;
+    if (major != 10 || minor != 0) return COLI_ERR_UNSUPPORTED;  // built for sm_100a only
+
+    coli_moe* h = new (std::nothrow) coli_moe;
+    if (!h) return COLI_ERR_INVALID_ARG;
+    h->device = dev;
+    h->H = d->hidden;
+    h->I = d->inter;
+    h->E = d->n_routed;
+    h->k = d->top_k;
+    h->n_shared = d->n_shared;
+    h->prefill_min = d->prefill_min_tokens;
+    h->num_sms = sms;
+    h->d_experts = nullptr;
+    coli::DevExpert* host = static_cast<coli::DevExpert*>(std::malloc(sizeof(coli::DevExpert) * n));
+    if (!host) {
+        delete h;
+        return COLI_ERR_INVALID_ARG;
+    }
+    for (int e = 0; e < n; ++e) {
+        host[e].gate_q = d->experts[e].gate_q;
+        host[e].up_q = d->experts[e].up_q;
+        host[e].down_q = d->experts[e].down_q;
+        host[e].gate_s = d->experts[e].gate_s;
+        host[e].up_s = d->experts[e].up_s;
+        host[e].down_s = d->experts[e].down_s;
+    }
+    cudaError_t err = cudaMalloc(&h->d_experts, sizeof(coli::DevExpert) * n);
+    if (err == cudaSuccess)
+        err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
+    std::free(host);
+    if (err != cudaSuccess) {
+        if (h->d_experts) cudaFree(h->d_experts);
+        delete h;
+        return COLI_ERR_CUDA;
+    }
+    *out = h;
+    return COLI_OK;
+}
+
+void coli_moe_destroy(coli_moe* h) {
+    if (!h) return;
+    cudaFree(h->d_experts);
+    delete h;
+}
+
+size_t coli_moe_workspace_size(const coli_moe* h, int32_t max_tokens) {
+    if (!h || max_tokens < 0) return 0;
+    return layout_for(h, max_tokens).total;
+}
+
+coli_status coli_moe_workspace_clear(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes < coli::kHeaderBytes) return COLI_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return COLI_ERR_ALIGN;
+    return from_cuda(cudaMemsetAsync(ws, 0, coli::kHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_route(int32_t T, int32_t E, int32_t k, const float* logits,
+                           int32_t* topk_idx, float* topk_w, void* stream) {
+    coli_status s = check_route_dims(T, E, k);
+    if (s != COLI_OK || T == 0) return s;
+    if (!logits || !topk_idx || !topk_w) return COLI_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return COLI_ERR_ALIGN;
+    return from_cuda(coli::launch_route(T, E, k, logits, topk_idx, topk_w,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_union(int32_t T, int32_t E, int32_t k, const int32_t* topk_idx,
+                           int32_t* counts, int32_t* offsets, int32_t* pairs, int32_t* active,
+                           int32_t* n_active, void* ws, size_t ws_bytes, void* stream) {
+    coli_status s = check_route_dims(T, E, k);
+    if (s != COLI_OK) return s;
+    if (!counts || !offsets || !active || !n_active) return COLI_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !pairs)) return COLI_ERR_INVALID_ARG;
+    const void* ptrs[6] = {topk_idx, counts, offsets, pairs, active, n_active};
+    for (const void* p : ptrs)
+        if (p && !aligned(p, 4)) return COLI_ERR_ALIGN;
+    if (ws && (ws_bytes < coli::kHeaderBytes || !aligned(ws, 256))) return COLI_ERR_WORKSPACE;
+    // T == 0 still writes empty lists (counts 0, offsets 0, no active experts).
+    return from_cuda(coli::launch_union(T, E, k, topk_idx, counts, offsets, pairs, active,
+                                        n_active, ws ? static_cast<int*>(ws) : nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_ffn(const coli_moe* h, int32_t T, const void* x_bf16, const float* topk_w,
+                         const int32_t* counts, const int32_t* offsets, const int32_t* pairs,
+                         const int32_t* active, const int32_t* n_active, const void* residual,
+                         void* out, coli_out_dtype out_dtype, void* ws, size_t ws_bytes,
+                         void* stream) {
+    coli_status s = check_ffn_common(h, T, x_bf16, residual, out, out_dtype, ws, ws_bytes);
+    if (s != COLI_OK || T == 0) return s;
+    if (!topk_w || !counts || !offsets || !pairs || !active || !n_active) return COLI_ERR_INVALID_ARG;
+    const void* ptrs[6] = {topk_w, counts, offsets, pairs, active, n_active};
+    for (const void* p : ptrs)
+        if (!aligned(p, 4)) return COLI_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    coli::FfnArgs a = make_args(h, T, x_bf16, topk_w, offsets, pairs, active, n_active, residual,
+                                out, out_dtype, ws);
+    profile_begin_call(st);
+    cudaError_t err = coli::launch_inverse_pairs(T * h->k, pairs, a.inv, a.status, st);
+    if (err == cudaSuccess) err = coli::launch_ffn_gemv(a, h->num_sms, st);
+    profile_end_call();
+    return from_cuda(err);
+}
+
+coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, const float* logits,
+                           const float* router_w, const void* residual, void* out,
+                           coli_out_dtype out_dtype, int32_t* topk_idx_out, float* topk_w_out,
+                           void* ws, size_t ws_bytes, void* stream) {
+    coli_status s = check_ffn_common(h, T, x_bf16, residual, out, out_dtype, ws, ws_bytes);
+    if (s != COLI_OK) return s;
+    if ((logits == nullptr) == (router_w == nullptr)) return COLI_ERR_INVALID_ARG;
+    if (T == 0) return COLI_OK;
+    const void* ptrs[4] = {logits, router_w, topk_idx_out, topk_w_out};
+    for (const void* p : ptrs)
+        if (p && !aligned(p, 4)) return COLI_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const coli::WsLayout L = layout_for(h, T);
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
+    profile_begin_call(st);
+    cudaError_t err = cudaSuccess;
+    const float* lg = logits;
+    if (router_w) {
+        float* wl = at<float>(ws, L.logits);
+        err = coli::launch_router_logits(T, h->E, h->H, x, router_w, wl, st);
+        lg = wl;
+    }
+    int* idx = topk_idx_out ? topk_idx_out : at<int>(ws, L.idx);
+    float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+    if (err == cudaSuccess) err = coli::launch_route(T, h->E, h->k, lg, idx, w, st);
+    int* counts = at<int>(ws, L.counts);
+    int* offsets = at<int>(ws, L.offsets);
+    int* pairs = at<int>(ws, L.pairs);
+    int* active = at<int>(ws, L.active);
+    int* n_active = at<int>(ws, L.n_active);
+    if (err == cudaSuccess)
+        err = coli::launch_union(T, h->E, h->k, idx, counts, offsets, pairs, active, n_active,
+                                 at<int>(ws, 0), st);
+    coli::FfnArgs a = make_args(h, T, x_bf16, w, offsets, pairs, active, n_active, residual, out,
+                                out_dtype, ws);
+    if (err == cudaSuccess) err = coli::launch_inverse_pairs(T * h->k, pairs, a.inv, a.status, st);
+    if (err == cudaSuccess) err = coli::launch_ffn_gemv(a, h->num_sms, st);
+    profile_end_call();
+    return from_cuda(err);
+}
+
+coli_status coli_moe_get_status(const void* ws, void* stream) {
+    if (!ws) return COLI_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return COLI_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return COLI_ERR_CUDA;
+    return static_cast<coli_status>(word);
+}
+
+const char* coli_status_string(coli_status s) {
+    switch (s) {
+        case COLI_OK: return "ok";
+        case COLI_ERR_INVALID_ARG: return "invalid argument";
+        case COLI_ERR_SHAPE: return "unsupported shape";
+        case COLI_ERR_ALIGN: return "misaligned pointer";
+        case COLI_ERR_WORKSPACE: return "workspace too small";
+        case COLI_ERR_CUDA: return "CUDA runtime error";
+        case COLI_ERR_TIMEOUT: return "device wait timed out";
+        case COLI_ERR_UNSUPPORTED: return "unsupported device or feature";
+        case COLI_ERR_BAD_INDEX: return "expert index out of range";
+        case COLI_ERR_RANGE: return "intermediate outside the fp16 range (clamped)";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

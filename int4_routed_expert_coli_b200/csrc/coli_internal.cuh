@@ -1,0 +1,120 @@
+// Internal declarations shared by the CUDA translation units of libcoli_moe.
+// Not part of the public ABI (include/coli_moe.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "coli_moe.h"
+
+namespace coli {
+
+constexpr int kGroup = 64;        // codes per bf16 scale (gs64)
+constexpr int kMaxExperts = 1024; // E limit (one union thread per expert)
+constexpr int kMaxTopK = 32;      // k limit (one route lane per slot)
+constexpr int kMaxShared = 4;
+constexpr size_t kHeaderBytes = 4096; // status word + counters at the start of ws
+
+// Device status codes live in the first word of the workspace.
+struct WsHeader {
+    int status;   // first device-detected error (coli_status), 0 = none
+    int pad[31];
+};
+
+// One expert as the kernels see it (device table, routed then shared).
+struct DevExpert {
+    const uint8_t* gate_q;   // [I][H/2]
+    const uint8_t* up_q;     // [I][H/2]
+    const uint8_t* down_q;   // [H][I/2]
+    const uint16_t* gate_s;  // [I][H/64] bf16
+    const uint16_t* up_s;    // [I][H/64] bf16
+    const uint16_t* down_s;  // [H][I/64] bf16
+};
+
+// Byte offsets of the workspace regions for a call with T tokens.
+struct WsLayout {
+    size_t logits;   // [T][E] f32   (router GEMV output)
+    size_t idx;      // [T][k] i32
+    size_t w;        // [T][k] f32
+    size_t counts;   // [E] i32
+    size_t offsets;  // [E+1] i32
+    size_t pairs;    // [T*k] i32
+    size_t active;   // [E] i32
+    size_t n_active; // [1] i32
+    size_t inv;      // [T*k] i32: position of pair p in `pairs`
+    size_t xp;       // [T][H] bf16, fragment-permuted copy of x
+    size_t hp;       // [S][I] f16, fragment-permuted SwiGLU output, S = T*k + T*n_shared
+    size_t y;        // [S][H] f32, per-(pair) expert outputs
+    size_t total;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int n_shared) {
+    WsLayout L;
+    size_t o = kHeaderBytes;
+    auto take = [&](size_t bytes) {
+        size_t r = o;
+        o = align_up(o + bytes, 256);
+        return r;
+    };
+    const int64_t P = T * k, S = P + T * n_shared;
+    L.logits = take(sizeof(float) * T * E);
+    L.idx = take(sizeof(int) * P);
+    L.w = take(sizeof(float) * P);
+    L.counts = take(sizeof(int) * E);
+    L.offsets = take(sizeof(int) * (E + 1));
+    L.pairs = take(sizeof(int) * P);
+    L.active = take(sizeof(int) * E);
+    L.n_active = take(sizeof(int));
+    L.inv = take(sizeof(int) * P);
+    L.xp = take(sizeof(uint16_t) * T * H);
+    L.hp = take(sizeof(uint16_t) * S * I);
+    L.y = take(sizeof(float) * S * H);
+    L.total = o;
+    return L;
+}
+
+// Everything the FFN kernels need for one call.
+struct FfnArgs {
+    const DevExpert* experts;
+    int H, I, E, k, n_shared, T;
+    const int* offsets;        // [E+1]
+    const int* pairs;          // [T*k]
+    const int* active;         // [E]
+    const int* n_active;       // [1]
+    const float* topk_w;       // [T][k]
+    const __nv_bfloat16* x;    // [T][H]
+    __nv_bfloat16* xp;         // [T][H] permuted
+    int* inv;                  // [T*k]
+    __half* hp;                // [S][I] permuted
+    float* y;                  // [S][H]
+    const void* residual;      // [T][H] nullable
+    void* out;                 // [T][H]
+    int out_bf16;
+    int* status;
+};
+
+// ---- timing diagnostics (coli_moe_profile_*) ------------------------------
+// Returns the event to record at phase boundary `i` (0..4) of the current
+// call, or nullptr when profiling is off.
+cudaEvent_t profile_event(int i);
+
+// ---- launchers (each returns cudaGetLastError() of its launch) ----------
+cudaError_t launch_router_logits(int T, int E, int H, const __nv_bfloat16* x, const float* wr,
+                                 float* logits, cudaStream_t st);
+cudaError_t launch_route(int T, int E, int k, const float* logits, int* idx, float* w,
+                         cudaStream_t st);
+cudaError_t launch_union(int T, int E, int k, const int* idx, int* counts, int* offsets,
+                         int* pairs, int* active, int* n_active, int* status, cudaStream_t st);
+cudaError_t launch_ffn_gemv(const FfnArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_inverse_pairs(int P, const int* pairs, int* inv, int* status, cudaStream_t st);
+
+// ---- device helpers --------------------------------------------------------
+__device__ __forceinline__ void report(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace coli

@@ -1,0 +1,76 @@
+"""GPU batch-union (coli_moe_union) against the oracle: every output bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import requires_gpu
+from int4_routed_expert_coli_b200 import synth
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+
+def _run(idx: np.ndarray, E: int, ws=None):
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    T, k = idx.shape
+    dev = "cuda"
+    d_idx = torch.from_numpy(np.ascontiguousarray(idx, np.int32)).to(dev) if T else \
+        torch.zeros(1, k, dtype=torch.int32, device=dev)
+    counts = torch.full((E,), -5, dtype=torch.int32, device=dev)
+    offsets = torch.full((E + 1,), -5, dtype=torch.int32, device=dev)
+    pairs = torch.full((max(T * k, 1),), -5, dtype=torch.int32, device=dev)
+    active = torch.full((E,), -5, dtype=torch.int32, device=dev)
+    na = torch.full((1,), -5, dtype=torch.int32, device=dev)
+    c.coli_moe_union(T, E, k, d_idx, counts, offsets, pairs, active, na, ws=ws)
+    torch.cuda.synchronize()
+    return dict(counts=counts.cpu().numpy(), offsets=offsets.cpu().numpy(),
+                pairs=pairs.cpu().numpy()[:T * k], active=active.cpu().numpy(),
+                n_active=int(na.item()))
+
+
+def _check(idx, E):
+    got = _run(idx, E)
+    ref = oracle.union(idx, E)
+    for key in ("counts", "offsets", "pairs", "active"):
+        assert np.array_equal(got[key], ref[key]), key
+    assert got["n_active"] == ref["n_active"]
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 256, 8), (4, 16, 2), (7, 16, 2), (4096, 256, 8),
+                                   (100, 1024, 32), (1000, 37, 5), (1, 1, 1)])
+def test_union_from_routed_logits(T, E, k):
+    lg = np.random.default_rng(T + E).random((T, E), dtype=np.float32)
+    idx, _ = oracle.route(lg, k)
+    _check(idx, E)
+
+
+@pytest.mark.parametrize("T", [4, 32, 64])
+def test_union_zipf_routing(T):
+    sets, logits = synth.zipf_routing(T, 256, 8, steps=3, seed=T)
+    for lg in logits:
+        idx, _ = oracle.route(lg, 8)
+        _check(idx, 256)
+
+
+def test_union_all_to_one_expert_and_empty():
+    idx = np.tile(np.arange(8, dtype=np.int32), (512, 1))   # every token picks 0..7
+    _check(idx, 256)
+    _check(np.zeros((0, 8), np.int32), 256)
+
+
+def test_union_bad_index_sets_status():
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    idx = np.array([[0, 3], [300, 1]], np.int32)
+    got = _run(idx, 16, ws=ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX
+    assert got["offsets"][16] == 3 and got["n_active"] == 3
+
+
+def test_union_deterministic():
+    lg = np.random.default_rng(9).random((4096, 256), dtype=np.float32)
+    idx, _ = oracle.route(lg, 8)
+    a = _run(idx, 256)
+    b = _run(idx, 256)
+    for key in ("counts", "offsets", "pairs", "active"):
+        assert np.array_equal(a[key], b[key])
