@@ -96,8 +96,8 @@ typedef struct {
  * entries, routed experts first, shared experts last; it is copied by
  * coli_moe_create. */
 typedef struct {
-    int32_t hidden;             /* H, multiple of 128 */
-    int32_t inter;              /* I, multiple of 128 */
+    int32_t hidden;             /* H, multiple of 128, at most 12288 */
+    int32_t inter;              /* I, multiple of 128, at most 12288 */
     int32_t n_routed;           /* E, 1..1024 */
     int32_t top_k;              /* k, 1..min(E, 32) */
     int32_t group_size;         /* must be 64 */
@@ -122,7 +122,9 @@ void coli_moe_destroy(coli_moe *h);
 size_t coli_moe_workspace_size(const coli_moe *h, int32_t max_tokens);
 
 /* Zero the workspace's status word and counters (async on `stream`).  Needed
- * once for a new workspace; later calls leave the counters at zero. */
+ * once for a new workspace; later calls leave the counters at zero.  The
+ * first COLI_WS_HEADER_BYTES of a workspace are this header. */
+#define COLI_WS_HEADER_BYTES 16384
 coli_status coli_moe_workspace_clear(void *ws, size_t ws_bytes, void *stream);
 
 /* Router top-k (step 1 of the layer).
@@ -145,8 +147,9 @@ coli_status coli_moe_route(int32_t T, int32_t E, int32_t k, const float *logits,
  *   active   [E]    out: experts with counts > 0, ascending; the rest -1
  *   n_active [1]    out: number of active experts
  * Deterministic: positions come from scans, never from atomic tickets.
- * `ws` may be NULL; if given, an index outside [0, E) is recorded in its
- * status word (the pair is dropped from the lists).
+ * `ws` may be NULL; if given (at least COLI_WS_HEADER_BYTES), an index
+ * outside [0, E) is recorded in its status word (the pair is dropped from
+ * the lists).
  * Errors: INVALID_ARG, SHAPE (as coli_moe_route; T*k > 2^24). */
 coli_status coli_moe_union(int32_t T, int32_t E, int32_t k, const int32_t *topk_idx,
                            int32_t *counts, int32_t *offsets, int32_t *pairs,
@@ -175,7 +178,7 @@ coli_status coli_moe_ffn(const coli_moe *h, int32_t T, const void *x_bf16, const
  * COLI_WS_LOGITS_OFFSET, [T][E] fp32, until the next call.  topk_idx_out /
  * topk_w_out ([T][k]) receive the routing when non-NULL.  Other arguments as
  * coli_moe_ffn. */
-#define COLI_WS_LOGITS_OFFSET 4096
+#define COLI_WS_LOGITS_OFFSET 16384
 coli_status coli_moe_layer(const coli_moe *h, int32_t T, const void *x_bf16, const float *logits,
                            const float *router_w, const void *residual, void *out,
                            coli_out_dtype out_dtype, int32_t *topk_idx_out, float *topk_w_out,
@@ -195,6 +198,16 @@ coli_status coli_moe_get_status(const void *ws, void *stream);
  * reading is host-global state: use it from one thread. */
 coli_status coli_moe_profile_enable(int32_t enable);
 coli_status coli_moe_profile_read(double *ms, int32_t *n_calls);
+
+/* Fault injection for tests (host-global, one thread).  With
+ * COLI_INJECT_WITHHOLD_STAGE the next coli_moe_layer / coli_moe_ffn call's
+ * gate/up kernel never fills one staged tile: its consumers' bounded wait
+ * (about one second) runs out, the kernel winds down without hanging or
+ * faulting, and the status word reads COLI_ERR_TIMEOUT; the output of that
+ * call is undefined and the context stays usable.  0 switches it off.
+ * Returns COLI_ERR_INVALID_ARG for an unknown code. */
+#define COLI_INJECT_WITHHOLD_STAGE 1
+coli_status coli_moe_debug_inject(int32_t what);
 
 /* Static English text for a status code (never NULL). */
 const char *coli_status_string(coli_status s);

@@ -29,12 +29,14 @@ COLI_ERR_UNSUPPORTED = 7
 COLI_ERR_BAD_INDEX = 8
 COLI_ERR_RANGE = 9
 COLI_OUT_F32 = 0
-COLI_WS_LOGITS_OFFSET = 4096  # router logits left in the workspace by coli_moe_layer
+COLI_WS_LOGITS_OFFSET = 16384  # router logits left in the workspace by coli_moe_layer
+COLI_WS_HEADER_BYTES = 16384
 COLI_OUT_BF16 = 1
 
 EXPORTS = ("coli_moe_create", "coli_moe_destroy", "coli_moe_workspace_size",
            "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union", "coli_moe_ffn",
-           "coli_moe_layer", "coli_moe_get_status", "coli_moe_profile_enable",
+           "coli_moe_layer", "coli_moe_get_status", "coli_moe_debug_inject",
+           "coli_moe_profile_enable",
            "coli_moe_profile_read", "coli_status_string")
 
 
@@ -81,6 +83,8 @@ def _load():
     L.coli_moe_layer.restype = ctypes.c_int
     L.coli_moe_get_status.argtypes = [P, P]
     L.coli_moe_get_status.restype = ctypes.c_int
+    L.coli_moe_debug_inject.argtypes = [i32]
+    L.coli_moe_debug_inject.restype = ctypes.c_int
     L.coli_moe_profile_enable.argtypes = [i32]
     L.coli_moe_profile_enable.restype = ctypes.c_int
     L.coli_moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32)]
@@ -161,6 +165,13 @@ def coli_moe_workspace_clear(ws, stream=None, raise_on_error=True):
 
 def coli_moe_get_status(ws, stream=None):
     return lib.coli_moe_get_status(_ptr(ws), _stream(stream))
+
+
+COLI_INJECT_WITHHOLD_STAGE = 1
+
+
+def coli_moe_debug_inject(what: int):
+    return lib.coli_moe_debug_inject(int(what))
 
 
 def coli_moe_profile_enable(enable: bool):

@@ -83,6 +83,7 @@ coli::FfnArgs make_args(const coli_moe* h, int32_t T, const void* x, const float
     a.out = out;
     a.out_bf16 = od == COLI_OUT_BF16;
     a.status = at<int>(ws, 0);
+    a.withhold_item = -1;
     return a;
 }
 
@@ -93,6 +94,7 @@ struct ProfileState {
     int open_call = -1;               // index of the call being recorded
 };
 ProfileState g_prof;
+int g_withhold_item = -1;
 
 void profile_begin_call(cudaStream_t st) {
     if (!g_prof.enabled) return;
@@ -114,6 +116,12 @@ void profile_end_call() { g_prof.open_call = -1; }
 }  // namespace
 
 namespace coli {
+int take_withhold_item() {
+    const int v = g_withhold_item;
+    g_withhold_item = -1;
+    return v;
+}
+
 cudaEvent_t profile_event(int i) {
     if (!g_prof.enabled || g_prof.open_call < 0 || i < 0 || i > 4) return nullptr;
     return g_prof.events[(size_t)g_prof.open_call * 5 + i];
@@ -121,6 +129,18 @@ cudaEvent_t profile_event(int i) {
 }  // namespace coli
 
 extern "C" {
+
+coli_status coli_moe_debug_inject(int32_t what) {
+    if (what == 0) {
+        g_withhold_item = -1;
+        return COLI_OK;
+    }
+    if (what == COLI_INJECT_WITHHOLD_STAGE) {
+        g_withhold_item = 0;  // the first item of CTA 0: a shared-expert gate/up tile
+        return COLI_OK;
+    }
+    return COLI_ERR_INVALID_ARG;
+}
 
 coli_status coli_moe_profile_enable(int32_t enable) {
     g_prof.enabled = enable != 0;
@@ -159,6 +179,8 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (d->top_k < 1 || d->top_k > d->n_routed || d->top_k > coli::kMaxTopK) return COLI_ERR_SHAPE;
     if (d->n_shared < 0 || d->n_shared > coli::kMaxShared) return COLI_ERR_SHAPE;
     if (d->prefill_min_tokens < 0) return COLI_ERR_INVALID_ARG;
+    if (d->hidden > 12288 || d->inter > 12288 || !coli::stream_shapes_fit(d->hidden, d->inter))
+        return COLI_ERR_SHAPE;
     const int n = d->n_routed + d->n_shared;
     for (int e = 0; e < n; ++e) {
         const coli_expert& x = d->experts[e];
@@ -253,7 +275,7 @@ coli_status coli_moe_union(int32_t T, int32_t E, int32_t k, const int32_t* topk_
     if (ws && (ws_bytes < coli::kHeaderBytes || !aligned(ws, 256))) return COLI_ERR_WORKSPACE;
     // T == 0 still writes empty lists (counts 0, offsets 0, no active experts).
     return from_cuda(coli::launch_union(T, E, k, topk_idx, counts, offsets, pairs, active,
-                                        n_active, ws ? static_cast<int*>(ws) : nullptr,
+                                        n_active, nullptr, ws ? static_cast<int*>(ws) : nullptr,
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -273,7 +295,8 @@ coli_status coli_moe_ffn(const coli_moe* h, int32_t T, const void* x_bf16, const
                                 out, out_dtype, ws);
     profile_begin_call(st);
     cudaError_t err = coli::launch_inverse_pairs(T * h->k, pairs, a.inv, a.status, st);
-    if (err == cudaSuccess) err = coli::launch_ffn_gemv(a, h->num_sms, st);
+    if (err == cudaSuccess) err = coli::launch_permute_x(T, h->H, a.x, a.xp, st);
+    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
     profile_end_call();
     return from_cuda(err);
 }
@@ -302,19 +325,29 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
     }
     int* idx = topk_idx_out ? topk_idx_out : at<int>(ws, L.idx);
     float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
-    if (err == cudaSuccess) err = coli::launch_route(T, h->E, h->k, lg, idx, w, st);
     int* counts = at<int>(ws, L.counts);
     int* offsets = at<int>(ws, L.offsets);
     int* pairs = at<int>(ws, L.pairs);
     int* active = at<int>(ws, L.active);
     int* n_active = at<int>(ws, L.n_active);
-    if (err == cudaSuccess)
-        err = coli::launch_union(T, h->E, h->k, idx, counts, offsets, pairs, active, n_active,
-                                 at<int>(ws, 0), st);
     coli::FfnArgs a = make_args(h, T, x_bf16, w, offsets, pairs, active, n_active, residual, out,
                                 out_dtype, ws);
-    if (err == cudaSuccess) err = coli::launch_inverse_pairs(T * h->k, pairs, a.inv, a.status, st);
-    if (err == cudaSuccess) err = coli::launch_ffn_gemv(a, h->num_sms, st);
+    if (T <= coli::kSmallT) {
+        // one launch: route, union, inverse map and activation permutation
+        coli::PrepArgs p;
+        p.T = T; p.E = h->E; p.k = h->k; p.H = h->H;
+        p.logits = lg; p.idx = idx; p.w = w; p.counts = counts; p.offsets = offsets;
+        p.pairs = pairs; p.active = active; p.n_active = n_active; p.inv = a.inv;
+        p.x = x; p.xp = a.xp; p.status = a.status;
+        if (err == cudaSuccess) err = coli::launch_prep_small(p, st);
+    } else {
+        if (err == cudaSuccess) err = coli::launch_route(T, h->E, h->k, lg, idx, w, st);
+        if (err == cudaSuccess)
+            err = coli::launch_union(T, h->E, h->k, idx, counts, offsets, pairs, active, n_active,
+                                     a.inv, a.status, st);
+        if (err == cudaSuccess) err = coli::launch_permute_x(T, h->H, x, a.xp, st);
+    }
+    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
     profile_end_call();
     return from_cuda(err);
 }

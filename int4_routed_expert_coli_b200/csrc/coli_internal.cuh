@@ -15,7 +15,9 @@ constexpr int kGroup = 64;        // codes per bf16 scale (gs64)
 constexpr int kMaxExperts = 1024; // E limit (one union thread per expert)
 constexpr int kMaxTopK = 32;      // k limit (one route lane per slot)
 constexpr int kMaxShared = 4;
-constexpr size_t kHeaderBytes = 4096; // status word + counters at the start of ws
+constexpr size_t kHeaderBytes = 16384; // status word + tile counters at the start of ws
+constexpr size_t kCounterOffset = 256; // int counters, one per 16-row output tile
+constexpr int kSmallT = 64;            // calls with T <= kSmallT use the fused prep kernel
 
 // Device status codes live in the first word of the workspace.
 struct WsHeader {
@@ -95,12 +97,33 @@ struct FfnArgs {
     void* out;                 // [T][H]
     int out_bf16;
     int* status;
+    int withhold_item;         // test hook: producer never fills this item (-1 = off)
+};
+
+// Arguments of the fused small-batch preparation kernel.
+struct PrepArgs {
+    int T, E, k, H;
+    const float* logits;      // [T][E]
+    int* idx;                 // [T][k] out
+    float* w;                 // [T][k] out
+    int* counts;              // [E]
+    int* offsets;             // [E+1]
+    int* pairs;               // [T*k]
+    int* active;              // [E]
+    int* n_active;            // [1]
+    int* inv;                 // [T*k]
+    const __nv_bfloat16* x;   // [T][H]
+    __nv_bfloat16* xp;        // [T][H] permuted
+    int* status;
 };
 
 // ---- timing diagnostics (coli_moe_profile_*) ------------------------------
 // Returns the event to record at phase boundary `i` (0..4) of the current
 // call, or nullptr when profiling is off.
 cudaEvent_t profile_event(int i);
+// Test hook (coli_moe_debug_inject): item index the next FFN launch's producer
+// withholds, or -1.  Reading it clears it.
+int take_withhold_item();
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----------
 cudaError_t launch_router_logits(int T, int E, int H, const __nv_bfloat16* x, const float* wr,
@@ -108,9 +131,14 @@ cudaError_t launch_router_logits(int T, int E, int H, const __nv_bfloat16* x, co
 cudaError_t launch_route(int T, int E, int k, const float* logits, int* idx, float* w,
                          cudaStream_t st);
 cudaError_t launch_union(int T, int E, int k, const int* idx, int* counts, int* offsets,
-                         int* pairs, int* active, int* n_active, int* status, cudaStream_t st);
-cudaError_t launch_ffn_gemv(const FfnArgs& a, int num_sms, cudaStream_t st);
+                         int* pairs, int* active, int* n_active, int* inv, int* status,
+                         cudaStream_t st);
+cudaError_t launch_prep_small(const PrepArgs& p, cudaStream_t st);
+cudaError_t launch_ffn_stream(const FfnArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_permute_x(int T, int H, const __nv_bfloat16* x, __nv_bfloat16* xp,
+                             cudaStream_t st);
 cudaError_t launch_inverse_pairs(int P, const int* pairs, int* inv, int* status, cudaStream_t st);
+bool stream_shapes_fit(int H, int I);  // the streaming FFN's 2 stages fit in shared memory
 
 // ---- device helpers --------------------------------------------------------
 __device__ __forceinline__ void report(int* status, int code) {

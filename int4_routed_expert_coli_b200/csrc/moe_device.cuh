@@ -1,0 +1,230 @@
+// Device bodies of the routing and batch-union steps, shared by their
+// stand-alone kernels and by the fused small-batch preparation kernel.
+#pragma once
+
+#include "coli_internal.cuh"
+
+namespace coli {
+
+// ---------------------------------------------------------------------------
+// Routing: the router picks k of the E routed experts for every token
+// ("zhichai.net/topic/178503686", MoE-sparsity section).  Exact and
+// deterministic: each logit becomes a 64-bit key that orders by value
+// descending (NaN lowest, -0 == +0) and then by expert index ascending; k
+// rounds of a warp-wide max pick the winners in slot order.
+
+__device__ __forceinline__ uint64_t rank_key(float v, int e) {
+    uint32_t k32;
+    if (isnan(v)) {
+        k32 = 0u;
+    } else {
+        const uint32_t b = __float_as_uint(v + 0.0f);  // -0 + 0 = +0
+        k32 = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    }
+    return ((uint64_t)k32 << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t other = __shfl_xor_sync(0xffffffffu, v, o);
+        v = other > v ? other : v;
+    }
+    return v;
+}
+
+// One warp routes one token row.  NV = logits per lane (E <= 32 * NV).
+// Weights: w_j = exp(l_j - m) / sum_i exp(l_i - m) over the chosen set in
+// double, rounded to fp32 once; +inf entries share the weight when m = +inf;
+// 1/k each when m is -inf or NaN; NaN entries contribute 0.
+template <int NV>
+__device__ __forceinline__ void route_row(const float* __restrict__ row, int E, int k, int lane,
+                                          int* __restrict__ idx_out, float* __restrict__ w_out) {
+    uint64_t key[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = e < E ? rank_key(row[e], e) : 0ull;  // padding never wins (k <= E)
+    }
+    int my_idx = -1;  // lane j keeps the j-th winner
+    for (int j = 0; j < k; ++j) {
+        uint64_t best = 0ull;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+        best = warp_max_u64(best);
+        const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
+        if ((e & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+                if (i == (e >> 5)) key[i] = 0ull;
+        }
+        if (lane == j) my_idx = e;
+    }
+    const float v = (lane < k) ? row[my_idx] : 0.f;
+    const float m = __shfl_sync(0xffffffffu, v, 0);
+    double wj;
+    if (isinf(m) && m > 0.f) {
+        const bool pinf = lane < k && isinf(v) && v > 0.f;
+        const unsigned inf_mask = __ballot_sync(0xffffffffu, pinf);
+        wj = pinf ? 1.0 / (double)__popc(inf_mask) : 0.0;
+    } else if (isnan(m) || (isinf(m) && m < 0.f)) {
+        wj = 1.0 / (double)k;
+    } else {
+        const double ej = (lane < k && !isnan(v)) ? exp((double)v - (double)m) : 0.0;
+        double z = ej;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        wj = ej / z;
+    }
+    if (lane < k) {
+        idx_out[lane] = my_idx;
+        w_out[lane] = (float)wj;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Batch-union: all positions routed to one expert are listed together so the
+// expert is read once for all of them ("yunpan.plus/t/30351-1-1",
+// capability two, batch-union bullet).  A stable counting sort of the P
+// pairs by expert in one CTA of kUnionThreads threads: per-warp histograms
+// (one leader per distinct expert in a 32-pair slice), a scan over
+// (expert, warp), then a second pass writing each pair at
+// base + rank-among-equal-keys.  No position comes from an atomic ticket.
+
+constexpr int kUnionThreads = 1024;
+constexpr int kUnionWarps = kUnionThreads / 32;
+
+__host__ __device__ constexpr size_t union_smem_bytes(int E) {
+    return sizeof(int) * (size_t)kUnionWarps * E;
+}
+
+// Exclusive scan of one int per thread over a block of <= 1024 threads.
+// `tmp` holds 32 ints.  Returns the prefix; *total gets the block sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        int s = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += n;
+        }
+        tmp[lane] = s;
+    }
+    __syncthreads();
+    const int base = warp > 0 ? tmp[warp - 1] : 0;
+    *total = tmp[(blockDim.x >> 5) - 1];
+    __syncthreads();
+    return base + incl - v;
+}
+
+// Must be called by all kUnionThreads threads of the block.  `hist` is
+// union_smem_bytes(E) of shared memory.  `inv` (nullable) receives, for each
+// pair p, its position in `pairs` (-1 for a dropped pair).
+__device__ __forceinline__ void union_block(int P, int E, const int* __restrict__ idx,
+                                            int* __restrict__ counts, int* __restrict__ offsets,
+                                            int* __restrict__ pairs, int* __restrict__ active,
+                                            int* __restrict__ n_active, int* __restrict__ inv,
+                                            int* status, int* hist, int* scan_tmp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < kUnionWarps * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+
+    const int chunk = ((P + kUnionWarps - 1) / kUnionWarps + 31) / 32 * 32;
+    const int p_begin = warp * chunk;
+    const int p_end = min(P, p_begin + chunk);
+    int* my_hist = hist + warp * E;
+
+    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+        const int p = p0 + lane;
+        int e = p < p_end ? idx[p] : -1;
+        if (p < p_end && (e < 0 || e >= E)) {
+            report(status, COLI_ERR_BAD_INDEX);
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (peers & lt_mask) == 0) my_hist[e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+
+    int cnt = 0;
+    const int e_self = threadIdx.x;
+    if (e_self < E) {
+        for (int w = 0; w < kUnionWarps; ++w) {
+            const int c = hist[w * E + e_self];
+            hist[w * E + e_self] = cnt;
+            cnt += c;
+        }
+    }
+    int total;
+    const int off = block_exclusive_scan(e_self < E ? cnt : 0, scan_tmp, &total);
+    int act_total;
+    const int act_pos =
+        block_exclusive_scan((e_self < E && cnt > 0) ? 1 : 0, scan_tmp, &act_total);
+    if (e_self < E) {
+        counts[e_self] = cnt;
+        offsets[e_self] = off;
+        for (int w = 0; w < kUnionWarps; ++w) hist[w * E + e_self] += off;
+        if (cnt > 0) active[act_pos] = e_self;
+    }
+    if (threadIdx.x == 0) {
+        offsets[E] = total;
+        *n_active = act_total;
+    }
+    for (int e = act_total + threadIdx.x; e < E; e += blockDim.x) active[e] = -1;
+    __syncthreads();
+
+    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+        const int p = p0 + lane;
+        int e = p < p_end ? idx[p] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0) {
+            const int pos = my_hist[e] + __popc(peers & lt_mask);
+            pairs[pos] = p;
+            if (inv) inv[p] = pos;
+        } else if (p < p_end && inv) {
+            inv[p] = -1;
+        }
+        __syncwarp();
+        if (e >= 0 && (peers & lt_mask) == 0) my_hist[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fragment order of a 64-element scale group (see gemv.cu): position of
+// element j of the group in the permuted activation layout.
+__host__ __device__ __forceinline__ int perm64(int j) {
+    const int c = j >> 4, jj = j & 15;
+    const int m = ((jj >> 3) << 1) + ((jj & 3) >> 1);
+    const int e = (jj & 7) >> 2;
+    const int odd = jj & 1;
+    return c * 16 + 4 * m + 2 * odd + e;
+}
+
+// Permute one 16-element slice of a bf16 row into fragment order.
+__device__ __forceinline__ void permute_slice16(const uint16_t* src, uint16_t* dst) {
+    const uint4 in0 = *reinterpret_cast<const uint4*>(src);
+    const uint4 in1 = *reinterpret_cast<const uint4*>(src + 8);
+    uint16_t v[16], o[16];
+    *reinterpret_cast<uint4*>(&v[0]) = in0;
+    *reinterpret_cast<uint4*>(&v[8]) = in1;
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) o[perm64(jj) & 15] = v[jj];
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(&o[0]);
+    *reinterpret_cast<uint4*>(dst + 8) = *reinterpret_cast<uint4*>(&o[8]);
+}
+
+}  // namespace coli

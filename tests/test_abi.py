@@ -35,6 +35,16 @@ def test_library_exports_every_declared_symbol():
                                                       "coli_status_string"), n
 
 
+def test_header_constants_match_binding():
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    src = open(HEADER).read()
+    for name in ("COLI_WS_LOGITS_OFFSET", "COLI_WS_HEADER_BYTES", "COLI_INJECT_WITHHOLD_STAGE"):
+        m = re.search(r"#define\s+" + name + r"\s+(\d+)", src)
+        assert m and int(m.group(1)) == getattr(c, name), name
+    for name, val in re.findall(r"\b(COLI_(?:OK|ERR_\w+|OUT_\w+))\s*=\s*(\d+)", src):
+        assert getattr(c, name) == int(val), name
+
+
 def test_status_strings():
     from int4_routed_expert_coli_b200 import coli_moe as c
     for s in range(10):
@@ -81,6 +91,9 @@ def test_host_validation_without_gpu():
     assert L.coli_moe_ffn(None, 1, None, None, None, None, None, None, None, None, None, 0,
                           None, 0, None) == c.COLI_ERR_INVALID_ARG
     assert L.coli_moe_workspace_clear(None, 0, None) == c.COLI_ERR_INVALID_ARG
+    # fault injection: unknown codes are refused, 0 switches it off
+    assert L.coli_moe_debug_inject(12345) == c.COLI_ERR_INVALID_ARG
+    assert L.coli_moe_debug_inject(0) == c.COLI_OK
 
 
 def test_binding_refuses_host_tensors():

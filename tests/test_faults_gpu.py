@@ -1,0 +1,64 @@
+"""Failure detection on the GPU without faulting it: a staged tile that is
+never filled makes the consumers' bounded wait (about one second) run out;
+the kernel winds down, the status word reads COLI_ERR_TIMEOUT, and the
+context stays usable for the next call."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import assert_close, reference_layer, requires_gpu
+from int4_routed_expert_coli_b200 import synth
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+
+def test_withheld_stage_times_out_and_context_survives():
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    H, I, E, k, T = 256, 128, 16, 2, 4
+    bank = synth.make_expert_bank(H, I, E + 1, seed=21, device="cuda")
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=1)
+    x = synth.make_activations(T, H, seed=22, device="cuda")
+    lg = synth.make_logits_normal(T, E, seed=23, device="cuda")
+    ws = layer.workspace(T)
+    assert c.coli_moe_debug_inject(c.COLI_INJECT_WITHHOLD_STAGE) == c.COLI_OK
+    try:
+        layer.layer(x, logits=lg, ws=ws)
+    finally:
+        c.coli_moe_debug_inject(0)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_TIMEOUT
+    # the context is still usable and the next call is correct
+    c.coli_moe_workspace_clear(ws)
+    out = layer.layer(x, logits=lg, ws=ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_OK
+    ref, _, _ = reference_layer(bank, E, k, 1, x, lg)
+    assert_close(out.cpu().numpy(), ref, "after timeout")
+
+
+def test_bad_union_input_reports_not_faults():
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    H, I, E, k, T = 256, 128, 16, 2, 4
+    bank = synth.make_expert_bank(H, I, E + 1, seed=24, device="cuda")
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=1)
+    x = synth.make_activations(T, H, seed=25, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), 0.5, device="cuda")
+    counts = torch.zeros(E, **i32)
+    offsets = torch.zeros(E + 1, **i32)
+    offsets[1:] = 8
+    offsets[0] = 0
+    counts[0] = 8
+    pairs = torch.arange(T * k, **i32)
+    pairs[3] = 10 ** 6                      # out of range pair id
+    active = torch.full((E,), -1, **i32)
+    active[0] = 0
+    na = torch.tensor([1], **i32)
+    ws = layer.workspace(T)
+    out = torch.empty(T, H, device="cuda")
+    c.coli_moe_ffn(layer.handle, T, x, w, counts, offsets, pairs, active, na, None, out,
+                   c.COLI_OUT_F32, ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX
+    na.fill_(5000)                          # n_active beyond E
+    c.coli_moe_workspace_clear(ws)
+    c.coli_moe_ffn(layer.handle, T, x, w, counts, offsets, pairs, active, na, None, out,
+                   c.COLI_OUT_F32, ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX

@@ -50,7 +50,8 @@ def test_tiny_layer_with_router_weight(tiny):
     x = synth.make_activations(4, 256, seed=0, device="cuda")
     wr = synth.make_router_weight(16, 256, seed=0, device="cuda")
     out, idx, w, ws = _layer(layer, x, router_w=wr)
-    lg_gpu = ws[4096:4096 + 4 * 16 * 4].view(torch.float32).view(4, 16).cpu().numpy()
+    off = c.COLI_WS_LOGITS_OFFSET
+    lg_gpu = ws[off:off + 4 * 16 * 4].view(torch.float32).view(4, 16).cpu().numpy()
     lg_ref = oracle.router_logits(bits(x), wr.cpu().numpy())
     assert np.linalg.norm(lg_gpu - lg_ref) / np.linalg.norm(lg_ref) <= 1e-5
     ref, ri, rw = reference_layer(bank, 16, 2, 1, x, lg_gpu)

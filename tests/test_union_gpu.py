@@ -60,7 +60,7 @@ def test_union_all_to_one_expert_and_empty():
 
 def test_union_bad_index_sets_status():
     from int4_routed_expert_coli_b200 import coli_moe as c
-    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(c.COLI_WS_HEADER_BYTES, dtype=torch.uint8, device="cuda")
     idx = np.array([[0, 3], [300, 1]], np.int32)
     got = _run(idx, 16, ws=ws)
     assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX
