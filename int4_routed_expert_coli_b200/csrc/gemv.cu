@@ -32,9 +32,8 @@
 // hp), so every dot product is unchanged.  One 64-code scale group is one
 // 8-byte slice per lane of a quad, i.e. exactly four MMAs.
 //
-// Combine.  The down kernel writes each expert's rows of y; the CTA that
-// finishes the last expert of a 16-row output tile (a counter per tile,
-// last arriver does the work, counter reset to zero) forms
+// Combine.  The down kernel writes each expert's rows of y (fp32); a small
+// kernel chained to it by programmatic dependent launch forms
 //   out[t][m] = sum_j w[t][j] y[(t,j)][m] (j ascending) + y_shared[t][m]
 //               (+ residual[t][m])
 // in fp32, in that fixed order, so the result does not depend on timing.
@@ -206,11 +205,16 @@ __device__ __forceinline__ void item_sources(const DevExpert& ex, int tile, cons
     }
 }
 
-// Combine one 16-row output tile for every token (fixed order, fp32).
-__device__ void combine_tile(const FfnArgs& a, int m0, int tid, int nthreads) {
+// out[t][m] = sum_j w[t][j] y[inv[t*k+j]][m] (j ascending) + sum_shared y
+// (+ residual), fp32 in that fixed order.  One thread per output element.
+// Launched as a programmatic dependent of the down kernel.
+__global__ void combine_kernel(const FfnArgs a) {
+    pdl_wait();
     const int H = a.H, k = a.k, P = a.T * a.k;
-    for (int idx = tid; idx < a.T * 16; idx += nthreads) {
-        const int t = idx >> 4, m = m0 + (idx & 15);
+    const int64_t n = (int64_t)a.T * H;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(idx / H), m = (int)(idx % H);
         float acc = 0.f;
         for (int j = 0; j < k; ++j) {
             const int s = a.inv[t * k + j];
@@ -218,10 +222,9 @@ __device__ void combine_tile(const FfnArgs& a, int m0, int tid, int nthreads) {
                 report(a.status, COLI_ERR_BAD_INDEX);
                 continue;
             }
-            acc = fmaf(a.topk_w[t * k + j], __ldcg(a.y + (int64_t)s * H + m), acc);
+            acc = fmaf(a.topk_w[t * k + j], a.y[(int64_t)s * H + m], acc);
         }
-        for (int sh = 0; sh < a.n_shared; ++sh)
-            acc += __ldcg(a.y + (int64_t)(P + sh * a.T + t) * H + m);
+        for (int sh = 0; sh < a.n_shared; ++sh) acc += a.y[(int64_t)(P + sh * a.T + t) * H + m];
         const int64_t o = (int64_t)t * H + m;
         if (a.out_bf16) {
             if (a.residual)
@@ -236,7 +239,7 @@ __device__ void combine_tile(const FfnArgs& a, int m0, int tid, int nthreads) {
 
 // ---------------------------------------------------------------------------
 // The streaming FFN kernel.  kGU: gate/up + SwiGLU (bf16 MMA, writes hp);
-// otherwise down + combine (fp16 MMA, writes y then out).  NT = N-tiles of 8
+// otherwise down (fp16 MMA, writes y).  NT = N-tiles of 8
 // tokens per pass.
 template <int NT, bool kGU>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -244,7 +247,7 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
-    volatile int* flags = reinterpret_cast<volatile int*>(smem + 256);  // [0] abort, [1] last
+    volatile int* flags = reinterpret_cast<volatile int*>(smem + 256);  // [0] abort
     float* red = reinterpret_cast<float*>(smem + kFixedSmem);            // [8][NT][4][32]
     uint8_t* stage0 = smem + kFixedSmem + kConsumerWarps * NT * 4 * 32 * 4;
 
@@ -255,7 +258,6 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
             mbar_init(&empty[s], kConsumerWarps);
         }
         flags[0] = 0;
-        flags[1] = 0;
         fence_barrier_init();
     }
     __syncthreads();
@@ -323,7 +325,6 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
     const int r = lane >> 2, c = lane & 3;
     const int g_lo = (g.G * warp) / kConsumerWarps, g_hi = (g.G * (warp + 1)) / kConsumerWarps;
     const int tid = threadIdx.x;
-    int* tile_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(a.status) + kCounterOffset);
 
     int j = 0;
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
@@ -455,24 +456,6 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
         // release the stage (all lanes' shared-memory reads are done)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
-
-        if constexpr (!kGU) {
-            // y rows of this item are written; the last expert of the tile combines
-            __threadfence();
-            named_barrier(1, kConsumers);
-            if (tid == 0) {
-                const int old = atomicAdd(&tile_cnt[tile], 1);
-                flags[1] = (old == n_slots - 1) ? 1 : 0;
-            }
-            named_barrier(1, kConsumers);
-            if (flags[0]) goto done;
-            if (flags[1]) {
-                __threadfence();
-                combine_tile(a, tile * 16, tid, kConsumers);
-                if (tid == 0) tile_cnt[tile] = 0;
-            }
-            named_barrier(1, kConsumers);
-        }
     }
 done:
     return;
@@ -532,6 +515,21 @@ cudaError_t launch_stream(const FfnArgs& a, const Geo& g, int num_sms, cudaStrea
     return cudaLaunchKernelEx(&cfg, stream_ffn_kernel<NT, kGU>, a, g, stages);
 }
 
+cudaError_t launch_combine(const FfnArgs& a, int num_sms, cudaStream_t st) {
+    const int64_t n = (int64_t)a.T * a.H;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 8));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel, a);
+}
+
 template <int NT>
 cudaError_t launch_pair(const FfnArgs& a_in, int num_sms, cudaStream_t st) {
     FfnArgs a = a_in;
@@ -542,7 +540,9 @@ cudaError_t launch_pair(const FfnArgs& a_in, int num_sms, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     mark(2, st);
     err = launch_stream<NT, false>(a, make_geo(a.I, a.H / 16), num_sms, st);
+    if (err != cudaSuccess) return err;
     mark(3, st);
+    err = launch_combine(a, num_sms, st);
     mark(4, st);
     return err;
 }
