@@ -8,13 +8,19 @@
 #include <vector>
 
 #include "coli_internal.cuh"
+#include "prefill.cuh"
 
 struct coli_moe {
     int device;
     int H, I, E, k, n_shared, prefill_min;
     int num_sms;
     coli::DevExpert* d_experts;  // device table, E + n_shared entries
+    CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)
 };
+
+// Average routed tokens per expert (T*k/E) at or above which a call runs the
+// tensor-core grouped GEMM instead of the streaming dequant-GEMV.
+constexpr int kDefaultPrefillMin = 32;
 
 namespace {
 
@@ -75,7 +81,8 @@ coli::FfnArgs make_args(const coli_moe* h, int32_t T, const void* x, const float
     a.n_active = n_active;
     a.topk_w = w;
     a.x = static_cast<const __nv_bfloat16*>(x);
-    a.xp = at<__nv_bfloat16>(ws, L.xp);
+    a.xp = at<__half>(ws, L.xp);
+    a.corr = at<float>(ws, L.corr);
     a.inv = at<int>(ws, L.inv);
     a.hp = at<__half>(ws, L.hp);
     a.y = at<float>(ws, L.y);
@@ -112,6 +119,30 @@ void profile_begin_call(cudaStream_t st) {
 }
 
 void profile_end_call() { g_prof.open_call = -1; }
+
+// True when a call with T tokens runs the tensor-core grouped GEMM.
+bool use_prefill(const coli_moe* h, int64_t T) {
+    return h->d_wmaps != nullptr && T * h->k >= (int64_t)h->prefill_min * h->E;
+}
+
+// The FFN of a call whose union lists (and inverse map) are ready: tensor-core
+// grouped GEMM for prefill-sized batches, streaming GEMV otherwise.
+// `x_prepared`: the fused prep kernel already built the GEMV operand of x.
+cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* ws,
+                    cudaStream_t st, bool x_prepared) {
+    const coli::WsLayout L = layout_for(h, T);
+    cudaError_t err = cudaSuccess;
+    if (use_prefill(h, T)) {
+        err = coli::launch_prefill(a, h->d_wmaps, at<__half>(ws, L.xg), at<int>(ws, L.ntile),
+                                   h->num_sms, st);
+        if (err == cudaSuccess) err = coli::launch_combine(a, h->num_sms, st);
+        coli::profile_mark(4, st);
+        return err;
+    }
+    if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
+    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
+    return err;
+}
 
 }  // namespace
 
@@ -209,6 +240,8 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     h->prefill_min = d->prefill_min_tokens;
     h->num_sms = sms;
     h->d_experts = nullptr;
+    h->d_wmaps = nullptr;
+    if (h->prefill_min == 0) h->prefill_min = kDefaultPrefillMin;
     coli::DevExpert* host = static_cast<coli::DevExpert*>(std::malloc(sizeof(coli::DevExpert) * n));
     if (!host) {
         delete h;
@@ -225,9 +258,12 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     cudaError_t err = cudaMalloc(&h->d_experts, sizeof(coli::DevExpert) * n);
     if (err == cudaSuccess)
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
+    if (err == cudaSuccess && coli::prefill_available())
+        err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
     std::free(host);
     if (err != cudaSuccess) {
         if (h->d_experts) cudaFree(h->d_experts);
+        if (h->d_wmaps) cudaFree(h->d_wmaps);
         delete h;
         return COLI_ERR_CUDA;
     }
@@ -238,6 +274,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
 void coli_moe_destroy(coli_moe* h) {
     if (!h) return;
     cudaFree(h->d_experts);
+    if (h->d_wmaps) cudaFree(h->d_wmaps);
     delete h;
 }
 
@@ -295,8 +332,7 @@ coli_status coli_moe_ffn(const coli_moe* h, int32_t T, const void* x_bf16, const
                                 out, out_dtype, ws);
     profile_begin_call(st);
     cudaError_t err = coli::launch_inverse_pairs(T * h->k, pairs, a.inv, a.status, st);
-    if (err == cudaSuccess) err = coli::launch_permute_x(T, h->H, a.x, a.xp, st);
-    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
+    if (err == cudaSuccess) err = run_ffn(h, T, a, ws, st, false);
     profile_end_call();
     return from_cuda(err);
 }
@@ -332,22 +368,22 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
     int* n_active = at<int>(ws, L.n_active);
     coli::FfnArgs a = make_args(h, T, x_bf16, w, offsets, pairs, active, n_active, residual, out,
                                 out_dtype, ws);
-    if (T <= coli::kSmallT) {
-        // one launch: route, union, inverse map and activation permutation
+    const bool prefill = use_prefill(h, T);
+    if (T <= coli::kSmallT && !prefill) {
+        // one launch: route, union, inverse map and activation preparation
         coli::PrepArgs p;
         p.T = T; p.E = h->E; p.k = h->k; p.H = h->H;
         p.logits = lg; p.idx = idx; p.w = w; p.counts = counts; p.offsets = offsets;
         p.pairs = pairs; p.active = active; p.n_active = n_active; p.inv = a.inv;
-        p.x = x; p.xp = a.xp; p.status = a.status;
+        p.x = x; p.xp = a.xp; p.corr = a.corr; p.status = a.status;
         if (err == cudaSuccess) err = coli::launch_prep_small(p, st);
     } else {
         if (err == cudaSuccess) err = coli::launch_route(T, h->E, h->k, lg, idx, w, st);
         if (err == cudaSuccess)
             err = coli::launch_union(T, h->E, h->k, idx, counts, offsets, pairs, active, n_active,
                                      a.inv, a.status, st);
-        if (err == cudaSuccess) err = coli::launch_permute_x(T, h->H, x, a.xp, st);
     }
-    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
+    if (err == cudaSuccess) err = run_ffn(h, T, a, ws, st, T <= coli::kSmallT && !prefill);
     profile_end_call();
     return from_cuda(err);
 }

@@ -46,9 +46,12 @@ struct WsLayout {
     size_t active;   // [E] i32
     size_t n_active; // [1] i32
     size_t inv;      // [T*k] i32: position of pair p in `pairs`
-    size_t xp;       // [T][H] bf16, fragment-permuted copy of x
+    size_t xp;       // [T][H] f16, fragment-permuted operand copy of x
+    size_t corr;     // [T][H/64] f32, unpack-offset sums of each x group
     size_t hp;       // [S][I] f16, fragment-permuted SwiGLU output, S = T*k + T*n_shared
     size_t y;        // [S][H] f32, per-(pair) expert outputs
+    size_t xg;       // [T*k + T][H] f16, expert-sorted activations (tensor-core path)
+    size_t ntile;    // [E + n_shared + 1] i32, token-tile prefix (tensor-core path)
     size_t total;
 };
 
@@ -73,8 +76,11 @@ inline WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int n_shared) {
     L.n_active = take(sizeof(int));
     L.inv = take(sizeof(int) * P);
     L.xp = take(sizeof(uint16_t) * T * H);
+    L.corr = take(sizeof(float) * T * (H / 64));
     L.hp = take(sizeof(uint16_t) * S * I);
     L.y = take(sizeof(float) * S * H);
+    L.xg = take(sizeof(uint16_t) * (P + T) * H);
+    L.ntile = take(sizeof(int) * (E + n_shared + 2));
     L.total = o;
     return L;
 }
@@ -89,7 +95,8 @@ struct FfnArgs {
     const int* n_active;       // [1]
     const float* topk_w;       // [T][k]
     const __nv_bfloat16* x;    // [T][H]
-    __nv_bfloat16* xp;         // [T][H] permuted
+    __half* xp;                // [T][H] operand copy of x (fragment order)
+    float* corr;               // [T][H/64] unpack-offset sums
     int* inv;                  // [T*k]
     __half* hp;                // [S][I] permuted
     float* y;                  // [S][H]
@@ -113,7 +120,8 @@ struct PrepArgs {
     int* n_active;            // [1]
     int* inv;                 // [T*k]
     const __nv_bfloat16* x;   // [T][H]
-    __nv_bfloat16* xp;        // [T][H] permuted
+    __half* xp;               // [T][H] operand copy of x
+    float* corr;              // [T][H/64]
     int* status;
 };
 
@@ -121,6 +129,9 @@ struct PrepArgs {
 // Returns the event to record at phase boundary `i` (0..4) of the current
 // call, or nullptr when profiling is off.
 cudaEvent_t profile_event(int i);
+inline void profile_mark(int i, cudaStream_t st) {
+    if (cudaEvent_t ev = profile_event(i)) cudaEventRecord(ev, st);
+}
 // Test hook (coli_moe_debug_inject): item index the next FFN launch's producer
 // withholds, or -1.  Reading it clears it.
 int take_withhold_item();
@@ -135,10 +146,11 @@ cudaError_t launch_union(int T, int E, int k, const int* idx, int* counts, int* 
                          cudaStream_t st);
 cudaError_t launch_prep_small(const PrepArgs& p, cudaStream_t st);
 cudaError_t launch_ffn_stream(const FfnArgs& a, int num_sms, cudaStream_t st);
-cudaError_t launch_permute_x(int T, int H, const __nv_bfloat16* x, __nv_bfloat16* xp,
-                             cudaStream_t st);
+cudaError_t launch_prepare_x(int T, int H, const __nv_bfloat16* x, __half* xp, float* corr,
+                             int* status, cudaStream_t st);
 cudaError_t launch_inverse_pairs(int P, const int* pairs, int* inv, int* status, cudaStream_t st);
 bool stream_shapes_fit(int H, int I);  // the streaming FFN's 2 stages fit in shared memory
+cudaError_t launch_combine(const FfnArgs& a, int num_sms, cudaStream_t st);
 
 // ---- device helpers --------------------------------------------------------
 __device__ __forceinline__ void report(int* status, int code) {

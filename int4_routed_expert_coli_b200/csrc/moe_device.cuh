@@ -204,8 +204,10 @@ __device__ __forceinline__ void union_block(int P, int E, const int* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Fragment order of a 64-element scale group (see gemv.cu): position of
-// element j of the group in the permuted activation layout.
+// Activation operand of the streaming gate/up GEMV (see gemv.cu).
+//
+// Fragment order: position of element j (0..63) of a 64-element scale group
+// in the permuted layout the m16n8k16 B fragments read.
 __host__ __device__ __forceinline__ int perm64(int j) {
     const int c = j >> 4, jj = j & 15;
     const int m = ((jj >> 3) << 1) + ((jj & 3) >> 1);
@@ -214,17 +216,39 @@ __host__ __device__ __forceinline__ int perm64(int j) {
     return c * 16 + 4 * m + 2 * odd + e;
 }
 
-// Permute one 16-element slice of a bf16 row into fragment order.
-__device__ __forceinline__ void permute_slice16(const uint16_t* src, uint16_t* dst) {
-    const uint4 in0 = *reinterpret_cast<const uint4*>(src);
-    const uint4 in1 = *reinterpret_cast<const uint4*>(src + 8);
-    uint16_t v[16], o[16];
-    *reinterpret_cast<uint4*>(&v[0]) = in0;
-    *reinterpret_cast<uint4*>(&v[8]) = in1;
+// One 64-element group of a bf16 activation row -> fp16 operand in fragment
+// order, odd elements divided by 16 (they meet codes unpacked as 16 (q + 72)),
+// and the group's offset sum
+//   corr = 1032 * sum_{k even} x_k + 1152 * sum_{k odd} (x_k / 16),
+// the part of the MMA result that the unpack offsets contribute (even codes
+// are unpacked as 1032 + q, odd ones as 1152 + 16 q).  Values outside the
+// fp16 range are clamped and reported as COLI_ERR_RANGE.
+__device__ __forceinline__ float prepare_group64(const uint16_t* __restrict__ src,
+                                                 __half* __restrict__ dst, int* status) {
+    float se = 0.f, so = 0.f;
+    uint16_t o[64];
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) o[perm64(jj) & 15] = v[jj];
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(&o[0]);
-    *reinterpret_cast<uint4*>(dst + 8) = *reinterpret_cast<uint4*>(&o[8]);
+    for (int q = 0; q < 8; ++q) {
+        const uint4 in = *reinterpret_cast<const uint4*>(src + q * 8);
+        const uint16_t* v = reinterpret_cast<const uint16_t*>(&in);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int j = q * 8 + i;
+            float f = __uint_as_float((uint32_t)v[i] << 16);
+            if (fabsf(f) > 65504.f) {
+                report(status, COLI_ERR_RANGE);
+                f = copysignf(65504.f, f);
+            }
+            __half h = __float2half_rn((j & 1) ? f * 0.0625f : f);
+            if (j & 1) so += __half2float(h);
+            else se += __half2float(h);
+            o[perm64(j)] = *reinterpret_cast<uint16_t*>(&h);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(o)[q];
+    return 1032.f * se + 1152.f * so;
 }
 
 }  // namespace coli

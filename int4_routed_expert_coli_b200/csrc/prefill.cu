@@ -1,0 +1,655 @@
+// Expert FFN for prefill-sized batches: a grouped GEMM per expert on the
+// fifth-generation tensor cores (tcgen05, accumulators in tensor memory),
+// used when the tokens routed to an expert make its FFN a dense contraction.
+//
+// Shapes.  For expert e with a token list of n_e rows (the batch-union lists,
+// "yunpan.plus/t/30351-1-1", capability two), gate/up is
+//   [2 x I rows of int4 codes] x [n_e tokens x H]  -> h [n_e][I]
+// and down is [H rows] x [n_e x I] -> y [n_e][H].  The weight rows are the MMA
+// M dimension (tiles of 128), the tokens the N dimension (tiles of up to 128,
+// rounded to 16), K is walked in 64-element blocks (one gs64 scale group).
+//
+// Pipeline (one CTA per SM, persistent over a flattened list of tiles):
+//   warp 0      TMA producer: packed int4 codes of the tile rows (a 2-D tensor
+//               map per expert matrix, 32 bytes x 128 rows per K-block) and the
+//               activation tile (128-byte swizzled, fp16);
+//   warps 4-7   dequant: each thread owns one weight row, turns its 64 codes
+//               into fp16 q * s (exact: a 3-bit code magnitude times an 8-bit
+//               bf16 scale fits fp16's 11 bits) and writes the 128-byte
+//               swizzled K-major operand tile;
+//   warp 1      one thread issues tcgen05.mma (kind::f16, fp32 accumulate in
+//               tensor memory; gate and up share the activation tile and have
+//               two accumulators) and commits stage release / tile completion;
+//   warps 8-11  epilogue: tcgen05.ld of the accumulator (each warp its 32
+//               lanes), SwiGLU to fp16 h, or the fp32 y rows of the down GEMM.
+//   Two accumulator buffers let the epilogue of one tile overlap the next.
+// Every wait is bounded (COLI_ERR_TIMEOUT) so nothing can hang the GPU.
+//
+// K order.  Within each group of 8 consecutive K elements the dequant unpack
+// yields codes in the order 0,4,1,5,2,6,3,7; the activation operands (the
+// gathered x and the h written by the gate/up epilogue) are stored in that
+// same order, so every dot product is unchanged.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <new>
+
+#include "moe_device.cuh"
+#include "prefill.cuh"
+#include "ptx.cuh"
+
+namespace coli {
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int kThreadsP = 384;
+constexpr int kHeaderP = 2048;
+constexpr int kSmemLimitP = 227 * 1024;
+
+// Position of element k (0..7) of an 8-group in the operand order.
+__host__ __device__ __forceinline__ int perm8(int k) { return (k & 3) * 2 + (k >> 2); }
+__host__ __device__ __forceinline__ int perm_col(int n) { return (n & ~7) + perm8(n & 7); }
+
+// ---- tcgen05 / TMA wrappers ------------------------------------------------
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= (uint64_t)1 << 16;                    // leading byte offset (unused for SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ uint32_t idesc_f16(int n) {
+    return (1u << 4)                          // D: f32
+           | ((uint32_t)(n >> 3) << 17)       // N
+           | ((uint32_t)(BM >> 4) << 24);     // M = 128; A, B: f16, K-major
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, int c0, int c1,
+                                                 uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// ---- tile bookkeeping --------------------------------------------------------
+struct TileInfo {
+    int e;          // expert row in the table
+    int out_row0;   // first output row (hp / y) of this tile's tokens
+    int b_row0;     // first activation row of this tile's tokens
+    int ntok;       // valid tokens in the tile (<= BN)
+    int n_mma;      // MMA N (ntok rounded up to 16)
+    int m_tile;
+    bool valid;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_t tile,
+                                              int n_slots, int m_tiles) {
+    TileInfo ti;
+    // slot with ntile_start[slot] * m_tiles <= tile < ntile_start[slot + 1] * m_tiles
+    int lo = 0, hi = n_slots;  // invariant: start(lo) <= tile < start(hi)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)__ldg(a.ntile_start + mid) * m_tiles <= tile) lo = mid;
+        else hi = mid;
+    }
+    const int slot = lo;
+    const int s0 = __ldg(a.ntile_start + slot), s1 = __ldg(a.ntile_start + slot + 1);
+    const int nt = s1 - s0;
+    const int64_t local = tile - (int64_t)s0 * m_tiles;
+    ti.m_tile = (int)(local / nt);
+    const int n_tile = (int)(local % nt);
+    const int P = a.T * a.k;
+    int list_begin, ntok_total;
+    ti.valid = true;
+    if (slot < a.n_shared) {
+        ti.e = a.E + slot;
+        list_begin = P + slot * a.T;
+        ntok_total = a.T;
+        ti.b_row0 = (gu ? P : list_begin) + n_tile * BN;
+    } else {
+        const int e = a.active[slot - a.n_shared];
+        const int b = (e >= 0 && e < a.E) ? a.offsets[e] : 0;
+        const int en = (e >= 0 && e < a.E) ? a.offsets[e + 1] : 0;
+        ti.valid = e >= 0 && e < a.E && b >= 0 && en >= b && en <= P;
+        ti.e = ti.valid ? e : 0;
+        list_begin = ti.valid ? b : 0;
+        ntok_total = ti.valid ? en - b : 0;
+        ti.b_row0 = list_begin + n_tile * BN;
+    }
+    ti.out_row0 = list_begin + n_tile * BN;
+    ti.ntok = min(BN, max(0, ntok_total - n_tile * BN));
+    ti.n_mma = max(16, (ti.ntok + 15) & ~15);
+    return ti;
+}
+
+// ---- the GEMM kernel -------------------------------------------------------
+template <bool kGU>
+__global__ void __launch_bounds__(kThreadsP, 1)
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, int stages) {
+    constexpr int NA = kGU ? 2 : 1;                          // weight matrices per tile
+    constexpr int kDqBytes = BM * BK * 2;                    // 16 KB per matrix
+    constexpr int kBBytes = BN * BK * 2;                     // 16 KB
+    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
+    constexpr int kStage = NA * kDqBytes + kBBytes + NA * kPkBytes;
+    constexpr uint32_t kTmemCols = kGU ? 512 : 256;          // 2 buffers x NA x 128
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // TMA landed
+    uint64_t* dq_full = full + 16;                             // operand tile written
+    uint64_t* empty = full + 32;                               // MMAs done reading the stage
+    uint64_t* acc_full = full + 48;                            // [2] accumulator ready
+    uint64_t* acc_empty = full + 50;                           // [2] accumulator drained
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 512);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
+    uint8_t* stage0 = smem + kHeaderP;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&dq_full[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr((const void*)tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait();
+
+    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
+    if (n_act < 0 || n_act > a.E) {
+        if (threadIdx.x == 0) report(a.status, COLI_ERR_BAD_INDEX);
+        n_act = 0;
+    }
+    const int n_slots = n_act + a.n_shared;
+    const int m_tiles = kGU ? a.I / BM : a.H / BM;
+    const int K = kGU ? a.H : a.I;
+    const int KB = K / BK;
+    const int G = K / kGroup;
+    const int64_t n_tiles = (int64_t)__ldg(a.ntile_start + n_slots) * m_tiles;
+
+    auto stage_ptr = [&](int s) { return stage0 + (size_t)s * kStage; };
+    auto timeout = [&]() {
+        report(a.status, COLI_ERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            const uint64_t policy = policy_evict_first();
+            int64_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+                const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+                const CUtensorMap* m0 = a.wmaps + (size_t)ti.e * 3 + (kGU ? 0 : 2);
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = (int)(it % stages);
+                    const uint32_t use = (uint32_t)(it / stages);
+                    if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
+                        timeout();
+                        break;
+                    }
+                    uint8_t* st = stage_ptr(s);
+                    mbar_arrive_expect_tx(&full[s], NA * kPkBytes + kBBytes);
+                    uint8_t* pk = st + NA * kDqBytes + kBBytes;
+                    tma_load_2d_hint(pk, m0, kb * (BK / 2), ti.m_tile * BM, &full[s], policy);
+                    if constexpr (kGU)
+                        tma_load_2d_hint(pk + kPkBytes, a.wmaps + (size_t)ti.e * 3 + 1, kb * (BK / 2),
+                                         ti.m_tile * BM, &full[s], policy);
+                    tma_load_2d(st + NA * kDqBytes, &bmap, kb * BK, ti.b_row0, &full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------- MMA --------------------------------
+        if (lane == 0) {
+            int64_t it = 0, lt = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
+                 tile += gridDim.x, ++lt) {
+                const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+                const int buf = (int)(lt & 1);
+                const uint32_t ause = (uint32_t)(lt >> 1);
+                if (ause > 0 && !mbar_wait(&acc_empty[buf], (ause - 1) & 1)) {
+                    timeout();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t idesc = idesc_f16(ti.n_mma);
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * NA * BM);
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = (int)(it % stages);
+                    if (!mbar_wait(&dq_full[s], (uint32_t)(it / stages) & 1)) {
+                        timeout();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t* st = stage_ptr(s);
+                    const uint32_t b_addr = smem_addr(st + NA * kDqBytes);
+#pragma unroll
+                    for (int m = 0; m < NA; ++m) {
+                        const uint32_t a_addr = smem_addr(st + m * kDqBytes);
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_f16(d0 + m * BM, desc_sw128(a_addr + kk * 32),
+                                    desc_sw128(b_addr + kk * 32), idesc, (kb | kk) != 0);
+                    }
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&acc_full[buf]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------- dequant -------------------------------
+        const int row = threadIdx.x - 128;  // weight row of the tile owned by this thread
+        int64_t it = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+            const DevExpert ex = a.experts[ti.e];
+            const int64_t srow = (int64_t)(ti.m_tile * BM + row) * G;
+            const uint16_t* sc0 = (kGU ? ex.gate_s : ex.down_s) + srow;
+            const uint16_t* sc1 = kGU ? ex.up_s + srow : nullptr;
+            uint16_t nxt0 = __ldg(sc0), nxt1 = kGU ? __ldg(sc1) : 0;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                const uint16_t cur[2] = {nxt0, nxt1};
+                if (kb + 1 < KB) {
+                    nxt0 = __ldg(sc0 + kb + 1);
+                    if (kGU) nxt1 = __ldg(sc1 + kb + 1);
+                }
+                const int s = (int)(it % stages);
+                if (!mbar_wait(&full[s], (uint32_t)(it / stages) & 1)) {
+                    if (lane == 0) timeout();
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = stage_ptr(s);
+#pragma unroll
+                for (int m = 0; m < NA; ++m) {
+                    const uint4* pk = reinterpret_cast<const uint4*>(st + NA * kDqBytes + kBBytes +
+                                                                     m * kPkBytes + row * 32);
+                    const uint4 p0 = pk[0], p1 = pk[1];
+                    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    // bf16 scale -> fp16 (exact for scales in fp16's normal range)
+                    const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur[m] << 16));
+                    const __half2 s2 = __halves2half2(sh, sh);
+                    uint8_t* dq = st + m * kDqBytes + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t w = words[c], w8 = w >> 8;
+                        uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
+                        uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
+                        uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
+                        uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
+                        const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
+                        const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
+                        const __half2 hi = __floats2half2_rn(-72.f, -72.f);
+                        __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
+                        __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
+                        __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
+                        __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
+                        uint4 out;
+                        out.x = *reinterpret_cast<uint32_t*>(&v0);
+                        out.y = *reinterpret_cast<uint32_t*>(&v1);
+                        out.z = *reinterpret_cast<uint32_t*>(&v2);
+                        out.w = *reinterpret_cast<uint32_t*>(&v3);
+                        *reinterpret_cast<uint4*>(dq + ((c ^ (row & 7)) << 4)) = out;
+                    }
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dq_full[s]);
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= 8) {
+        // ------------------------------- epilogue ------------------------------
+        const int q = warp & 3;
+        const int row = q * 32 + lane;  // accumulator lane = weight row of the tile
+        int64_t lt = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
+            const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+            const int buf = (int)(lt & 1);
+            if (!mbar_wait(&acc_full[buf], (uint32_t)(lt >> 1) & 1)) {
+                if (lane == 0) timeout();
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BM);
+            const int feat = ti.m_tile * BM + row;
+            for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
+                uint32_t v0[32];
+                tmem_ld32(tq + c0, v0);
+                if constexpr (kGU) {
+                    uint32_t v1[32];
+                    tmem_ld32(tq + BM + c0, v1);
+                    const int col = perm_col(feat);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < ti.ntok) {
+                            const float g = __uint_as_float(v0[j]), u = __uint_as_float(v1[j]);
+                            float hv = g / (1.f + expf(-g)) * u;
+                            if (fabsf(hv) > 65504.f) {
+                                report(a.status, COLI_ERR_RANGE);
+                                hv = copysignf(65504.f, hv);
+                            }
+                            a.hbuf[(int64_t)(ti.out_row0 + c0 + j) * a.I + col] = __float2half_rn(hv);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < ti.ntok)
+                            a.y[(int64_t)(ti.out_row0 + c0 + j) * a.H + feat] = __uint_as_float(v0[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---- gather: expert-sorted fp16 activations ----------------------------------
+// xg[s] = fp16(x[pairs[s] / k]) for s < P (the union's order), xg[P + t] =
+// fp16(x[t]) (the shared experts' rows), columns in operand order.  Block 0
+// also lays out the tile list: ntile_start[slot] = sum over earlier slots of
+// ceil(tokens / 128).
+__global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int P = g.T * g.k;
+    if (blockIdx.x == 0) {
+        __shared__ int scan_tmp[32];
+        int n_act = *reinterpret_cast<const volatile int*>(g.n_active);
+        if (n_act < 0 || n_act > g.E) n_act = 0;
+        const int n_slots = n_act + g.n_shared;
+        int cnt[2];
+        for (int u = 0; u < 2; ++u) {
+            const int slot = threadIdx.x * 2 + u;
+            int ntok = 0;
+            if (slot < g.n_shared) {
+                ntok = g.T;
+            } else if (slot < n_slots) {
+                const int e = g.active[slot - g.n_shared];
+                if (e >= 0 && e < g.E) ntok = g.offsets[e + 1] - g.offsets[e];
+            }
+            cnt[u] = slot < n_slots ? (max(ntok, 0) + BN - 1) / BN : 0;
+        }
+        int total;
+        const int base = block_exclusive_scan(cnt[0] + cnt[1], scan_tmp, &total);
+        const int s0 = threadIdx.x * 2;
+        if (s0 <= n_slots) g.ntile_start[s0] = base;
+        if (s0 + 1 <= n_slots) g.ntile_start[s0 + 1] = base + cnt[0];
+        return;
+    }
+    const int chunks = g.H / 8;
+    const int64_t n = (int64_t)(P + g.T) * chunks;
+    for (int64_t i = (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)(gridDim.x - 1) * blockDim.x) {
+        const int64_t s = i / chunks;
+        const int c = (int)(i % chunks);
+        int t;
+        if (s < P) {
+            const int p = g.pairs[s];
+            t = (p >= 0 && p < P) ? p / g.k : -1;
+        } else {
+            t = (int)(s - P);
+        }
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (t >= 0) {
+            const uint4 in = *reinterpret_cast<const uint4*>(
+                reinterpret_cast<const uint16_t*>(g.x) + (int64_t)t * g.H + c * 8);
+            const uint16_t* v = reinterpret_cast<const uint16_t*>(&in);
+            uint16_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float f = __uint_as_float((uint32_t)v[j] << 16);
+                if (fabsf(f) > 65504.f) {
+                    report(g.status, COLI_ERR_RANGE);
+                    f = copysignf(65504.f, f);
+                }
+                const __half h = __float2half_rn(f);
+                o[perm8(j)] = *reinterpret_cast<const uint16_t*>(&h);
+            }
+            out = *reinterpret_cast<uint4*>(o);
+        }
+        *reinterpret_cast<uint4*>(g.xg + s * g.H + c * 8) = out;
+    }
+}
+
+// ---- host --------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+               CUtensorMapSwizzle sw) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kGU>
+int gemm_stages() {
+    constexpr int NA = kGU ? 2 : 1;
+    constexpr int kStage = NA * BM * BK * 2 + BN * BK * 2 + NA * BM * BK / 2;
+    return std::min(16, (kSmemLimitP - kHeaderP - 1024) / kStage);
+}
+
+template <bool kGU>
+cudaError_t launch_gemm(const CUtensorMap& bmap, const GemmArgs& a, int num_sms, cudaStream_t st) {
+    constexpr int NA = kGU ? 2 : 1;
+    constexpr int kStage = NA * BM * BK * 2 + BN * BK * 2 + NA * BM * BK / 2;
+    const int stages = gemm_stages<kGU>();
+    const int smem = kHeaderP + 1024 + stages * kStage;
+    cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms);
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<kGU>, bmap, a, stages);
+}
+
+}  // namespace
+
+cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I,
+                              CUtensorMap** d_maps) {
+    *d_maps = nullptr;
+    CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * 3];
+    if (!maps) return cudaErrorMemoryAllocation;
+    for (int e = 0; e < n; ++e) {
+        const DevExpert& x = host_experts[e];
+        const bool ok =
+            encode_2d(&maps[e * 3 + 0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.gate_q, H / 2, I, H / 2,
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&maps[e * 3 + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.up_q, H / 2, I, H / 2,
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&maps[e * 3 + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.down_q, I / 2, H, I / 2,
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (!ok) {
+            delete[] maps;
+            return cudaErrorInvalidValue;
+        }
+    }
+    cudaError_t err = cudaMalloc(d_maps, sizeof(CUtensorMap) * (size_t)n * 3);
+    if (err == cudaSuccess)
+        err = cudaMemcpy(*d_maps, maps, sizeof(CUtensorMap) * (size_t)n * 3, cudaMemcpyHostToDevice);
+    delete[] maps;
+    if (err != cudaSuccess && *d_maps) {
+        cudaFree(*d_maps);
+        *d_maps = nullptr;
+    }
+    return err;
+}
+
+cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* xg, int* ntile_start,
+                           int num_sms, cudaStream_t st) {
+    const int P = f.T * f.k;
+    const int S = P + f.T * f.n_shared;
+    GatherArgs g;
+    g.T = f.T;
+    g.k = f.k;
+    g.E = f.E;
+    g.H = f.H;
+    g.n_shared = f.n_shared;
+    g.x = f.x;
+    g.pairs = f.pairs;
+    g.offsets = f.offsets;
+    g.active = f.active;
+    g.n_active = f.n_active;
+    g.xg = xg;
+    g.ntile_start = ntile_start;
+    g.status = f.status;
+    {
+        const int64_t n = (int64_t)(P + f.T) * (f.H / 8);
+        const int blocks = 1 + (int)std::min<int64_t>((n + 1023) / 1024, (int64_t)num_sms * 2);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(1024);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t err = cudaLaunchKernelEx(&cfg, gather_kernel, g);
+        if (err != cudaSuccess) return err;
+    }
+    GemmArgs a;
+    a.experts = f.experts;
+    a.H = f.H;
+    a.I = f.I;
+    a.E = f.E;
+    a.k = f.k;
+    a.n_shared = f.n_shared;
+    a.T = f.T;
+    a.offsets = f.offsets;
+    a.active = f.active;
+    a.n_active = f.n_active;
+    a.ntile_start = ntile_start;
+    a.wmaps = wmaps;
+    a.hbuf = f.hp;
+    a.y = f.y;
+    a.status = f.status;
+    CUtensorMap xmap, hmap;
+    if (!encode_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xg, f.H, (uint64_t)(P + f.T),
+                   (uint64_t)f.H * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, f.hp, f.I, (uint64_t)S,
+                   (uint64_t)f.I * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    profile_mark(1, st);
+    cudaError_t err = launch_gemm<true>(xmap, a, num_sms, st);
+    if (err != cudaSuccess) return err;
+    profile_mark(2, st);
+    err = launch_gemm<false>(hmap, a, num_sms, st);
+    profile_mark(3, st);
+    return err;
+}
+
+bool prefill_available() { return get_encode() != nullptr; }
+
+}  // namespace coli

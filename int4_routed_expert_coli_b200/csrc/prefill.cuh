@@ -1,0 +1,44 @@
+// Internal interface of the tensor-core prefill path (prefill.cu).
+#pragma once
+
+#include <cuda.h>
+
+#include "coli_internal.cuh"
+
+namespace coli {
+
+struct GemmArgs {
+    const DevExpert* experts;
+    int H, I, E, k, n_shared, T;
+    const int* offsets;      // [E+1]
+    const int* active;       // [E]
+    const int* n_active;     // [1]
+    const int* ntile_start;  // [n_slots+1] token tiles before each slot
+    const CUtensorMap* wmaps;  // [experts][3] packed gate / up / down codes
+    __half* hbuf;            // [S][I] SwiGLU output, operand order
+    float* y;                // [S][H]
+    int* status;
+};
+
+struct GatherArgs {
+    int T, k, E, H, n_shared;
+    const __nv_bfloat16* x;  // [T][H]
+    const int* pairs;        // [T*k]
+    const int* offsets;
+    const int* active;
+    const int* n_active;
+    __half* xg;              // [T*k + T][H] expert-sorted activations, operand order
+    int* ntile_start;
+    int* status;
+};
+
+// Tensor maps of every expert's packed code matrices (device array, 3 per
+// expert: gate, up, down).  Returns an error if the driver lacks tensor maps.
+cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I,
+                              CUtensorMap** d_maps);
+// gather -> gate/up GEMM -> down GEMM (writes y); the caller runs the combine.
+cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* xg,
+                           int* ntile_start, int num_sms, cudaStream_t st);
+bool prefill_available();
+
+}  // namespace coli

@@ -17,7 +17,8 @@ union_kernel(int P, int E, const int* __restrict__ idx, int* __restrict__ counts
 }
 
 // Block 0 routes every token (one warp per token), then builds the union
-// lists and the inverse map; the other blocks permute x into fragment order.
+// lists and the inverse map; the other blocks build the fp16 operand copy of
+// x and its per-group offset sums.
 // Launched as a programmatic dependent: it waits for the previous kernel on
 // the stream before touching the workspace, and lets the FFN kernel start
 // streaming shared-expert weights as early as possible.
@@ -37,13 +38,11 @@ prep_small_kernel(PrepArgs p) {
         union_block(p.T * p.k, p.E, p.idx, p.counts, p.offsets, p.pairs, p.active, p.n_active,
                     p.inv, p.status, hist, scan_tmp);
     } else {
-        const int64_t n_slices = (int64_t)p.T * p.H / 16;
-        for (int64_t s = (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x; s < n_slices;
-             s += (int64_t)(gridDim.x - 1) * blockDim.x) {
-            const int64_t e0 = s * 16;
-            permute_slice16(reinterpret_cast<const uint16_t*>(p.x) + e0,
-                            reinterpret_cast<uint16_t*>(p.xp) + e0);
-        }
+        const int64_t n_groups = (int64_t)p.T * p.H / kGroup;
+        for (int64_t g = (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x; g < n_groups;
+             g += (int64_t)(gridDim.x - 1) * blockDim.x)
+            p.corr[g] = prepare_group64(reinterpret_cast<const uint16_t*>(p.x) + g * kGroup,
+                                        p.xp + g * kGroup, p.status);
     }
 }
 
@@ -73,8 +72,8 @@ static cudaError_t launch_prep_nv(const PrepArgs& p, cudaStream_t st) {
         err = cudaFuncSetAttribute(prep_small_kernel<NV>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int64_t n_slices = (int64_t)p.T * p.H / 16;
-    const int perm_blocks = (int)std::min<int64_t>(64, (n_slices + kUnionThreads - 1) / kUnionThreads);
+    const int64_t n_groups = (int64_t)p.T * p.H / kGroup;
+    const int perm_blocks = (int)std::min<int64_t>(64, (n_groups + 255) / 256);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1 + perm_blocks);
     cfg.blockDim = dim3(kUnionThreads);
