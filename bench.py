@@ -383,6 +383,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's tokens per step (small profiler cases)")
     ap.add_argument("--routed-experts", type=int, default=GLM["E"],
                     help="resident routed experts (default 256); fewer keeps a profiler "
                          "capture small while every step still runs 8 + 1 experts")
@@ -390,6 +392,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     GLM["E"] = args.routed_experts
+    if args.tokens > 0:
+        T0, kind, desc = WORKLOADS[args.workload]
+        WORKLOADS[args.workload] = (args.tokens, kind, desc.replace(f"T={T0}", f"T={args.tokens}"))
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
