@@ -184,6 +184,32 @@ coli_status coli_moe_layer(const coli_moe *h, int32_t T, const void *x_bf16, con
                            coli_out_dtype out_dtype, int32_t *topk_idx_out, float *topk_w_out,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* The layer step (coli_moe_layer with `logits`) for callers that cannot
+ * allocate device memory: it takes no handle and no workspace and allocates
+ * nothing.  The pages have no counterpart of this entry point; it serves
+ * callers whose device memory is owned by a host framework that forbids side
+ * allocations, or latency-critical loops that must not call cudaMalloc (it
+ * can synchronise the device).
+ *   desc       layer description as for coli_moe_create (host struct; the
+ *              expert pointers are device pointers); prefill_min_tokens is
+ *              ignored (the streaming path always runs)
+ *   T          tokens, at most 8; the call's workspace must also fit the
+ *              library's 4 MiB scratch (H 6144 / I 2048 / 257 experts needs
+ *              about 3 MB at T = 8); larger calls return COLI_ERR_WORKSPACE
+ *              before anything is launched
+ *   x_bf16, logits, residual, out, out_dtype: as coli_moe_layer
+ *   status_out nullable device int32: receives the call's device status word
+ *              (as coli_moe_get_status would read it) at the end of the call
+ * The scratch is one fixed __device__ array per GPU that loads the library,
+ * held until exit.  The first call on a device (with that device current)
+ * looks up the array's device address; make that first call before any stream
+ * capture.  Every call shares the array and clears its status word itself;
+ * calls whose work overlaps on the GPU race on it, so order them on one
+ * stream.  Other errors as coli_moe_create and coli_moe_layer. */
+coli_status coli_moe_layer_noalloc(const coli_moe_desc *desc, int32_t T, const void *x_bf16,
+                                   const float *logits, const void *residual, void *out,
+                                   coli_out_dtype out_dtype, int32_t *status_out, void *stream);
+
 /* Synchronise `stream` and return the workspace's device status word
  * (COLI_OK, COLI_ERR_BAD_INDEX or COLI_ERR_TIMEOUT), or COLI_ERR_CUDA if the
  * stream reports an error.  The word stays set until coli_moe_workspace_clear. */

@@ -35,7 +35,8 @@ COLI_OUT_BF16 = 1
 
 EXPORTS = ("coli_moe_create", "coli_moe_destroy", "coli_moe_workspace_size",
            "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union", "coli_moe_ffn",
-           "coli_moe_layer", "coli_moe_get_status", "coli_moe_debug_inject",
+           "coli_moe_layer", "coli_moe_layer_noalloc", "coli_moe_get_status",
+           "coli_moe_debug_inject",
            "coli_moe_profile_enable",
            "coli_moe_profile_read", "coli_status_string")
 
@@ -81,6 +82,8 @@ def _load():
     L.coli_moe_ffn.restype = ctypes.c_int
     L.coli_moe_layer.argtypes = [P, i32, P, P, P, P, P, ctypes.c_int, P, P, P, sz, P]
     L.coli_moe_layer.restype = ctypes.c_int
+    L.coli_moe_layer_noalloc.argtypes = [ctypes.POINTER(CDesc), i32, P, P, P, P, ctypes.c_int, P, P]
+    L.coli_moe_layer_noalloc.restype = ctypes.c_int
     L.coli_moe_get_status.argtypes = [P, P]
     L.coli_moe_get_status.restype = ctypes.c_int
     L.coli_moe_debug_inject.argtypes = [i32]
@@ -158,6 +161,15 @@ def coli_moe_layer(handle, T, x, logits, router_w, residual, out, out_dtype, top
     return _check(s, "coli_moe_layer", raise_on_error)
 
 
+def coli_moe_layer_noalloc(desc, T, x, logits, residual, out, out_dtype, status_out=None,
+                           stream=None, raise_on_error=True):
+    """Layer step without handle or workspace (see include/coli_moe.h):
+    `desc` is a CDesc (e.g. MoELayer.desc), T <= 8."""
+    s = lib.coli_moe_layer_noalloc(ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(residual),
+                                   _ptr(out), out_dtype, _ptr(status_out), _stream(stream))
+    return _check(s, "coli_moe_layer_noalloc", raise_on_error)
+
+
 def coli_moe_workspace_clear(ws, stream=None, raise_on_error=True):
     s = lib.coli_moe_workspace_clear(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     return _check(s, "coli_moe_workspace_clear", raise_on_error)
@@ -206,6 +218,8 @@ class MoELayer:
                 t = getattr(bank, name)[e]
                 setattr(tab[e], name, t.data_ptr())
         desc = CDesc(bank.hidden, bank.inter, n_routed, top_k, 64, n_shared, tab, prefill_min_tokens)
+        self._table = tab
+        self.desc = desc
         h = ctypes.c_void_p()
         s = lib.coli_moe_create(ctypes.byref(desc), ctypes.byref(h))
         if s != COLI_OK:

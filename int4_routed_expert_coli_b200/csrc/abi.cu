@@ -8,15 +8,8 @@
 #include <vector>
 
 #include "coli_internal.cuh"
+#include "handle.cuh"
 #include "prefill.cuh"
-
-struct coli_moe {
-    int device;
-    int H, I, E, k, n_shared, prefill_min;
-    int num_sms;
-    coli::DevExpert* d_experts;  // device table, E + n_shared entries
-    CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)
-};
 
 // Average routed tokens per expert (T*k/E) at or above which a call runs the
 // tensor-core grouped GEMM instead of the streaming dequant-GEMV.

@@ -1,0 +1,14 @@
+// Definition of the opaque coli_moe handle (internal).
+#pragma once
+
+#include <cuda.h>
+
+#include "coli_internal.cuh"
+
+struct coli_moe {
+    int device;
+    int H, I, E, k, n_shared, prefill_min;
+    int num_sms;
+    coli::DevExpert* d_experts;  // device table, E + n_shared entries
+    CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)
+};
