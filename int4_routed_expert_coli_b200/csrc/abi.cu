@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "coli_internal.cuh"
+#include "decode.cuh"
 #include "handle.cuh"
 #include "prefill.cuh"
 
@@ -132,9 +133,16 @@ cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* 
         coli::profile_mark(4, st);
         return err;
     }
-    if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
-    if (err == cudaSuccess) err = coli::launch_ffn_stream(a, h->num_sms, st);
-    return err;
+    const bool fused = h->d_dmaps != nullptr && coli::decode_supported(h->H, h->I, T);
+    if (!x_prepared) {
+        err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
+        if (err == cudaSuccess && fused)  // the fused kernel's counters start at zero
+            err = cudaMemsetAsync(static_cast<char*>(ws) + coli::kSlotCntOffset, 0,
+                                  coli::kHeaderBytes - coli::kSlotCntOffset, st);
+    }
+    if (err != cudaSuccess) return err;
+    if (fused) return coli::launch_decode_fused(a, h->d_dmaps, h->num_sms, st);
+    return coli::launch_ffn_stream(a, h->num_sms, st);
 }
 
 }  // namespace
@@ -234,6 +242,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     h->num_sms = sms;
     h->d_experts = nullptr;
     h->d_wmaps = nullptr;
+    h->d_dmaps = nullptr;
     if (h->prefill_min == 0) h->prefill_min = kDefaultPrefillMin;
     coli::DevExpert* host = static_cast<coli::DevExpert*>(std::malloc(sizeof(coli::DevExpert) * n));
     if (!host) {
@@ -253,10 +262,16 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
     if (err == cudaSuccess && coli::prefill_available())
         err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
+    if (err == cudaSuccess && h->d_wmaps && coli::decode_supported(h->H, h->I, 1) &&
+        coli::build_decode_maps(host, n, h->H, h->I, &h->d_dmaps) != cudaSuccess) {
+        h->d_dmaps = nullptr;  // the fused decode path is an optimisation: go without it
+        cudaGetLastError();
+    }
     std::free(host);
     if (err != cudaSuccess) {
         if (h->d_experts) cudaFree(h->d_experts);
         if (h->d_wmaps) cudaFree(h->d_wmaps);
+        if (h->d_dmaps) cudaFree(h->d_dmaps);
         delete h;
         return COLI_ERR_CUDA;
     }
@@ -268,6 +283,7 @@ void coli_moe_destroy(coli_moe* h) {
     if (!h) return;
     cudaFree(h->d_experts);
     if (h->d_wmaps) cudaFree(h->d_wmaps);
+    if (h->d_dmaps) cudaFree(h->d_dmaps);
     delete h;
 }
 
@@ -365,7 +381,7 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
     if (T <= coli::kSmallT && !prefill) {
         // one launch: route, union, inverse map and activation preparation
         coli::PrepArgs p;
-        p.T = T; p.E = h->E; p.k = h->k; p.H = h->H;
+        p.T = T; p.E = h->E; p.k = h->k; p.H = h->H; p.n_shared = h->n_shared;
         p.logits = lg; p.idx = idx; p.w = w; p.counts = counts; p.offsets = offsets;
         p.pairs = pairs; p.active = active; p.n_active = n_active; p.inv = a.inv;
         p.x = x; p.xp = a.xp; p.corr = a.corr; p.status = a.status;

@@ -16,7 +16,8 @@ constexpr int kMaxExperts = 1024; // E limit (one union thread per expert)
 constexpr int kMaxTopK = 32;      // k limit (one route lane per slot)
 constexpr int kMaxShared = 4;
 constexpr size_t kHeaderBytes = 16384; // status word + tile counters at the start of ws
-constexpr size_t kCounterOffset = 256; // int counters, one per 16-row output tile
+constexpr size_t kSlotCntOffset = 1024; // int counters: finished gate/up items per expert slot
+constexpr size_t kTileCntOffset = 8192; // int counters: finished down items per 32-row tile
 constexpr int kSmallT = 64;            // calls with T <= kSmallT use the fused prep kernel
 
 // Device status codes live in the first word of the workspace.
@@ -109,7 +110,7 @@ struct FfnArgs {
 
 // Arguments of the fused small-batch preparation kernel.
 struct PrepArgs {
-    int T, E, k, H;
+    int T, E, k, H, n_shared;
     const float* logits;      // [T][E]
     int* idx;                 // [T][k] out
     float* w;                 // [T][k] out

@@ -37,6 +37,7 @@
 #include <new>
 
 #include "moe_device.cuh"
+#include "decode.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
 
@@ -651,5 +652,18 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
 }
 
 bool prefill_available() { return get_encode() != nullptr; }
+
+bool encode_tma(CUtensorMap* m, const void* base, int rank, int rows, int row_bytes, int segs,
+                int box_rows) {
+    auto enc = get_encode();
+    if (!enc || rank != 3 || row_bytes % 128) return false;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)(row_bytes / 128), (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)row_bytes};
+    const cuuint32_t box[3] = {128, (cuuint32_t)segs, (cuuint32_t)box_rows};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace coli

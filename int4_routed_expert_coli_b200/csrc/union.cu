@@ -30,6 +30,11 @@ prep_small_kernel(PrepArgs p) {
     pdl_wait();
     pdl_launch_dependents();
     if (blockIdx.x == 0) {
+        // per-call counters of the fused decode kernel start at zero
+        int* slot_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(p.status) + kSlotCntOffset);
+        int* tile_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(p.status) + kTileCntOffset);
+        for (int i = threadIdx.x; i < p.E + p.n_shared; i += blockDim.x) slot_cnt[i] = 0;
+        for (int i = threadIdx.x; i < p.H / 32; i += blockDim.x) tile_cnt[i] = 0;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         for (int t = warp; t < p.T; t += kUnionWarps)
             route_row<NV>(p.logits + (int64_t)t * p.E, p.E, p.k, lane, p.idx + (int64_t)t * p.k,

@@ -62,3 +62,27 @@ def test_bad_union_input_reports_not_faults():
     c.coli_moe_ffn(layer.handle, T, x, w, counts, offsets, pairs, active, na, None, out,
                    c.COLI_OUT_F32, ws)
     assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX
+
+
+def test_withheld_stage_in_fused_decode_times_out():
+    """GLM-5.2 shape, one token: the fused decode kernel (one persistent
+    launch for gate/up, down and combine) with one staged tile withheld; the
+    stalled consumers and every down item waiting on that expert's h give up
+    after their bounded waits."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    bank = synth.make_expert_bank(6144, 2048, 257, seed=26, device="cuda")
+    layer = c.MoELayer(bank, n_routed=256, top_k=8, n_shared=1)
+    x = synth.make_activations(1, 6144, seed=27, device="cuda")
+    lg = synth.make_logits_normal(1, 256, seed=28, device="cuda")
+    ws = layer.workspace(1)
+    assert c.coli_moe_debug_inject(c.COLI_INJECT_WITHHOLD_STAGE) == c.COLI_OK
+    try:
+        layer.layer(x, logits=lg, ws=ws)
+    finally:
+        c.coli_moe_debug_inject(0)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_TIMEOUT
+    c.coli_moe_workspace_clear(ws)
+    out = layer.layer(x, logits=lg, ws=ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_OK
+    ref, _, _ = reference_layer(bank, 256, 8, 1, x, lg)
+    assert_close(out.cpu().numpy(), ref, "after timeout")

@@ -201,3 +201,39 @@ def test_host_errors_launch_nothing(tiny):
                             ws, raise_on_error=False) == c.COLI_ERR_INVALID_ARG
     assert c.coli_moe_layer(layer.handle, 0, x, lg, None, None, out, c.COLI_OUT_F32, None, None,
                             ws, raise_on_error=False) == c.COLI_OK
+
+
+def test_glm_decode_eight_tokens(glm):
+    """T = 8: every token is one of the 8 MMA columns of the fused decode path."""
+    bank, layer = glm
+    x = synth.make_activations(8, 6144, seed=6000, device="cuda")
+    lg = synth.make_logits_normal(8, 256, seed=6001, device="cuda")
+    res = synth.make_residual(8, 6144, seed=6002, device="cuda")
+    out, idx, w, _ = _layer(layer, x, logits=lg, residual=res)
+    ref, ri, rw = reference_layer(bank, 256, 8, 1, x, lg, residual=res)
+    assert np.array_equal(idx, ri)
+    assert_close(out.cpu().numpy(), ref, "decode T=8")
+
+
+def test_glm_fused_decode_matches_streaming_path(glm):
+    """The fused decode kernel (handle with tensor maps) and the streaming
+    kernels (the no-handle entry point) on the same inputs."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    bank, layer = glm
+    for T in (1, 3):
+        x = synth.make_activations(T, 6144, seed=6100 + T, device="cuda")
+        lg = synth.make_logits_normal(T, 256, seed=6200 + T, device="cuda")
+        a = _layer(layer, x, logits=lg)[0]
+        b = torch.empty_like(a)
+        c.coli_moe_layer_noalloc(layer.desc, T, x, lg, None, b, c.COLI_OUT_F32)
+        torch.cuda.synchronize()
+        assert_close(a.cpu().numpy(), b.double().cpu().numpy(), f"fused vs streaming T={T}")
+
+
+def test_glm_decode_deterministic(glm):
+    bank, layer = glm
+    x = synth.make_activations(1, 6144, seed=6300, device="cuda")
+    lg = synth.make_logits_normal(1, 256, seed=6301, device="cuda")
+    a = _layer(layer, x, logits=lg)[0]
+    b = _layer(layer, x, logits=lg)[0]
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
