@@ -54,6 +54,10 @@ WORKLOADS = {
 }
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) of one fused decode launch, from the ncu capture
+# summarised in profiles/decode_fused_kernel_glm_t1.md (tokens per step ->
+# bytes); a workload without a capture of the current kernel reports null.
+FUSED_DECODE_DRAM_BYTES = {}
 
 
 def expert_bytes(H, I):
@@ -251,9 +255,14 @@ def run_ours(args, rank, world, local):
     out = torch.empty(T, H, dtype=torch.float32, device=dev)
     idx = torch.empty(T, k, dtype=torch.int32, device=dev)
     flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    fence_buf = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def flush_l2():
-        return flush_buf.sum()
+        # a read of 256 MiB evicts the weights from L2; the one-element kernel
+        # after it is what the layer's first kernel (launched as a programmatic
+        # dependent, so it may start early) overlaps, instead of the flush
+        flush_buf.sum()
+        fence_buf.zero_()
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
@@ -346,9 +355,14 @@ def run_ours(args, rank, world, local):
     value = tokens / (total_ms / 1e3)
     n_uniq = statistics.mean(uniq)
     step_bytes = (n_uniq + n_sh) * expert_bytes(H, I)
-    gu_ms = phase_ms[1] / max(n_calls, 1)
-    gu_bytes = (n_uniq + n_sh) * gateup_bytes(H, I)
-    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    # dominant kernel: up to 8 tokens the fused decode kernel (routing, gate/up,
+    # down and combine; it streams every active expert whole), otherwise the
+    # gate/up kernel of the streaming or tensor-core path
+    fused = T <= 8
+    k_ms = phase_ms[1] / max(n_calls, 1)
+    k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
+    achieved = k_bytes / (k_ms / 1e3) / 1e9
+    traffic = FUSED_DECODE_DRAM_BYTES.get(T) if fused else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -360,16 +374,17 @@ def run_ours(args, rank, world, local):
                    "l2": "flushed between timed steps (256 MiB read), steps timed alone",
                    "parallelism": f"replicas x{world}"},
         "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": achieved,
-                     "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
-                     "peak_source": P["src"], "traffic": None,
-                     "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms},
-        "phase_ms_per_step": {"prep": phase_ms[0] / max(n_calls, 1), "gateup": gu_ms,
-                              "down_and_combine": phase_ms[2] / max(n_calls, 1)},
+        "roofline": {"bound": "hbm",
+                     "kernel": "decode_fused_kernel" if fused else "gateup_kernel",
+                     "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
+                     "frac": achieved / P["hbm"], "peak_source": P["src"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
+        "phase_ms_per_step": {"before": phase_ms[0] / max(n_calls, 1), "main": k_ms,
+                              "after": phase_ms[2] / max(n_calls, 1)},
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 4},
-        "gpu_launches": (4 if T <= 64 else 6) * args.steps,
+        "gpu_launches": (1 if fused else 4 if T <= 64 else 6) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -119,8 +119,30 @@ bool use_prefill(const coli_moe* h, int64_t T) {
     return h->d_wmaps != nullptr && T * h->k >= (int64_t)h->prefill_min * h->E;
 }
 
+// True when a call with T tokens runs the fused decode kernel.
+bool use_fused(const coli_moe* h, int64_t T) {
+    return h->d_dmaps != nullptr && !use_prefill(h, T) &&
+           coli::decode_supported(h->H, h->I, (int)T, h->E, h->k, h->n_shared, h->num_sms);
+}
+
+// The fused decode kernel: routing from `logits` (or the union in `a` when
+// logits is null), gate/up, down and combine in one launch.
+cudaError_t run_fused(const coli_moe* h, const coli::FfnArgs& a, const float* logits,
+                      int32_t* idx_out, float* w_out, void* ws, cudaStream_t st) {
+    coli::DecodeArgs d;
+    d.f = a;
+    d.maps = h->d_dmaps;
+    d.logits = logits;
+    d.idx_out = idx_out;
+    d.w_out = w_out;
+    d.sync = at<int>(ws, coli::kSlotCntOffset);
+    d.max_slots = 0;  // set by the launcher
+    return coli::launch_decode_fused(d, h->num_sms, st);
+}
+
 // The FFN of a call whose union lists (and inverse map) are ready: tensor-core
-// grouped GEMM for prefill-sized batches, streaming GEMV otherwise.
+// grouped GEMM for prefill-sized batches, the fused decode kernel for up to
+// 8 tokens, streaming GEMV otherwise.
 // `x_prepared`: the fused prep kernel already built the GEMV operand of x.
 cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* ws,
                     cudaStream_t st, bool x_prepared) {
@@ -133,15 +155,9 @@ cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* 
         coli::profile_mark(4, st);
         return err;
     }
-    const bool fused = h->d_dmaps != nullptr && coli::decode_supported(h->H, h->I, T);
-    if (!x_prepared) {
-        err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
-        if (err == cudaSuccess && fused)  // the fused kernel's counters start at zero
-            err = cudaMemsetAsync(static_cast<char*>(ws) + coli::kSlotCntOffset, 0,
-                                  coli::kHeaderBytes - coli::kSlotCntOffset, st);
-    }
+    if (use_fused(h, T)) return run_fused(h, a, nullptr, nullptr, nullptr, ws, st);
+    if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
     if (err != cudaSuccess) return err;
-    if (fused) return coli::launch_decode_fused(a, h->d_dmaps, h->num_sms, st);
     return coli::launch_ffn_stream(a, h->num_sms, st);
 }
 
@@ -262,7 +278,8 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
     if (err == cudaSuccess && coli::prefill_available())
         err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
-    if (err == cudaSuccess && h->d_wmaps && coli::decode_supported(h->H, h->I, 1) &&
+    if (err == cudaSuccess && h->d_wmaps &&
+        coli::decode_supported(h->H, h->I, 1, h->E, h->k, h->n_shared, h->num_sms) &&
         coli::build_decode_maps(host, n, h->H, h->I, &h->d_dmaps) != cudaSuccess) {
         h->d_dmaps = nullptr;  // the fused decode path is an optimisation: go without it
         cudaGetLastError();
@@ -378,6 +395,12 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
     coli::FfnArgs a = make_args(h, T, x_bf16, w, offsets, pairs, active, n_active, residual, out,
                                 out_dtype, ws);
     const bool prefill = use_prefill(h, T);
+    if (err == cudaSuccess && use_fused(h, T)) {
+        // one launch: every CTA routes the tokens itself
+        err = run_fused(h, a, lg, topk_idx_out, topk_w_out, ws, st);
+        profile_end_call();
+        return from_cuda(err);
+    }
     if (T <= coli::kSmallT && !prefill) {
         // one launch: route, union, inverse map and activation preparation
         coli::PrepArgs p;

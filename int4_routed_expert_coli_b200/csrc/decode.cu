@@ -1,36 +1,41 @@
-// Fused decode step (T <= 8 tokens): gate/up + SwiGLU, down and the
-// weighted combine in one persistent kernel, streaming every active
-// expert's int4 gs64 weights from HBM exactly once per call ("batch-union",
-// "yunpan.plus/t/30351-1-1", capability two).
+// Fused decode step (T <= 8 tokens): routing, batch-union, gate/up +
+// SwiGLU, down and the weighted combine in one persistent kernel that streams
+// every active expert's int4 gs64 weights from HBM exactly once per call
+// ("batch-union", "yunpan.plus/t/30351-1-1", capability two).
 //
-// Items.  A CTA (one per SM) walks one list of items: first every gate/up
-// item (8 gate rows + the same 8 up rows of one expert slot; shared experts
-// first, so their weights stream while routing finishes), then every down
-// item (32 rows of W_d).  A slot's down items read the h rows its gate/up
-// items wrote; a per-slot counter (incremented after each gate/up item's h is
-// written, read with acquire semantics) orders them, and because every CTA
-// finishes all of its gate/up items before any down item, the waits cannot
-// form a cycle.  The last down item of each 32-row output tile combines it:
-//   out[t][m] = sum_j w[t][j] y[(t,j)][m] (j ascending) + y_shared[t][m] (+ residual)
-// in fp32 in that fixed order.
+// Routing.  Every CTA routes the T tokens itself from the logits (one warp
+// per token, the exact rule of the routing step) and builds the same slot
+// table in shared memory: shared experts first, then the active routed
+// experts in ascending order, each with the positions and gate weights of
+// its tokens.  Given a precomputed union instead (the FFN entry point), the
+// table is read from it.
 //
-// Data movement.  A producer warp loads each item with one 3-D TMA tensor
-// copy per 8 (gate/up) or 32 (down) rows: the row is viewed as chunks of 128
-// bytes plus one or two chunks past its end (zero-filled), 128-byte swizzle.
-// The odd number of chunks per staged row makes the swizzle put the same
-// column of different rows on different banks, so the consumers' fragment
-// reads are conflict-free without per-row copies.  Scales come by bulk copy.
+// Gate/up.  An item is 8 gate rows + the same 8 up rows of one slot over the
+// whole hidden dimension; items are dealt round-robin to the CTAs (one per
+// SM), shared experts first, so their weights stream while routing runs.
+// The gate weight is folded into the epilogue: h' = w * silu(g) * u (fp16).
+// After writing an item's h' values a warp bumps the slot's counter.
 //
-// Arithmetic as in the streaming GEMV (gemv.cu): raw fp16 unpack plus
-// per-(token, group) offset sums for gate/up, exact unpack for down, m16n8k16
-// MMA with fp32 accumulation, gs64 scale applied to each group's partial sum.
-// For T <= 8 all tokens are the 8 MMA columns of every gate/up item, so those
-// activation fragments stay in registers for the whole kernel.
+// Down + combine.  A CTA owns a fixed set of 16-row tiles of the output and
+// streams, slot after slot, those rows of W_d.  The MMA columns are the
+// tokens, so y = sum over slots of W_d h' accumulates in registers: the
+// combine is the accumulation itself, in a fixed order (slot order, then a
+// fixed sum over the warps).  A slot's h' rows are read once its counter says
+// all its gate/up tiles are done.
 //
-// Reduction.  Eleven consumer warps split K; their partials go to one of two
-// reduction buffers and one rotating warp per item sums them in a fixed order
-// and writes the outputs, while the other warps go on to the next item.
-// Every wait is bounded (COLI_ERR_TIMEOUT).
+// Data movement.  A producer warp loads each stage with 3-D TMA tensor copies
+// of the packed code rows (viewed as 128-byte chunks plus zero-filled padding
+// chunks, 128-byte swizzle, so the consumers' fragment reads spread over the
+// banks) and 2-D copies of the scale rows (padded to 8 x odd columns).
+//
+// Arithmetic as in the streaming GEMV: raw fp16 unpack with the per-(token,
+// group) offset sum as the initial accumulator for gate/up, exact unpack for
+// down, m16n8k16 MMA with fp32 accumulation, gs64 scale applied to each
+// group's partial.  Eleven consumer warps split K; a gate/up item's partials
+// are summed by one rotating warp through four reduction buffers.
+//
+// Every wait is bounded (COLI_ERR_TIMEOUT).  The counters are zero on entry;
+// the last CTA to finish puts them back to zero.
 #include <algorithm>
 #include <new>
 
@@ -44,68 +49,98 @@ namespace {
 constexpr int kCW = 11;                      // consumer warps (12 warps in all)
 constexpr int kThreadsD = (kCW + 1) * 32;    // + producer warp
 constexpr int kStagesD = 3;
-constexpr int kRedBufs = 2;
+constexpr int kRedBufs = 4;
 constexpr int kSmemLimitD = 227 * 1024;
-constexpr int kGuRows = 16, kDnRows = 32;
+constexpr int kGuRows = 8;                   // gate rows (and up rows) per gate/up item
+constexpr int kDnRows = 16;                  // rows per down tile
+constexpr int kMaxMT = 3;                    // down tiles per CTA
+constexpr int kMaps = 6;                     // per expert: 3 code maps, 3 scale maps
+constexpr int kMaxPairs = 256;               // T * k
+constexpr int kRedFloats = kRedBufs * kCW * 4 * 32;
+static_assert(kRedFloats >= kCW * kMaxMT * 4 * 32, "final reduction reuses the buffers");
 
-struct Layout {
-    int gu_segs, dn_segs;       // 128-byte chunks per staged row (odd)
-    int gu_op, dn_op;           // bytes of one TMA copy (8 or 32 rows)
-    int gu_scale, dn_scale;     // offset of the scale block in a stage
-    int gu_tx, dn_tx;           // bytes a stage receives
-    int stage_bytes;
-    int red_off, corr_off, stage_off, smem;
+struct SlotEntry {
+    int e;           // expert index (E + i for shared expert i); -1: invalid slot
+    int list_begin;  // h row of the first token on the slot's list
+    int8_t pos[8];   // position of token t on the list; -1: not routed here
+    float w[8];      // gate weight of token t (1 for a shared expert)
 };
+static_assert(sizeof(SlotEntry) == 48, "slot entry layout");
 
-__host__ __device__ inline int odd_segs(int row_bytes) {
+// A padded scale row: 8 * odd bf16 columns, so 8 rows fall on distinct banks.
+__host__ __device__ inline int padded_groups(int G) {
+    int p = (G + 1 + 7) / 8 * 8;
+    if ((p / 8) % 2 == 0) p += 8;
+    return p;
+}
+
+// Chunks per staged gate/up row: = 2 (mod 8), so rows r and r + 1 differ by
+// two in the swizzle phase and a half-warp's 8-byte reads hit 32 banks.
+__host__ __device__ inline int gu_segs_for(int row_bytes) {
+    int s = row_bytes / 128;
+    while (s % 8 != 2) ++s;
+    return s;
+}
+
+// Chunks per staged down row: odd (costs less shared memory than the rule above).
+__host__ __device__ inline int dn_segs_for(int row_bytes) {
     const int chunks = row_bytes / 128;
     return chunks + ((chunks % 2 == 0) ? 1 : 2);
 }
 
-__host__ __device__ inline Layout make_layout(int H, int I) {
+struct Layout {
+    int gu_segs, dn_segs;       // 128-byte chunks per staged code row
+    int gGp, dGp;               // padded scale row lengths (bf16 elements)
+    int gu_op, gu_sc, gu_tx;    // gate/up item: code copy, scale copy, bytes per stage
+    int dn_op, dn_sc;           // down tile: code copy, scale copy
+    int stage_bytes;
+    int red_off, corr_off, route_off, table_off, stage_off, smem;
+};
+
+__host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
     Layout L;
-    L.gu_segs = odd_segs(H / 2);
-    L.dn_segs = odd_segs(I / 2);
-    L.gu_op = 8 * L.gu_segs * 128;
+    L.gu_segs = gu_segs_for(H / 2);
+    L.dn_segs = dn_segs_for(I / 2);
+    // every consumer warp owns kMaxGW (kMaxDW) consecutive groups; the groups
+    // past the end read zero scales from the padding columns
+    L.gGp = padded_groups(kCW * kMaxGW > H / kGroup ? kCW * kMaxGW : H / kGroup);
+    L.dGp = padded_groups(kCW * kMaxDW > I / kGroup ? kCW * kMaxDW : I / kGroup);
+    L.gu_op = kGuRows * L.gu_segs * 128;
+    L.gu_sc = kGuRows * L.gGp * 2;
+    L.gu_tx = 2 * L.gu_op + 2 * L.gu_sc;
     L.dn_op = kDnRows * L.dn_segs * 128;
-    const int gG = H / kGroup, dG = I / kGroup;
-    L.gu_scale = 2 * L.gu_op;
-    L.dn_scale = L.dn_op;
-    L.gu_tx = 2 * L.gu_op + kGuRows * gG * 2;
-    L.dn_tx = L.dn_op + kDnRows * dG * 2;
-    L.stage_bytes = ((L.gu_tx > L.dn_tx ? L.gu_tx : L.dn_tx) + 1023) / 1024 * 1024;
+    L.dn_sc = kDnRows * L.dGp * 2;
+    const int dn_stage = kMaxMT * (L.dn_op + L.dn_sc);
+    L.stage_bytes = ((L.gu_tx > dn_stage ? L.gu_tx : dn_stage) + 1023) / 1024 * 1024;
     L.red_off = 1024;
-    L.corr_off = L.red_off + kRedBufs * kCW * 2 * 4 * 32 * 4;
-    const int corr_bytes = 8 * gG * 4;
-    L.stage_off = (L.corr_off + corr_bytes + 1023) / 1024 * 1024;
+    L.corr_off = L.red_off + kRedFloats * 4;
+    L.route_off = L.corr_off + kCW * kMaxGW * 8 * 4;
+    L.table_off = L.route_off + 3 * kMaxPairs * 4;
+    L.stage_off = (L.table_off + max_slots * (int)sizeof(SlotEntry) + 1023) / 1024 * 1024;
     L.smem = L.stage_off + kStagesD * L.stage_bytes + 1024;  // + alignment slack
     return L;
 }
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-__device__ __forceinline__ void unpack_raw(uint32_t w, uint32_t o[4]) {
-    const uint32_t w8 = w >> 8;
-    o[0] = (w & 0x000F000Fu) ^ 0x64086408u;
-    o[1] = (w & 0x00F000F0u) ^ 0x64806480u;
-    o[2] = (w8 & 0x000F000Fu) ^ 0x64086408u;
-    o[3] = (w8 & 0x00F000F0u) ^ 0x64806480u;
+// Unpack of a packed word (8 codes, two k16 steps of a lane's fragment) by
+// the fp16 magic-number trick: step 0 takes bytes 0 and 2, step 1 bytes 1 and
+// 3; e holds the even-k codes as 1032 + q, o the odd-k codes as 1152 + 16 q.
+__device__ __forceinline__ void unpack_raw_step(uint32_t w, int step, uint32_t& e, uint32_t& o) {
+    const uint32_t v = step ? (w >> 8) : w;
+    e = (v & 0x000F000Fu) ^ 0x64086408u;
+    o = (v & 0x00F000F0u) ^ 0x64806480u;
 }
 
-__device__ __forceinline__ void unpack_exact(uint32_t w, uint32_t o[4]) {
-    const __half2 bias_lo = __floats2half2_rn(1032.f, 1032.f);
-    const __half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
-    const __half2 bias_hi = __floats2half2_rn(-72.f, -72.f);
-    uint32_t t[4];
-    unpack_raw(w, t);
-    __half2 v0 = __hsub2(*reinterpret_cast<__half2*>(&t[0]), bias_lo);
-    __half2 v1 = __hfma2(*reinterpret_cast<__half2*>(&t[1]), sixteenth, bias_hi);
-    __half2 v2 = __hsub2(*reinterpret_cast<__half2*>(&t[2]), bias_lo);
-    __half2 v3 = __hfma2(*reinterpret_cast<__half2*>(&t[3]), sixteenth, bias_hi);
-    o[0] = *reinterpret_cast<uint32_t*>(&v0);
-    o[1] = *reinterpret_cast<uint32_t*>(&v1);
-    o[2] = *reinterpret_cast<uint32_t*>(&v2);
-    o[3] = *reinterpret_cast<uint32_t*>(&v3);
+// The same, exact: e = q_even, o = q_odd as fp16.
+__device__ __forceinline__ void unpack_exact_step(uint32_t w, int step, uint32_t& e, uint32_t& o) {
+    uint32_t re, ro;
+    unpack_raw_step(w, step, re, ro);
+    const __half2 v0 = __hsub2(*reinterpret_cast<__half2*>(&re), __floats2half2_rn(1032.f, 1032.f));
+    const __half2 v1 = __hfma2(*reinterpret_cast<__half2*>(&ro), __floats2half2_rn(0.0625f, 0.0625f),
+                               __floats2half2_rn(-72.f, -72.f));
+    e = *reinterpret_cast<const uint32_t*>(&v0);
+    o = *reinterpret_cast<const uint32_t*>(&v1);
 }
 
 __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t a0, uint32_t a1,
@@ -118,54 +153,68 @@ __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t 
           "f"(c[3]));
 }
 
-template <bool kExact>
-__device__ __forceinline__ void group_partial(float part[4], uint2 wa, uint2 wb,
-                                              const uint32_t bw[8]) {
-    uint32_t aa[8], ab[8];
-    if constexpr (kExact) {
-        unpack_exact(wa.x, aa);
-        unpack_exact(wa.y, aa + 4);
-        unpack_exact(wb.x, ab);
-        unpack_exact(wb.y, ab + 4);
-    } else {
-        unpack_raw(wa.x, aa);
-        unpack_raw(wa.y, aa + 4);
-        unpack_raw(wb.x, ab);
-        unpack_raw(wb.y, ab + 4);
-    }
-    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-    float p0[4], p1[4];
-    mma16816(p0, zero, aa[0], ab[0], aa[1], ab[1], bw[0], bw[1]);
-    mma16816(p1, zero, aa[2], ab[2], aa[3], ab[3], bw[2], bw[3]);
-    mma16816(p0, p0, aa[4], ab[4], aa[5], ab[5], bw[4], bw[5]);
-    mma16816(p1, p1, aa[6], ab[6], aa[7], ab[7], bw[6], bw[7]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) part[q] = p0[q] + p1[q];
-}
-
-// 8 bytes of a staged row: codes [64 grp + 16 c, +16) of row `row`, in the
-// padded, swizzled layout (segments of 128 bytes, segs per row, 16-byte
-// chunk j of segment s stored at chunk j ^ (s & 7)).
-__device__ __forceinline__ uint2 load_codes(const uint8_t* op_base, int row, int segs, int grp,
-                                            int c) {
-    const int kc = grp >> 2;                       // 128-byte segment of the row
-    const int j = ((grp & 3) << 1) + (c >> 1);     // 16-byte chunk in the segment
+// Byte offset (in a code copy) of the 8 bytes lane c of row `row` feeds to
+// group grp: the padded, swizzled layout (segments of 128 bytes, segs per
+// row, 16-byte chunk j of segment s stored at chunk j ^ (s & 7)).
+__device__ __forceinline__ int code_offset(int row, int segs, int grp, int c) {
+    const int kc = grp >> 2;
+    const int j = ((grp & 3) << 1) + (c >> 1);
     const int seg = row * segs + kc;
-    const uint8_t* p = op_base + seg * 128 + ((j ^ (seg & 7)) << 4) + ((c & 1) << 3);
-    return *reinterpret_cast<const uint2*>(p);
+    return seg * 128 + ((j ^ (seg & 7)) << 4) + ((c & 1) << 3);
 }
 
-__device__ __forceinline__ void load_b(uint32_t bw[8], const __half* p) {
+__device__ __forceinline__ void load_b_cg(uint32_t bw[8], const __half* p) {
     const uint4 b0 = __ldcg(reinterpret_cast<const uint4*>(p));
     const uint4 b1 = __ldcg(reinterpret_cast<const uint4*>(p) + 1);
     bw[0] = b0.x; bw[1] = b0.y; bw[2] = b0.z; bw[3] = b0.w;
     bw[4] = b1.x; bw[5] = b1.y; bw[6] = b1.z; bw[7] = b1.w;
 }
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
+// 16 consecutive bf16 activations (elements 16c .. 16c+15 of a group) -> this
+// lane's 8 fp16 pairs of the gate/up B fragment, in the fragment order of
+// the streaming GEMV: pair q holds elements e and e + 4, e = (q & 3) + 8 (q >> 2),
+// odd elements divided by 16.  Out-of-range values are clamped (|x| <= 65504,
+// |x / 16| <= 4094); amax collects |x| for the range report.
+__device__ __forceinline__ void x_fragment(const uint16_t* __restrict__ src, uint32_t bw[8],
+                                           float& amax) {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    const uint32_t in[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int e = (q & 3) + 8 * (q >> 2);
+        const uint32_t wl = in[e >> 1], wh = in[(e >> 1) + 2];
+        float lo = __uint_as_float((q & 1) ? (wl & 0xFFFF0000u) : (wl << 16));
+        float hi = __uint_as_float((q & 1) ? (wh & 0xFFFF0000u) : (wh << 16));
+        amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+        if (q & 1) {
+            lo = fminf(fmaxf(lo * 0.0625f, -4094.f), 4094.f);
+            hi = fminf(fmaxf(hi * 0.0625f, -4094.f), 4094.f);
+        }
+        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(bw[q]) : "f"(hi), "f"(lo));
+    }
+}
+
+// Offset sums of one group for this lane's two token columns: the MMA of the
+// constant part of the raw unpack (1032 at even k, 1152 at odd k, every row)
+// with the B fragment, i.e. 1032 * sum x_even + 1152 * sum (x_odd / 16).
+__device__ __forceinline__ void offset_sums(const uint32_t bw[8], float c[4]) {
+    const uint32_t ev = 0x64086408u, od = 0x64806480u;  // fp16 pairs (1032, 1032), (1152, 1152)
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    mma16816(c, zero, ev, ev, od, od, bw[0], bw[1]);
+    mma16816(c, c, ev, ev, od, od, bw[2], bw[3]);
+    mma16816(c, c, ev, ev, od, od, bw[4], bw[5]);
+    mma16816(c, c, ev, ev, od, od, bw[6], bw[7]);
+}
+
+__device__ __forceinline__ int ld_relaxed(const int* p) {
     int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int c0, int c1, int c2,
@@ -177,365 +226,564 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int c0,
         : "memory");
 }
 
-struct SlotD {
-    int e, list_begin, ntok;
-    bool shared, valid;
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Pointers into the dynamic shared memory.
+struct Smem {
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* red_empty;
+    uint64_t* tbl_ready;
+    volatile int* abort_flag;
+    volatile int* n_slots;
+    int* red_cnt;      // [kRedBufs] partials written into each reduction buffer
+    float* red;        // reduction buffers; during the prologue, the logits
+    float* corr;       // [H/64][8] offset sums of the 8 token columns
+    int* s_idx;        // [T*k] routing
+    float* s_w;
+    int* s_aux;
+    SlotEntry* table;
+    uint8_t* stage0;
 };
 
-__device__ __forceinline__ SlotD slot_of(const FfnArgs& a, int slot, int n_act) {
-    SlotD s;
-    const int P = a.T * a.k;
-    if (slot < a.n_shared) {
-        s.e = a.E + slot;
-        s.list_begin = P + slot * a.T;
-        s.ntok = a.T;
-        s.shared = true;
-        s.valid = true;
-        return s;
+__device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L) {
+    Smem S;
+    S.full = reinterpret_cast<uint64_t*>(smem);
+    S.empty = S.full + kStagesD;
+    S.red_empty = S.empty + kStagesD;
+    S.tbl_ready = S.red_empty + kRedBufs;
+    S.abort_flag = reinterpret_cast<volatile int*>(smem + 512);
+    S.n_slots = S.abort_flag + 1;
+    S.red_cnt = reinterpret_cast<int*>(smem + 528);
+    S.red = reinterpret_cast<float*>(smem + L.red_off);
+    S.corr = reinterpret_cast<float*>(smem + L.corr_off);
+    S.s_idx = reinterpret_cast<int*>(smem + L.route_off);
+    S.s_w = reinterpret_cast<float*>(S.s_idx + kMaxPairs);
+    S.s_aux = S.s_idx + 2 * kMaxPairs;
+    S.table = reinterpret_cast<SlotEntry*>(smem + L.table_off);
+    S.stage0 = smem + L.stage_off;
+    return S;
+}
+
+constexpr int kConsumerThreads = kCW * 32;
+
+__device__ __forceinline__ void consumers_sync() { named_barrier(1, kConsumerThreads); }
+
+__device__ void table_init(const FfnArgs& a, const Smem& S, int max_slots) {
+    for (int i = threadIdx.x; i < max_slots; i += kConsumerThreads) {
+        SlotEntry& en = S.table[i];
+        en.e = -1;
+        en.list_begin = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            en.pos[t] = -1;
+            en.w[t] = 0.f;
+        }
     }
-    s.shared = false;
-    const int r = slot - a.n_shared;
-    const int e = r < n_act ? a.active[r] : -1;
-    const int b = (e >= 0 && e < a.E) ? a.offsets[e] : 0;
-    const int en = (e >= 0 && e < a.E) ? a.offsets[e + 1] : 0;
-    s.valid = e >= 0 && e < a.E && b >= 0 && en >= b && en <= P && en - b <= 8;
-    s.e = s.valid ? e : 0;
-    s.list_begin = s.valid ? b : 0;
-    s.ntok = s.valid ? en - b : 0;
-    return s;
+    consumers_sync();
+    for (int i = threadIdx.x; i < a.n_shared; i += kConsumerThreads) {
+        SlotEntry& en = S.table[i];
+        en.e = a.E + i;
+        en.list_begin = a.T * a.k + i * a.T;
+        for (int t = 0; t < a.T; ++t) {
+            en.pos[t] = (int8_t)t;
+            en.w[t] = 1.f;
+        }
+    }
+}
+
+// Route the T tokens and build the slot table from the routing: the union
+// of the pairs p = t * k + j, experts ascending, tokens ascending inside an
+// expert (the lists the batch-union step defines).
+template <int NV>
+__device__ void table_from_logits(const DecodeArgs& d, const Smem& S, const float* lg) {
+    const FfnArgs& a = d.f;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int P = a.T * a.k;
+    if (warp < a.T)
+        route_row<NV>(lg + warp * a.E, a.E, a.k, lane, S.s_idx + warp * a.k, S.s_w + warp * a.k);
+    table_init(a, S, d.max_slots);
+    consumers_sync();
+    if (blockIdx.x == 0) {
+        for (int p = tid; p < P; p += kConsumerThreads) {
+            if (d.idx_out) d.idx_out[p] = S.s_idx[p];
+            if (d.w_out) d.w_out[p] = S.s_w[p];
+        }
+    }
+    // a pair is its expert's leader if no earlier pair has the same expert
+    for (int p = tid; p < P; p += kConsumerThreads) {
+        const int e = S.s_idx[p];
+        int lead = 1;
+        for (int q = 0; q < p; ++q) lead &= S.s_idx[q] != e;
+        S.s_aux[p] = lead;
+    }
+    consumers_sync();
+    for (int p = tid; p < P; p += kConsumerThreads) {
+        const int e = S.s_idx[p];
+        int before = 0, rank = 0, pos = 0;
+        for (int q = 0; q < P; ++q) {
+            const int eq = S.s_idx[q];
+            before += eq < e;
+            rank += (eq < e) & S.s_aux[q];
+            pos += (q < p) & (eq == e);
+        }
+        SlotEntry& en = S.table[a.n_shared + rank];
+        if (S.s_aux[p]) {
+            en.e = e;
+            en.list_begin = before;
+        }
+        const int t = p / a.k;
+        en.pos[t] = (int8_t)pos;
+        en.w[t] = S.s_w[p];
+    }
+    if (warp == 0) {
+        int n = 0;
+        for (int p = lane; p < P; p += 32) n += S.s_aux[p];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        if (lane == 0) *S.n_slots = a.n_shared + n;
+    }
+}
+
+// Slot table from a given union (counts / offsets / pairs / active /
+// n_active and the gate weights); an inconsistent entry is reported as
+// COLI_ERR_BAD_INDEX and its slot skipped.
+__device__ void table_from_union(const DecodeArgs& d, const Smem& S) {
+    const FfnArgs& a = d.f;
+    const int tid = threadIdx.x;
+    const int P = a.T * a.k;
+    table_init(a, S, d.max_slots);
+    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
+    const int cap = d.max_slots - a.n_shared;
+    if (n_act < 0 || n_act > cap) {
+        if (tid == 0) report(a.status, COLI_ERR_BAD_INDEX);
+        n_act = n_act < 0 ? 0 : cap;
+    }
+    consumers_sync();
+    for (int i = tid; i < n_act; i += kConsumerThreads) {
+        SlotEntry& en = S.table[a.n_shared + i];
+        const int e = a.active[i];
+        bool ok = e >= 0 && e < a.E;
+        const int b = ok ? a.offsets[e] : 0;
+        const int n = ok ? a.offsets[e + 1] - b : 0;
+        ok = ok && b >= 0 && n >= 1 && n <= a.T && b + n <= P;
+        for (int q = 0; ok && q < n; ++q) {
+            const int p = a.pairs[b + q];
+            ok = p >= 0 && p < P;
+            if (!ok) break;
+            const int t = p / a.k;
+            ok = en.pos[t] < 0;  // a token appears once per expert
+            en.pos[t] = (int8_t)q;
+            en.w[t] = a.topk_w[p];
+        }
+        if (ok) {
+            en.e = e;
+            en.list_begin = b;
+        } else {
+            report(a.status, COLI_ERR_BAD_INDEX);
+        }
+    }
+    if (tid == 0) *S.n_slots = a.n_shared + n_act;
 }
 
 struct Ctx {
     const FfnArgs& a;
     const Layout& L;
-    uint8_t* stage0;
-    uint64_t* full;
-    uint64_t* empty;
-    uint64_t* red_full;
-    uint64_t* red_empty;
-    volatile int* abort_flag;
-    float* red;
-    const float* corr_s;
-    int* slot_cnt;
-    int* tile_cnt;
-    int n_act, n_slots, gu_tiles, dn_tiles, gG, dG;
+    const Smem& S;
+    int* sync;
+    int n_slots, gu_tiles;
 };
 
 __device__ __forceinline__ void fail(const Ctx& x, int lane) {
     if (lane == 0) {
         report(x.a.status, COLI_ERR_TIMEOUT);
-        *x.abort_flag = 1;
+        *x.S.abort_flag = 1;
     }
 }
 
-// One item of the consumer walk (index `local` within its phase, `j` in the
-// CTA's item sequence).  Returns false when the kernel must wind down.
-template <bool kGU>
-__device__ __forceinline__ bool consume_item(const Ctx& x, int64_t local, int j,
-                                             const uint32_t (&breg)[kMaxGW][8], int& ready_slot) {
+// Partials of item j -> reduction buffer.  The warp that writes the last
+// partial sums them (in warp order, so the result does not depend on which
+// warp that is) and gets 1 with the sums in v; the others get 0 and move on
+// at once (-1: timeout).
+__device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&acc)[4],
+                                           float (&v)[4]) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rb = j % kRedBufs, ruse = j / kRedBufs;
+    if (ruse > 0 && !mbar_wait(&x.S.red_empty[rb], (ruse - 1) & 1)) return -1;
+    float* rbuf = x.S.red + rb * (kCW * 4 * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) rbuf[(warp * 4 + q) * 32 + lane] = acc[q];
+    __threadfence_block();
+    __syncwarp();
+    int arrived = 0;
+    if (lane == 0) arrived = atomicAdd(x.S.red_cnt + rb, 1);
+    arrived = __shfl_sync(0xffffffffu, arrived, 0);
+    if (arrived != kCW - 1) return 0;
+    __threadfence_block();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) s += rbuf[(w * 4 + q) * 32 + lane];
+        v[q] = s;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        x.S.red_cnt[rb] = 0;
+        mbar_arrive(&x.S.red_empty[rb]);
+    }
+    return 1;
+}
+
+// Make this warp's h' stores of `n` finished gate/up tiles of `slot` visible
+// GPU-wide, then count them on the slot's counter.
+__device__ __forceinline__ void publish(const Ctx& x, int slot, int n) {
+    fence_acq_rel_gpu();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicAdd(x.sync + 1 + slot, n);
+}
+
+// One gate/up item (j = position in the CTA's stage sequence).  Returns
+// false when the kernel must wind down.  A reducing warp publishes its tiles
+// one reduction late (pend_slot / pend_n), so the fence finds its stores
+// long finished instead of stalling on them.
+__device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
+                                            const uint32_t (&breg)[kMaxGW][8],
+                                            const int (&coff)[kMaxGW], int g_lo,
+                                            int& pend_slot, int& pend_n) {
     const FfnArgs& a = x.a;
     const Layout& L = x.L;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = lane >> 2, c = lane & 3;
-    if (*x.abort_flag) return false;
+    const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+    if (*x.S.abort_flag) return false;
     const int stage = j % kStagesD, use = j / kStagesD;
-    const int rb = j % kRedBufs, ruse = j / kRedBufs;
-    const int tiles = kGU ? x.gu_tiles : x.dn_tiles;
-    const int slot = (int)(local / tiles);
-    const int tile = (int)(local % tiles);
-    const SlotD sl = slot_of(a, slot, x.n_act);
-    if (!sl.valid && threadIdx.x == 0) report(a.status, COLI_ERR_BAD_INDEX);
-    const int G = kGU ? x.gG : x.dG;
-    const int g_lo = (G * warp) / kCW, g_hi = (G * (warp + 1)) / kCW;
+    const int slot = item / x.gu_tiles, tile = item - slot * x.gu_tiles;
+    const SlotEntry* en = x.S.table + slot;
+    const bool valid = en->e >= 0;
 
-    float acc[2][4];
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
-
-    bool ok = true;
-    uint32_t bdn[kGU ? 1 : kMaxDW][8];
-    if constexpr (!kGU) {
-        // this slot's h must be complete (every gate/up item counted)
-        if (sl.valid && slot > ready_slot) {
-            const uint64_t t0 = global_timer_ns();
-            while (ld_acquire(x.slot_cnt + slot) < x.gu_tiles) {
-                if (global_timer_ns() - t0 > kWaitLimitNs) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok) ready_slot = slot;
-        }
-        // B fragments: this expert's h rows, loaded before waiting on the stage
-#pragma unroll
-        for (int i = 0; i < kMaxDW; ++i) {
-            const int grp = g_lo + i;
-            if (ok && grp < g_hi && r < sl.ntok) {
-                load_b(bdn[i], a.hp + (int64_t)(sl.list_begin + r) * a.I + grp * kGroup + c * 16);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) bdn[i][q] = 0u;
-            }
-        }
-    }
-    if (!ok || !mbar_wait(&x.full[stage], use & 1)) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (!mbar_wait(&x.S.full[stage], use & 1)) {
         fail(x, lane);
         return false;
     }
-    const uint8_t* st = x.stage0 + (size_t)stage * L.stage_bytes;
-    if (sl.valid) {
-        if constexpr (kGU) {
-            const uint16_t* scA = reinterpret_cast<const uint16_t*>(st + L.gu_scale) + r * G;
-            const uint16_t* scB = reinterpret_cast<const uint16_t*>(st + L.gu_scale) + (8 + r) * G;
+    const uint8_t* st = x.S.stage0 + (size_t)stage * L.stage_bytes;
+    if (valid) {
+        const uint16_t* scA = reinterpret_cast<const uint16_t*>(st + 2 * L.gu_op) + r * L.gGp;
+        const uint16_t* scB = reinterpret_cast<const uint16_t*>(st + 2 * L.gu_op + L.gu_sc) + r * L.gGp;
+        // three independent MMA chains at a time.  A group past the end of
+        // H (the last warp's) has a zero B fragment, a zero offset sum and a
+        // zero scale, and reads real staged codes.
 #pragma unroll
-            for (int i = 0; i < kMaxGW; ++i) {
-                const int grp = g_lo + i;
-                if (grp >= g_hi) break;
-                const uint2 wa = load_codes(st, r, L.gu_segs, grp, c);
-                const uint2 wb = load_codes(st + L.gu_op, r, L.gu_segs, grp, c);
-                const float fa = bf16f(scA[grp]), fb = bf16f(scB[grp]);
-                const float cr0 = x.corr_s[(2 * c) * G + grp], cr1 = x.corr_s[(2 * c + 1) * G + grp];
-                float part[4];
-                group_partial<false>(part, wa, wb, breg[i]);
-                acc[0][0] = fmaf(fa, part[0] - cr0, acc[0][0]);
-                acc[0][1] = fmaf(fa, part[1] - cr1, acc[0][1]);
-                acc[0][2] = fmaf(fb, part[2] - cr0, acc[0][2]);
-                acc[0][3] = fmaf(fb, part[3] - cr1, acc[0][3]);
+        for (int i0 = 0; i0 < kMaxGW; i0 += 3) {
+            uint2 wa[3], wb[3];
+            float part[3][4], fa[3], fb[3];
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+                const int i = i0 + u, grp = g_lo + i;
+                wa[u] = *reinterpret_cast<const uint2*>(st + coff[i]);
+                wb[u] = *reinterpret_cast<const uint2*>(st + L.gu_op + coff[i]);
+                const float2 cr = *reinterpret_cast<const float2*>(x.S.corr + grp * 8 + 2 * c);
+                part[u][0] = -cr.x;
+                part[u][1] = -cr.y;
+                part[u][2] = -cr.x;
+                part[u][3] = -cr.y;
+                fa[u] = bf16f(scA[grp]);
+                fb[u] = bf16f(scB[grp]);
             }
-        } else {
-            const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + L.dn_scale);
 #pragma unroll
-            for (int i = 0; i < kMaxDW; ++i) {
-                const int grp = g_lo + i;
-                if (grp >= g_hi) break;
+            for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the group
+                uint32_t ae[3], ao[3], be[3], bo[3];
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    const uint2 wa = load_codes(st, m * 16 + r, L.dn_segs, grp, c);
-                    const uint2 wb = load_codes(st, m * 16 + 8 + r, L.dn_segs, grp, c);
-                    const float fa = bf16f(sc[(m * 16 + r) * G + grp]);
-                    const float fb = bf16f(sc[(m * 16 + 8 + r) * G + grp]);
-                    float part[4];
-                    group_partial<true>(part, wa, wb, bdn[i]);
-                    acc[m][0] = fmaf(fa, part[0], acc[m][0]);
-                    acc[m][1] = fmaf(fa, part[1], acc[m][1]);
-                    acc[m][2] = fmaf(fb, part[2], acc[m][2]);
-                    acc[m][3] = fmaf(fb, part[3], acc[m][3]);
+                for (int u = 0; u < 3; ++u) {
+                    unpack_raw_step((ks >> 1) ? wa[u].y : wa[u].x, ks & 1, ae[u], ao[u]);
+                    unpack_raw_step((ks >> 1) ? wb[u].y : wb[u].x, ks & 1, be[u], bo[u]);
                 }
+#pragma unroll
+                for (int u = 0; u < 3; ++u)
+                    mma16816(part[u], part[u], ae[u], be[u], ao[u], bo[u],
+                             breg[i0 + u][2 * ks], breg[i0 + u][2 * ks + 1]);
+            }
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+                acc[0] = fmaf(fa[u], part[u][0], acc[0]);
+                acc[1] = fmaf(fa[u], part[u][1], acc[1]);
+                acc[2] = fmaf(fb[u], part[u][2], acc[2]);
+                acc[3] = fmaf(fb[u], part[u][3], acc[3]);
             }
         }
     }
-    // the stage is no longer read by this warp
     __syncwarp();
-    if (lane == 0) mbar_arrive(&x.empty[stage]);
+    if (lane == 0) mbar_arrive(&x.S.empty[stage]);
 
-    // partials -> reduction buffer rb (free once item j - 2's epilogue read it)
-    if (ruse > 0 && !mbar_wait(&x.red_empty[rb], (ruse - 1) & 1)) {
+    float v[4];
+    const int red = reduce_item(x, j, acc, v);
+    if (red < 0) {
         fail(x, lane);
         return false;
     }
-    float* rbuf = x.red + rb * (kCW * 2 * 4 * 32);
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) rbuf[((warp * 2 + m) * 4 + q) * 32 + lane] = acc[m][q];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&x.red_full[rb]);
-
-    if (warp != j % kCW) return true;
-    // --------------------- epilogue of this item (one warp) ---------------------
-    if (!mbar_wait(&x.red_full[rb], ruse & 1)) {
-        fail(x, lane);
-        return false;
+    if (red == 0 || !valid) return true;
+    if (pend_n > 0 && pend_slot != slot) {
+        publish(x, pend_slot, pend_n);
+        pend_n = 0;
     }
-    float v[2][4];
+    // ---- epilogue (one warp): h' = w * silu(g) * u for the slot's tokens ----
+    const int n = tile * kGuRows + r;
+    const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
+    const int list_begin = en->list_begin;
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < kCW; ++w) s += rbuf[((w * 2 + m) * 4 + q) * 32 + lane];
-            v[m][q] = s;
+    for (int e2 = 0; e2 < 2; ++e2) {
+        const int t = 2 * c + e2;
+        if (t >= a.T) continue;
+        const int p = en->pos[t];
+        if (p < 0) continue;
+        const float gv = v[e2], uv = v[2 + e2];
+        float h = en->w[t] * (gv / (1.f + expf(-gv)) * uv);
+        if (fabsf(h) > 65504.f) {
+            report(a.status, COLI_ERR_RANGE);
+            h = copysignf(65504.f, h);
         }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&x.red_empty[rb]);
-    const int P = a.T * a.k;
-    if constexpr (kGU) {
-        if (!sl.valid) return true;
-        // columns are tokens 0..7: find each token's row on this expert's list
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-            const int t = 2 * c + e2;
-            int orow = -1;
-            if (t < a.T) {
-                if (sl.shared) {
-                    orow = sl.list_begin + t;
-                } else {
-                    for (int i = 0; i < sl.ntok; ++i)
-                        if (a.pairs[sl.list_begin + i] / a.k == t) orow = sl.list_begin + i;
-                }
-            }
-            if (orow < 0) continue;
-            const int n = tile * 8 + r;
-            const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
-            const float gv = v[0][e2], uv = v[0][2 + e2];
-            float h = gv / (1.f + expf(-gv)) * uv;
-            if (fabsf(h) > 65504.f) {
-                report(a.status, COLI_ERR_RANGE);
-                h = copysignf(65504.f, h);
-            }
-            a.hp[(int64_t)orow * a.I + hcol] = __float2half_rn(h);
-        }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(x.slot_cnt + slot, 1);
-    } else {
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-            const int i_tok = 2 * c + e2;  // column = position on the expert's list
-            if (!sl.valid || i_tok >= sl.ntok) continue;
-            float* yrow = a.y + (int64_t)(sl.list_begin + i_tok) * a.H + tile * kDnRows;
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                yrow[m * 16 + r] = v[m][e2];
-                yrow[m * 16 + 8 + r] = v[m][2 + e2];
-            }
-        }
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = atomicAdd(x.tile_cnt + tile, 1) == x.n_slots - 1;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            __threadfence();
-            // combine rows [tile * 32, +32) of every token, fixed order
-            for (int idx = lane; idx < a.T * kDnRows; idx += 32) {
-                const int t = idx / kDnRows, m = tile * kDnRows + idx % kDnRows;
-                float o = 0.f;
-                for (int jj = 0; jj < a.k; ++jj) {
-                    const int s = a.inv[t * a.k + jj];
-                    if (s < 0 || s >= P) {
-                        report(a.status, COLI_ERR_BAD_INDEX);
-                        continue;
-                    }
-                    o = fmaf(a.topk_w[t * a.k + jj], __ldcg(a.y + (int64_t)s * a.H + m), o);
-                }
-                for (int sh = 0; sh < a.n_shared; ++sh)
-                    o += __ldcg(a.y + (int64_t)(P + sh * a.T + t) * a.H + m);
-                const int64_t oi = (int64_t)t * a.H + m;
-                if (a.out_bf16) {
-                    if (a.residual)
-                        o += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.residual)[oi]);
-                    reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(o);
-                } else {
-                    if (a.residual) o += reinterpret_cast<const float*>(a.residual)[oi];
-                    reinterpret_cast<float*>(a.out)[oi] = o;
-                }
-            }
-        }
+        a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn(h);
     }
+    pend_slot = slot;
+    ++pend_n;
     return true;
 }
 
+// h' fragments of one slot for this warp's down groups (columns = tokens;
+// zero where a token is not on the slot's list or the group is past I).
+__device__ __forceinline__ void load_down_b(const FfnArgs& a, const SlotEntry* en, int g_lo,
+                                            uint32_t (&bdn)[kMaxDW][8]) {
+    const int g_hi = a.I / kGroup;
+    const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+    const int p = (r < a.T && en->e >= 0) ? en->pos[r] : -1;
+    const __half* row = a.hp + (int64_t)(en->list_begin + (p < 0 ? 0 : p)) * a.I;
+#pragma unroll
+    for (int i = 0; i < kMaxDW; ++i) {
+        const int grp = g_lo + i;
+        if (p >= 0 && grp < g_hi) {
+            load_b_cg(bdn[i], row + grp * kGroup + c * 16);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) bdn[i][q] = 0u;
+        }
+    }
+}
+
+// True once all gate/up tiles of slot s are published (an invalid slot has
+// nothing to wait for).  Relaxed read.
+__device__ __forceinline__ bool slot_ready(const Ctx& x, int s) {
+    return x.S.table[s].e < 0 || ld_relaxed(x.sync + 1 + s) >= x.gu_tiles;
+}
+
+// Move `frontier` (slots [0, frontier) are complete and their h' visible to
+// this warp) past slot `need`: the lanes poll 32 slots at once, the frontier
+// jumps over the leading complete ones, and one fence orders every later h'
+// read after those observations.  Bounded wait; false on timeout or abort.
+__device__ __forceinline__ bool advance_frontier(const Ctx& x, int& frontier, int need) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t t0 = global_timer_ns();
+    while (frontier <= need) {
+        const int s = frontier + lane;
+        const unsigned done = __ballot_sync(0xffffffffu, s >= x.n_slots || slot_ready(x, s));
+        frontier += done == 0xffffffffu ? 32 : __ffs(~done) - 1;
+        if (frontier > need) break;
+        if (*x.S.abort_flag) return false;
+        __nanosleep(256);
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            fail(x, lane);
+            return false;
+        }
+    }
+    fence_acq_rel_gpu();
+    return true;
+}
+
+// One down stage: this CTA's tiles of slot s's W_d, accumulated into acc.
+__device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt,
+                                           const uint32_t (&bcur)[kMaxDW][8],
+                                           const int (&dcoff)[kMaxDW], int g_lo,
+                                           float (&acc)[kMaxMT][4]) {
+    const Layout& L = x.L;
+    const int lane = threadIdx.x & 31, r = lane >> 2;
+    if (*x.S.abort_flag) return false;
+    const int stage = j % kStagesD, use = j / kStagesD;
+    if (!mbar_wait(&x.S.full[stage], use & 1)) {
+        fail(x, lane);
+        return false;
+    }
+    const uint8_t* st = x.S.stage0 + (size_t)stage * L.stage_bytes;
+    if (x.S.table[s].e >= 0) {
+        // per group, the three tiles' MMA chains run interleaved.  A group past
+        // the end of I has a zero B fragment and a zero scale (padding
+        // column) and reads real staged codes, so it adds zero; a tile this
+        // CTA does not own (m >= my_mt) computes on stale stage bytes into an
+        // accumulator that is never read.  Row r + 8 of a tile sits 8 staged
+        // rows after row r.
+        const int row8 = 8 * L.dn_segs * 128;
+        const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(st + kMaxMT * L.dn_op) + r * L.dGp;
+#pragma unroll
+        for (int i = 0; i < kMaxDW; ++i) {
+            const int gs = g_lo + i;
+            uint2 wa[kMaxMT], wb[kMaxMT];
+            float part[kMaxMT][4];
+#pragma unroll
+            for (int m = 0; m < kMaxMT; ++m) {
+                const uint8_t* codes = st + m * L.dn_op + dcoff[i];
+                wa[m] = *reinterpret_cast<const uint2*>(codes);
+                wb[m] = *reinterpret_cast<const uint2*>(codes + row8);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) part[m][q] = 0.f;
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t ae[kMaxMT], ao[kMaxMT], be[kMaxMT], bo[kMaxMT];
+#pragma unroll
+                for (int m = 0; m < kMaxMT; ++m) {
+                    unpack_exact_step((ks >> 1) ? wa[m].y : wa[m].x, ks & 1, ae[m], ao[m]);
+                    unpack_exact_step((ks >> 1) ? wb[m].y : wb[m].x, ks & 1, be[m], bo[m]);
+                }
+#pragma unroll
+                for (int m = 0; m < kMaxMT; ++m)
+                    mma16816(part[m], part[m], ae[m], be[m], ao[m], bo[m], bcur[i][2 * ks],
+                             bcur[i][2 * ks + 1]);
+            }
+#pragma unroll
+            for (int m = 0; m < kMaxMT; ++m) {
+                const uint16_t* sc = sc0 + m * (L.dn_sc / 2) + gs;
+                const float fa = bf16f(sc[0]);
+                const float fb = bf16f(sc[8 * L.dGp]);
+                acc[m][0] = fmaf(fa, part[m][0], acc[m][0]);
+                acc[m][1] = fmaf(fa, part[m][1], acc[m][1]);
+                acc[m][2] = fmaf(fb, part[m][2], acc[m][2]);
+                acc[m][3] = fmaf(fb, part[m][3], acc[m][3]);
+            }
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&x.S.empty[stage]);
+    return true;
+}
+
+template <int NV>
 __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const DecodeArgs d) {
     const FfnArgs& a = d.f;
-    const Layout L = make_layout(a.H, a.I);
+    const Layout L = make_layout(a.H, a.I, d.max_slots);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + kStagesD;
-    uint64_t* red_full = empty + kStagesD;
-    uint64_t* red_empty = red_full + kRedBufs;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 512);
-    float* red = reinterpret_cast<float*>(smem + L.red_off);  // [2][8 warps][2 mt][4][32]
-    float* corr_s = reinterpret_cast<float*>(smem + L.corr_off);  // [8 tokens][H/64]
-    uint8_t* stage0 = smem + L.stage_off;
+    const Smem S = carve(smem, L);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesD; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kCW);
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], kCW);
         }
         for (int b = 0; b < kRedBufs; ++b) {
-            mbar_init(&red_full[b], kCW);
-            mbar_init(&red_empty[b], 1);
+            mbar_init(&S.red_empty[b], 1);
+            S.red_cnt[b] = 0;
         }
-        *abort_flag = 0;
+        mbar_init(S.tbl_ready, 1);
+        *S.abort_flag = 0;
         fence_barrier_init();
     }
     __syncthreads();
     pdl_launch_dependents();
 
-    const int gG = a.H / kGroup, dG = a.I / kGroup;
-    const int gu_tiles = a.I / 8, dn_tiles = a.H / kDnRows;
-    int* slot_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(a.status) + kSlotCntOffset);
-    int* tile_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(a.status) + kTileCntOffset);
+    const int G = gridDim.x, b = blockIdx.x;
+    const int gu_tiles = a.I / kGuRows;
+    const int n_mt = a.H / kDnRows;
+    const int bm = G - 1 - b;  // this CTA's down tiles: bm, bm + G, ...
+    const int my_mt = bm < n_mt ? (n_mt - 1 - bm) / G + 1 : 0;
 
     if (warp == kCW) {
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
             const uint64_t policy = policy_evict_first();
-            const int64_t shared_gu = (int64_t)a.n_shared * gu_tiles;
-            int64_t n_gu = -1, n_all = -1;
-            int n_act = 0;
+            const int n_gu_shared = a.n_shared * gu_tiles;
+            int n_slots = -1;
             int j = 0;
-            bool aborted = false;
-            for (int64_t item = blockIdx.x;; item += gridDim.x, ++j) {
-                if (n_all < 0 && item >= shared_gu) {
-                    pdl_wait();
-                    n_act = *reinterpret_cast<const volatile int*>(a.n_active);
-                    if (n_act < 0 || n_act > a.E) n_act = 0;
-                    n_gu = (int64_t)(n_act + a.n_shared) * gu_tiles;
-                    n_all = n_gu + (int64_t)(n_act + a.n_shared) * dn_tiles;
-                }
-                if (n_all >= 0 && item >= n_all) break;
-                if (*abort_flag) break;
-                const int stage = j % kStagesD, use = j / kStagesD;
-                if (use > 0 && !mbar_wait(&empty[stage], (use - 1) & 1)) {
+            bool stop = false;
+            auto table_known = [&]() -> bool {
+                if (n_slots >= 0) return true;
+                if (!mbar_wait(S.tbl_ready, 0)) {
                     report(a.status, COLI_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    aborted = true;
+                    *S.abort_flag = 1;
+                    return false;
+                }
+                n_slots = *S.n_slots;
+                return true;
+            };
+            auto next_stage = [&](uint8_t*& st) -> bool {
+                const int stage = j % kStagesD, use = j / kStagesD;
+                if (use > 0 && !mbar_wait(&S.empty[stage], (use - 1) & 1)) {
+                    report(a.status, COLI_ERR_TIMEOUT);
+                    *S.abort_flag = 1;
+                    return false;
+                }
+                st = S.stage0 + (size_t)stage * L.stage_bytes;
+                return true;
+            };
+            for (int item = b;; item += G) {
+                if (item >= n_gu_shared && !table_known()) {
+                    stop = true;
                     break;
                 }
+                if (n_slots >= 0 && item >= n_slots * gu_tiles) break;
+                uint8_t* st;
+                if (*S.abort_flag || !next_stage(st)) {
+                    stop = true;
+                    break;
+                }
+                uint64_t* bar = &S.full[j % kStagesD];
+                ++j;
                 if (item == a.withhold_item) continue;  // test hook: this stage never fills
-                const bool gu = n_gu < 0 || item < n_gu;
-                const int64_t local = gu ? item : item - n_gu;
-                const int tiles = gu ? gu_tiles : dn_tiles;
-                const SlotD sl = slot_of(a, (int)(local / tiles), n_act);
-                uint8_t* st = stage0 + (size_t)stage * L.stage_bytes;
-                if (!sl.valid) {
-                    mbar_arrive(&full[stage]);
+                const int slot = item / gu_tiles, tile = item - slot * gu_tiles;
+                const int e = slot < a.n_shared ? a.E + slot : S.table[slot].e;
+                if (e < 0) {
+                    mbar_arrive(bar);
                     continue;
                 }
-                const int tile = (int)(local % tiles);
-                const DevExpert ex = a.experts[sl.e];
-                const CUtensorMap* maps = d.maps + (size_t)sl.e * 3;
-                if (gu) {
-                    mbar_arrive_expect_tx(&full[stage], L.gu_tx);
-                    const int n0 = tile * 8;
-                    tma_load_3d(st, maps + 0, 0, 0, n0, &full[stage], policy);
-                    tma_load_3d(st + L.gu_op, maps + 1, 0, 0, n0, &full[stage], policy);
-                    bulk_g2s_evict_first(st + L.gu_scale, ex.gate_s + (int64_t)n0 * gG, 8 * gG * 2,
-                                         &full[stage], policy);
-                    bulk_g2s_evict_first(st + L.gu_scale + 8 * gG * 2, ex.up_s + (int64_t)n0 * gG,
-                                         8 * gG * 2, &full[stage], policy);
-                } else {
-                    mbar_arrive_expect_tx(&full[stage], L.dn_tx);
-                    const int m0 = tile * kDnRows;
-                    tma_load_3d(st, maps + 2, 0, 0, m0, &full[stage], policy);
-                    bulk_g2s_evict_first(st + L.dn_scale, ex.down_s + (int64_t)m0 * dG,
-                                         kDnRows * dG * 2, &full[stage], policy);
+                const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
+                const int n0 = tile * kGuRows;
+                mbar_arrive_expect_tx(bar, L.gu_tx);
+                tma_load_3d(st, maps + 0, 0, 0, n0, bar, policy);
+                tma_load_3d(st + L.gu_op, maps + 1, 0, 0, n0, bar, policy);
+                tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
+                tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
+            }
+            if (!stop && my_mt > 0 && table_known()) {
+                for (int s = 0; s < n_slots; ++s) {
+                    uint8_t* st;
+                    if (*S.abort_flag || !next_stage(st)) break;
+                    uint64_t* bar = &S.full[j % kStagesD];
+                    ++j;
+                    const int e = S.table[s].e;
+                    if (e < 0) {
+                        mbar_arrive(bar);
+                        continue;
+                    }
+                    const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
+                    mbar_arrive_expect_tx(bar, my_mt * (L.dn_op + L.dn_sc));
+                    for (int m = 0; m < my_mt; ++m) {
+                        const int m0 = (bm + m * G) * kDnRows;
+                        tma_load_3d(st + m * L.dn_op, maps + 2, 0, 0, m0, bar, policy);
+                        tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0, bar,
+                                    policy);
+                    }
                 }
             }
-            if (aborted || *abort_flag) {
+            if (*S.abort_flag) {
                 // let the copies already issued land before the CTA goes away
                 for (int back = 1; back <= kStagesD && back <= j; ++back) {
                     const int jj = j - back;
-                    (void)mbar_wait(&full[jj % kStagesD], (jj / kStagesD) & 1);
+                    (void)mbar_wait(&S.full[jj % kStagesD], (jj / kStagesD) & 1);
                 }
             }
         }
@@ -544,77 +792,201 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
 
     // -------------------------------- consumers --------------------------------
     pdl_wait();
-    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
-    if (n_act < 0 || n_act > a.E) {
-        if (threadIdx.x == 0) report(a.status, COLI_ERR_BAD_INDEX);
-        n_act = 0;
+    // logits -> shared memory (the reduction buffers are free until the first
+    // item); they land while the activation operand is built
+    if (d.logits) {
+        const int n = a.T * a.E;
+        for (int i = threadIdx.x; i < n; i += kConsumerThreads) cp_async4(S.red + i, d.logits + i);
+        cp_async_commit();
     }
-    const int n_slots = n_act + a.n_shared;
-    const int64_t n_gu = (int64_t)n_slots * gu_tiles;
-    const int64_t n_all = n_gu + (int64_t)n_slots * dn_tiles;
     const int r = lane >> 2, c = lane & 3;
 
-    // gate/up activation fragments of all T tokens (columns) and offset sums
-    const int gg_lo = (gG * warp) / kCW, gg_hi = (gG * (warp + 1)) / kCW;
+    // gate/up operand: all T tokens as MMA columns, this warp's kMaxGW
+    // groups, in registers for the whole kernel; offset sums to shared memory
+    // (zero for the groups past the end of H)
+    const int gG = a.H / kGroup;
+    const int gg_lo = kMaxGW * warp;
     uint32_t breg[kMaxGW][8];
+    int coff[kMaxGW];
+    float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < kMaxGW; ++i) {
         const int grp = gg_lo + i;
-        if (grp < gg_hi && r < a.T) {
-            load_b(breg[i], a.xp + (int64_t)r * a.H + grp * kGroup + c * 16);
+        const bool in = grp < gG;
+        coff[i] = code_offset(r, L.gu_segs, in ? grp : gG - 1, c);
+        if (in && r < a.T) {
+            x_fragment(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)r * a.H + grp * kGroup +
+                           c * 16,
+                       breg[i], amax);
         } else {
 #pragma unroll
             for (int q = 0; q < 8; ++q) breg[i][q] = 0u;
         }
+        float cs[4];
+        offset_sums(breg[i], cs);
+        if (r == 0) {
+            S.corr[grp * 8 + 2 * c] = cs[0];
+            S.corr[grp * 8 + 2 * c + 1] = cs[1];
+        }
     }
-    for (int i = threadIdx.x; i < 8 * gG; i += kCW * 32)
-        corr_s[i] = (i / gG) < a.T ? a.corr[i] : 0.f;
-    named_barrier(1, kCW * 32);
+    if (amax > 65504.f) report(a.status, COLI_ERR_RANGE);
+    if (d.logits) cp_async_wait_all();
+    consumers_sync();
 
-    int ready_slot = -1;  // down: highest slot whose h this warp has seen complete
+    if (d.logits) table_from_logits<NV>(d, S, S.red);
+    else table_from_union(d, S);
+    consumers_sync();
+    if (threadIdx.x == 0) mbar_arrive(S.tbl_ready);
+    const int n_slots = *S.n_slots;
+    const Ctx ctx{a, L, S, d.sync, n_slots, gu_tiles};
+
+    // phase 1: gate/up items
     int j = 0;
-    Ctx ctx{a, L, stage0, full, empty, red_full, red_empty, abort_flag, red, corr_s,
-            slot_cnt, tile_cnt, n_act, n_slots, gu_tiles, dn_tiles, gG, dG};
-    // phase 1: gate/up items (activation fragments live in registers)
-    int64_t item = blockIdx.x;
-    for (; item < n_gu; item += gridDim.x, ++j)
-        if (!consume_item<true>(ctx, item, j, breg, ready_slot)) return;
-    // phase 2: down items
-    for (; item < n_all; item += gridDim.x, ++j)
-        if (!consume_item<false>(ctx, item - n_gu, j, breg, ready_slot)) return;
+    bool alive = true;
+    const int n_gu = n_slots * gu_tiles;
+    int pend_slot = -1, pend_n = 0;
+    for (int item = b; item < n_gu && alive; item += G, ++j)
+        alive = gateup_item(ctx, item, j, breg, coff, gg_lo, pend_slot, pend_n);
+    if (pend_n > 0) publish(ctx, pend_slot, pend_n);
+
+    // phase 2: down + combine over this CTA's output tiles, slot by slot;
+    // h' fragments of the next slot are loaded while this one is computed
+    const int dG = a.I / kGroup;
+    const int dg_lo = kMaxDW * warp;
+    float acc[kMaxMT][4];
+#pragma unroll
+    for (int m = 0; m < kMaxMT; ++m)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
+    if (alive && my_mt > 0 && n_slots > 0) {
+        int dcoff[kMaxDW];
+#pragma unroll
+        for (int i = 0; i < kMaxDW; ++i)
+            dcoff[i] = code_offset(r, L.dn_segs, dg_lo + i < dG ? dg_lo + i : dG - 1, c);
+        // h' fragments: b0 = this slot, b1 = the next one (loading)
+        uint32_t b0[kMaxDW][8], b1[kMaxDW][8];
+        int frontier = 0;
+        alive = advance_frontier(ctx, frontier, 0);
+        if (alive) load_down_b(a, S.table + 0, dg_lo, b1);
+        for (int s = 0; s < n_slots && alive; ++s, ++j) {
+#pragma unroll
+            for (int i = 0; i < kMaxDW; ++i)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) b0[i][q] = b1[i][q];
+            if (s + 1 < n_slots) {
+                if (frontier <= s + 1) alive = advance_frontier(ctx, frontier, s + 1);
+                if (alive) load_down_b(a, S.table + s + 1, dg_lo, b1);
+            }
+            if (alive) alive = down_stage(ctx, s, j, my_mt, b0, dcoff, dg_lo, acc);
+        }
+    }
+
+    // final: sum the warps' partials in a fixed order, add the residual
+    consumers_sync();  // every gate/up reduction is done with the buffers
+    if (my_mt > 0) {
+#pragma unroll
+        for (int m = 0; m < kMaxMT; ++m)
+            if (m < my_mt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    S.red[((warp * kMaxMT + m) * 4 + q) * 32 + lane] = acc[m][q];
+    }
+    consumers_sync();
+    if (my_mt > 0 && !*S.abort_flag) {
+        const int per_t = my_mt * kDnRows;
+        for (int o = threadIdx.x; o < a.T * per_t; o += kConsumerThreads) {
+            const int t = o / per_t, rem = o - t * per_t;
+            const int m = rem / kDnRows, row = rem - m * kDnRows;
+            const int src_lane = (row & 7) * 4 + (t >> 1);
+            const int q = (row >> 3) * 2 + (t & 1);
+            float y = 0.f;
+#pragma unroll
+            for (int w = 0; w < kCW; ++w) y += S.red[((w * kMaxMT + m) * 4 + q) * 32 + src_lane];
+            const int64_t oi = (int64_t)t * a.H + (bm + m * G) * kDnRows + row;
+            if (a.out_bf16) {
+                if (a.residual)
+                    y += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.residual)[oi]);
+                reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(y);
+            } else {
+                if (a.residual) y += reinterpret_cast<const float*>(a.residual)[oi];
+                reinterpret_cast<float*>(a.out)[oi] = y;
+            }
+        }
+    }
+    // the last CTA to get here returns the counters to zero
+    if (threadIdx.x == 0) {
+        fence_acq_rel_gpu();
+        if (atomicAdd(d.sync, 1) == G - 1) {
+            fence_acq_rel_gpu();
+            for (int s = 0; s < n_slots; ++s) d.sync[1 + s] = 0;
+            d.sync[0] = 0;
+        }
+    }
+}
+
+template <int NV>
+cudaError_t launch_nv(const DecodeArgs& d, int blocks, int smem, cudaStream_t st) {
+    cudaError_t err = cudaFuncSetAttribute(decode_fused_kernel<NV>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(kThreadsD);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+}
+
+int max_slots_for(int E, int k, int T, int n_shared) {
+    return std::min(E, T * k) + n_shared;
 }
 
 }  // namespace
 
-bool decode_supported(int H, int I, int T) {
-    if (T < 1 || T > 8 || H % 256 || I % 256) return false;
-    const Layout L = make_layout(H, I);
+bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_sms) {
+    if (T < 1 || T > 8 || T * k > kMaxPairs || H % 512 || I % 512 || num_sms < 1) return false;
+    // the slot counters live between the two counter offsets of the header
+    if (1 + max_slots_for(E, k, T, n_shared) > (int)((kTileCntOffset - kSlotCntOffset) / 4))
+        return false;
+    const Layout L = make_layout(H, I, max_slots_for(E, k, T, n_shared));
     if (L.smem > kSmemLimitD) return false;
-    if ((H / kGroup + kCW - 1) / kCW > kMaxGW) return false;
-    if ((I / kGroup + kCW - 1) / kCW > kMaxDW) return false;
-    return L.gu_segs <= 256 && L.dn_segs <= 256;
+    if (H / kGroup > kCW * kMaxGW || I / kGroup > kCW * kMaxDW) return false;
+    if (T * E > kRedFloats) return false;  // logits staged in the reduction buffers
+    if (H / kDnRows > kMaxMT * num_sms) return false;
+    return L.gu_segs <= 256 && L.dn_segs <= 256 && L.gGp <= 256 && L.dGp <= 256;
 }
 
 cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I,
                               CUtensorMap** d_maps) {
     *d_maps = nullptr;
-    const Layout L = make_layout(H, I);
-    CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * 3];
+    const Layout L = make_layout(H, I, 0);
+    CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * kMaps];
     if (!maps) return cudaErrorMemoryAllocation;
     bool ok = true;
+    const int gG = H / kGroup, dG = I / kGroup;
     for (int e = 0; e < n && ok; ++e) {
         const DevExpert& x = host_experts[e];
-        ok = encode_tma(&maps[e * 3 + 0], x.gate_q, 3, I, H / 2, L.gu_segs, 8) &&
-             encode_tma(&maps[e * 3 + 1], x.up_q, 3, I, H / 2, L.gu_segs, 8) &&
-             encode_tma(&maps[e * 3 + 2], x.down_q, 3, H, I / 2, L.dn_segs, kDnRows);
+        CUtensorMap* m = maps + (size_t)e * kMaps;
+        ok = encode_tma(&m[0], x.gate_q, 3, I, H / 2, L.gu_segs, kGuRows) &&
+             encode_tma(&m[1], x.up_q, 3, I, H / 2, L.gu_segs, kGuRows) &&
+             encode_tma(&m[2], x.down_q, 3, H, I / 2, L.dn_segs, kDnRows) &&
+             encode_tma_rows_u16(&m[3], x.gate_s, I, gG, L.gGp, kGuRows) &&
+             encode_tma_rows_u16(&m[4], x.up_s, I, gG, L.gGp, kGuRows) &&
+             encode_tma_rows_u16(&m[5], x.down_s, H, dG, L.dGp, kDnRows);
     }
     if (!ok) {
         delete[] maps;
         return cudaErrorInvalidValue;
     }
-    cudaError_t err = cudaMalloc(d_maps, sizeof(CUtensorMap) * (size_t)n * 3);
+    cudaError_t err = cudaMalloc(d_maps, sizeof(CUtensorMap) * (size_t)n * kMaps);
     if (err == cudaSuccess)
-        err = cudaMemcpy(*d_maps, maps, sizeof(CUtensorMap) * (size_t)n * 3, cudaMemcpyHostToDevice);
+        err = cudaMemcpy(*d_maps, maps, sizeof(CUtensorMap) * (size_t)n * kMaps,
+                         cudaMemcpyHostToDevice);
     delete[] maps;
     if (err != cudaSuccess && *d_maps) {
         cudaFree(*d_maps);
@@ -623,31 +995,21 @@ cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I
     return err;
 }
 
-cudaError_t launch_decode_fused(const FfnArgs& f, const CUtensorMap* maps, int num_sms,
-                                cudaStream_t st) {
-    DecodeArgs d;
-    d.f = f;
+cudaError_t launch_decode_fused(const DecodeArgs& d0, int num_sms, cudaStream_t st) {
+    DecodeArgs d = d0;
     d.f.withhold_item = take_withhold_item();
-    d.maps = maps;
-    const Layout L = make_layout(f.H, f.I);
-    cudaError_t err = cudaFuncSetAttribute(decode_fused_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, L.smem);
-    if (err != cudaSuccess) return err;
-    const int64_t max_slots = std::min<int64_t>(f.E, (int64_t)f.T * f.k) + f.n_shared;
-    const int64_t items = max_slots * (f.I / 8 + f.H / kDnRows);
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, items));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(kThreadsD);
-    cfg.dynamicSmemBytes = L.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    d.max_slots = max_slots_for(d.f.E, d.f.k, d.f.T, d.f.n_shared);
+    const Layout L = make_layout(d.f.H, d.f.I, d.max_slots);
+    const int blocks = num_sms;  // persistent: one CTA per SM, all resident
     profile_mark(1, st);
-    err = cudaLaunchKernelEx(&cfg, decode_fused_kernel, d);
+    cudaError_t err;
+    const int nv = d.logits ? (d.f.E + 31) / 32 : 1;
+    if (nv <= 1) err = launch_nv<1>(d, blocks, L.smem, st);
+    else if (nv <= 2) err = launch_nv<2>(d, blocks, L.smem, st);
+    else if (nv <= 4) err = launch_nv<4>(d, blocks, L.smem, st);
+    else if (nv <= 8) err = launch_nv<8>(d, blocks, L.smem, st);
+    else if (nv <= 16) err = launch_nv<16>(d, blocks, L.smem, st);
+    else err = launch_nv<32>(d, blocks, L.smem, st);
     profile_mark(2, st);
     profile_mark(3, st);
     profile_mark(4, st);

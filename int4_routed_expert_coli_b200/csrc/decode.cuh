@@ -11,23 +11,36 @@ constexpr int kMaxGW = 9;   // gate/up scale groups per consumer warp (H <= 6336
 constexpr int kMaxDW = 3;   // down scale groups per consumer warp (I <= 2112)
 
 struct DecodeArgs {
-    FfnArgs f;
-    const CUtensorMap* maps;  // [experts][3]: gate, up (8-row boxes), down (32-row box)
+    FfnArgs f;                // shapes, experts, x, the union (when logits is null), h rows,
+                              // residual, out, status
+    // [experts][6]: gate, up (8-row boxes), down (16-row box) codes; then
+    // the same three scale matrices (rows padded to 8 x odd bf16 columns)
+    const CUtensorMap* maps;
+    const float* logits;      // [T][E]: route inside the kernel; null: f holds the union
+    int32_t* idx_out;         // [T][k] nullable: the routing (with logits)
+    float* w_out;             // [T][k] nullable
+    int* sync;                // [0] finished CTAs, [1 + s] finished gate/up tiles of slot s;
+                              // zero on entry, left zero on exit
+    int max_slots;            // bound on shared + active experts (sizes the slot table)
 };
 
-// True when a call with T tokens can run the fused decode kernel.
-bool decode_supported(int H, int I, int T);
-// 3-D swizzled tensor maps of every expert's packed code matrices.
+// True when a call with T tokens can run the fused decode kernel on a GPU
+// with num_sms SMs.
+bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_sms);
+// Tensor maps of every expert's packed code matrices (3-D, swizzled) and
+// scale matrices (2-D, padded rows).
 cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I,
                               CUtensorMap** d_maps);
-// gate/up + down + combine in one launch; the union, inverse map, operand
-// copy of x and zeroed counters must be ready (prep kernel).
-cudaError_t launch_decode_fused(const FfnArgs& f, const CUtensorMap* maps, int num_sms,
-                                cudaStream_t st);
+// Routing (or the given union), gate/up, down and combine in one launch.
+cudaError_t launch_decode_fused(const DecodeArgs& d, int num_sms, cudaStream_t st);
 // Encode a 3-D uint8 tensor map over a [rows][row_bytes] matrix viewed as
 // [rows][row_bytes / 128][128], box {128, segs, box_rows}, 128-byte swizzle;
 // chunks past the row end read as zero.
 bool encode_tma(CUtensorMap* m, const void* base, int rank, int rows, int row_bytes, int segs,
                 int box_rows);
+// Encode a 2-D 16-bit tensor map over a [rows][cols] matrix (cols a multiple
+// of 8), box {box_cols, box_rows}; columns past cols read as zero.
+bool encode_tma_rows_u16(CUtensorMap* m, const void* base, int rows, int cols, int box_cols,
+                         int box_rows);
 
 }  // namespace coli
