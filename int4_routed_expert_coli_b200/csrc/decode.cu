@@ -121,7 +121,6 @@ __host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
     return L;
 }
 
-__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 // Unpack of a packed word (8 codes, two k16 steps of a lane's fragment) by
 // the fp16 magic-number trick: step 0 takes bytes 0 and 2, step 1 bytes 1 and
@@ -145,8 +144,7 @@ __device__ __forceinline__ void unpack_exact_step(uint32_t w, int step, uint32_t
 
 __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
         "{%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
@@ -170,16 +168,14 @@ __device__ __forceinline__ void load_b_cg(uint32_t bw[8], const __half* p) {
     bw[4] = b1.x; bw[5] = b1.y; bw[6] = b1.z; bw[7] = b1.w;
 }
 
-// 16 consecutive bf16 activations (elements 16c .. 16c+15 of a group) -> this
-// lane's 8 fp16 pairs of the gate/up B fragment, in the fragment order of
-// the streaming GEMV: pair q holds elements e and e + 4, e = (q & 3) + 8 (q >> 2),
-// odd elements divided by 16.  Out-of-range values are clamped (|x| <= 65504,
-// |x / 16| <= 4094); amax collects |x| for the range report.
-__device__ __forceinline__ void x_fragment(const uint16_t* __restrict__ src, uint32_t bw[8],
-                                           float& amax) {
-    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(src));
-    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-    const uint32_t in[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+// 16 consecutive bf16 activations (elements 16c .. 16c+15 of a group, as 8
+// words in bw) -> in place, this lane's 8 fp16 pairs of the gate/up B
+// fragment, in the fragment order of the streaming GEMV: pair q holds
+// elements e and e + 4, e = (q & 3) + 8 (q >> 2), odd elements divided by 16.
+// Out-of-range values are clamped (|x| <= 65504, |x / 16| <= 4094); amax
+// collects |x| for the range report.
+__device__ __forceinline__ void x_fragment(uint32_t bw[8], float& amax) {
+    const uint32_t in[8] = {bw[0], bw[1], bw[2], bw[3], bw[4], bw[5], bw[6], bw[7]};
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const int e = (q & 3) + 8 * (q >> 2);
@@ -245,7 +241,7 @@ struct Smem {
     volatile int* n_slots;
     int* red_cnt;      // [kRedBufs] partials written into each reduction buffer
     float* red;        // reduction buffers; during the prologue, the logits
-    float* corr;       // [H/64][8] offset sums of the 8 token columns
+    float* corr;       // [groups][8] negated offset sums of the 8 token columns
     int* s_idx;        // [T*k] routing
     float* s_w;
     int* s_aux;
@@ -417,9 +413,9 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rb = j % kRedBufs, ruse = j / kRedBufs;
     if (ruse > 0 && !mbar_wait(&x.S.red_empty[rb], (ruse - 1) & 1)) return -1;
-    float* rbuf = x.S.red + rb * (kCW * 4 * 32);
+    const uint32_t rbuf = smem_addr(x.S.red) + (rb * (kCW * 4 * 32) + lane) * 4;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) rbuf[(warp * 4 + q) * 32 + lane] = acc[q];
+    for (int q = 0; q < 4; ++q) sts_f(rbuf + (warp * 4 + q) * 128, acc[q]);
     __threadfence_block();
     __syncwarp();
     int arrived = 0;
@@ -431,7 +427,7 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
     for (int q = 0; q < 4; ++q) {
         float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < kCW; ++w) s += rbuf[(w * 4 + q) * 32 + lane];
+        for (int w = 0; w < kCW; ++w) s += lds_f(rbuf + (w * 4 + q) * 128);
         v[q] = s;
     }
     __syncwarp();
@@ -454,7 +450,7 @@ __device__ __forceinline__ void publish(const Ctx& x, int slot, int n) {
 // false when the kernel must wind down.  A reducing warp publishes its tiles
 // one reduction late (pend_slot / pend_n), so the fence finds its stores
 // long finished instead of stalling on them.
-__device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
+__device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, int j,
                                             const uint32_t (&breg)[kMaxGW][8],
                                             const int (&coff)[kMaxGW], int g_lo,
                                             int& pend_slot, int& pend_n) {
@@ -463,7 +459,6 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     if (*x.S.abort_flag) return false;
     const int stage = j % kStagesD, use = j / kStagesD;
-    const int slot = item / x.gu_tiles, tile = item - slot * x.gu_tiles;
     const SlotEntry* en = x.S.table + slot;
     const bool valid = en->e >= 0;
 
@@ -472,10 +467,11 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
         fail(x, lane);
         return false;
     }
-    const uint8_t* st = x.S.stage0 + (size_t)stage * L.stage_bytes;
+    const uint32_t st = smem_addr(x.S.stage0) + stage * L.stage_bytes;
     if (valid) {
-        const uint16_t* scA = reinterpret_cast<const uint16_t*>(st + 2 * L.gu_op) + r * L.gGp;
-        const uint16_t* scB = reinterpret_cast<const uint16_t*>(st + 2 * L.gu_op + L.gu_sc) + r * L.gGp;
+        const uint32_t scA = st + 2 * L.gu_op + r * L.gGp * 2;
+        const uint32_t scB = scA + L.gu_sc;
+        const uint32_t cor = smem_addr(x.S.corr) + c * 8;
         // three independent MMA chains at a time.  A group past the end of
         // H (the last warp's) has a zero B fragment, a zero offset sum and a
         // zero scale, and reads real staged codes.
@@ -486,15 +482,15 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
 #pragma unroll
             for (int u = 0; u < 3; ++u) {
                 const int i = i0 + u, grp = g_lo + i;
-                wa[u] = *reinterpret_cast<const uint2*>(st + coff[i]);
-                wb[u] = *reinterpret_cast<const uint2*>(st + L.gu_op + coff[i]);
-                const float2 cr = *reinterpret_cast<const float2*>(x.S.corr + grp * 8 + 2 * c);
-                part[u][0] = -cr.x;
-                part[u][1] = -cr.y;
-                part[u][2] = -cr.x;
-                part[u][3] = -cr.y;
-                fa[u] = bf16f(scA[grp]);
-                fb[u] = bf16f(scB[grp]);
+                wa[u] = lds_u2(st + coff[i]);
+                wb[u] = lds_u2(st + L.gu_op + coff[i]);
+                const float2 cr = lds_f2(cor + grp * 32);
+                part[u][0] = cr.x;
+                part[u][1] = cr.y;
+                part[u][2] = cr.x;
+                part[u][3] = cr.y;
+                fa[u] = __uint_as_float(lds_u16(scA + grp * 2) << 16);
+                fb[u] = __uint_as_float(lds_u16(scB + grp * 2) << 16);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the group
@@ -617,7 +613,7 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
         fail(x, lane);
         return false;
     }
-    const uint8_t* st = x.S.stage0 + (size_t)stage * L.stage_bytes;
+    const uint32_t st = smem_addr(x.S.stage0) + stage * L.stage_bytes;
     if (x.S.table[s].e >= 0) {
         // per group, the three tiles' MMA chains run interleaved.  A group past
         // the end of I has a zero B fragment and a zero scale (padding
@@ -626,7 +622,7 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
         // accumulator that is never read.  Row r + 8 of a tile sits 8 staged
         // rows after row r.
         const int row8 = 8 * L.dn_segs * 128;
-        const uint16_t* sc0 = reinterpret_cast<const uint16_t*>(st + kMaxMT * L.dn_op) + r * L.dGp;
+        const uint32_t sc0 = st + kMaxMT * L.dn_op + r * L.dGp * 2;
 #pragma unroll
         for (int i = 0; i < kMaxDW; ++i) {
             const int gs = g_lo + i;
@@ -634,9 +630,9 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
             float part[kMaxMT][4];
 #pragma unroll
             for (int m = 0; m < kMaxMT; ++m) {
-                const uint8_t* codes = st + m * L.dn_op + dcoff[i];
-                wa[m] = *reinterpret_cast<const uint2*>(codes);
-                wb[m] = *reinterpret_cast<const uint2*>(codes + row8);
+                const uint32_t codes = st + m * L.dn_op + dcoff[i];
+                wa[m] = lds_u2(codes);
+                wb[m] = lds_u2(codes + row8);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) part[m][q] = 0.f;
             }
@@ -655,9 +651,9 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
             }
 #pragma unroll
             for (int m = 0; m < kMaxMT; ++m) {
-                const uint16_t* sc = sc0 + m * (L.dn_sc / 2) + gs;
-                const float fa = bf16f(sc[0]);
-                const float fb = bf16f(sc[8 * L.dGp]);
+                const uint32_t sc = sc0 + m * L.dn_sc + gs * 2;
+                const float fa = __uint_as_float(lds_u16(sc) << 16);
+                const float fb = __uint_as_float(lds_u16(sc + 16 * L.dGp) << 16);
                 acc[m][0] = fmaf(fa, part[m][0], acc[m][0]);
                 acc[m][1] = fmaf(fa, part[m][1], acc[m][1]);
                 acc[m][2] = fmaf(fb, part[m][2], acc[m][2]);
@@ -675,8 +671,9 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     const FfnArgs& a = d.f;
     const Layout L = make_layout(a.H, a.I, d.max_slots);
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned start, by pointer arithmetic on the shared array (so
+    // the compiler keeps it a shared-memory pointer)
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const Smem S = carve(smem, L);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -809,24 +806,30 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     uint32_t breg[kMaxGW][8];
     int coff[kMaxGW];
     float amax = 0.f;
+    // all loads first (they are in flight together), then the conversions
 #pragma unroll
     for (int i = 0; i < kMaxGW; ++i) {
         const int grp = gg_lo + i;
-        const bool in = grp < gG;
-        coff[i] = code_offset(r, L.gu_segs, in ? grp : gG - 1, c);
-        if (in && r < a.T) {
-            x_fragment(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)r * a.H + grp * kGroup +
-                           c * 16,
-                       breg[i], amax);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) breg[i][q] = 0u;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (grp < gG && r < a.T) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const uint16_t*>(a.x) + (int64_t)r * a.H + grp * kGroup + c * 16);
+            v0 = __ldg(src);
+            v1 = __ldg(src + 1);
         }
+        breg[i][0] = v0.x; breg[i][1] = v0.y; breg[i][2] = v0.z; breg[i][3] = v0.w;
+        breg[i][4] = v1.x; breg[i][5] = v1.y; breg[i][6] = v1.z; breg[i][7] = v1.w;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxGW; ++i) {
+        const int grp = gg_lo + i;
+        coff[i] = code_offset(r, L.gu_segs, grp < gG ? grp : gG - 1, c);
+        x_fragment(breg[i], amax);
         float cs[4];
         offset_sums(breg[i], cs);
         if (r == 0) {
-            S.corr[grp * 8 + 2 * c] = cs[0];
-            S.corr[grp * 8 + 2 * c + 1] = cs[1];
+            S.corr[grp * 8 + 2 * c] = -cs[0];  // stored negated: the MMA's initial value
+            S.corr[grp * 8 + 2 * c + 1] = -cs[1];
         }
     }
     if (amax > 65504.f) report(a.status, COLI_ERR_RANGE);
@@ -845,8 +848,15 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     bool alive = true;
     const int n_gu = n_slots * gu_tiles;
     int pend_slot = -1, pend_n = 0;
-    for (int item = b; item < n_gu && alive; item += G, ++j)
-        alive = gateup_item(ctx, item, j, breg, coff, gg_lo, pend_slot, pend_n);
+    int slot = b / gu_tiles, tile = b - slot * gu_tiles;  // of item b + j * G
+    for (int item = b; item < n_gu && alive; item += G, ++j) {
+        alive = gateup_item(ctx, slot, tile, j, breg, coff, gg_lo, pend_slot, pend_n);
+        tile += G;
+        while (tile >= gu_tiles) {
+            tile -= gu_tiles;
+            ++slot;
+        }
+    }
     if (pend_n > 0) publish(ctx, pend_slot, pend_n);
 
     // phase 2: down + combine over this CTA's output tiles, slot by slot;

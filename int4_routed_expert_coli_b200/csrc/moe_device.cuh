@@ -24,15 +24,6 @@ __device__ __forceinline__ uint64_t rank_key(float v, int e) {
     return ((uint64_t)k32 << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)e);
 }
 
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t other = __shfl_xor_sync(0xffffffffu, v, o);
-        v = other > v ? other : v;
-    }
-    return v;
-}
-
 // One warp routes one token row.  NV = logits per lane (E <= 32 * NV).
 // Weights: w_j = exp(l_j - m) / sum_i exp(l_i - m) over the chosen set in
 // double, rounded to fp32 once; +inf entries share the weight when m = +inf;
@@ -51,14 +42,15 @@ __device__ __forceinline__ void route_row(const float* __restrict__ row, int E, 
         uint64_t best = 0ull;
 #pragma unroll
         for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
-        best = warp_max_u64(best);
-        const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-        if ((e & 31) == lane) {
+        // warp-wide max of the 64-bit keys: the high words, then the low words
+        // of the lanes holding that high word (keys are unique)
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
+        const uint32_t lo =
+            __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
+        const uint64_t win = ((uint64_t)hi << 32) | lo;
 #pragma unroll
-            for (int i = 0; i < NV; ++i)
-                if (i == (e >> 5)) key[i] = 0ull;
-        }
-        if (lane == j) my_idx = e;
+        for (int i = 0; i < NV; ++i) key[i] = key[i] == win ? 0ull : key[i];
+        if (lane == j) my_idx = (int)(0xFFFFFFFFu - lo);
     }
     const float v = (lane < k) ? row[my_idx] : 0.f;
     const float m = __shfl_sync(0xffffffffu, v, 0);
