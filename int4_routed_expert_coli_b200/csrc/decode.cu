@@ -37,6 +37,7 @@
 // Every wait is bounded (COLI_ERR_TIMEOUT).  The counters are zero on entry;
 // the last CTA to finish puts them back to zero.
 #include <algorithm>
+#include <climits>
 #include <new>
 
 #include "decode.cuh"
@@ -57,6 +58,10 @@ constexpr int kMaxMT = 3;                    // down tiles per CTA
 constexpr int kMaps = 6;                     // per expert: 3 code maps, 3 scale maps
 constexpr int kMaxPairs = 256;               // T * k
 constexpr int kRedFloats = kRedBufs * kCW * 4 * 32;
+// Counters of a call (ints at the workspace's counter offset, zero between calls)
+constexpr int kSyncDone = 0;   // CTAs finished
+constexpr int kSyncItems = 1;  // gate/up items handed out beyond the first one per CTA
+constexpr int kSyncSlots = 2;  // + s: gate/up tiles of slot s published
 static_assert(kRedFloats >= kCW * kMaxMT * 4 * 32, "final reduction reuses the buffers");
 
 struct SlotEntry {
@@ -94,7 +99,7 @@ struct Layout {
     int gu_op, gu_sc, gu_tx;    // gate/up item: code copy, scale copy, bytes per stage
     int dn_op, dn_sc;           // down tile: code copy, scale copy
     int stage_bytes;
-    int red_off, corr_off, route_off, table_off, stage_off, smem;
+    int red_off, corr_off, route_off, table_off, cnt_off, stage_off, smem;
 };
 
 __host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
@@ -114,9 +119,10 @@ __host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
     L.stage_bytes = ((L.gu_tx > dn_stage ? L.gu_tx : dn_stage) + 1023) / 1024 * 1024;
     L.red_off = 1024;
     L.corr_off = L.red_off + kRedFloats * 4;
-    L.route_off = L.corr_off + kCW * kMaxGW * 8 * 4;
+    L.route_off = L.corr_off + kCW * kMaxGW * 16 * 4;
     L.table_off = L.route_off + 3 * kMaxPairs * 4;
-    L.stage_off = (L.table_off + max_slots * (int)sizeof(SlotEntry) + 1023) / 1024 * 1024;
+    L.cnt_off = L.table_off + max_slots * (int)sizeof(SlotEntry);
+    L.stage_off = (L.cnt_off + 3 * max_slots * 4 + 1023) / 1024 * 1024;
     L.smem = L.stage_off + kStagesD * L.stage_bytes + 1024;  // + alignment slack
     return L;
 }
@@ -125,21 +131,34 @@ __host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
 // Unpack of a packed word (8 codes, two k16 steps of a lane's fragment) by
 // the fp16 magic-number trick: step 0 takes bytes 0 and 2, step 1 bytes 1 and
 // 3; e holds the even-k codes as 1032 + q, o the odd-k codes as 1152 + 16 q.
-__device__ __forceinline__ void unpack_raw_step(uint32_t w, int step, uint32_t& e, uint32_t& o) {
+// (a & b) ^ c as one LOP3 with all operands in registers (a mask and a
+// magic constant cannot both be immediates of one instruction).
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+struct Magic {
+    uint32_t lo_mask, lo_bias, hi_mask, hi_bias;
+};
+__device__ __forceinline__ Magic magic() { return {0x000F000Fu, 0x64086408u, 0x00F000F0u, 0x64806480u}; }
+
+__device__ __forceinline__ void unpack_raw_step(uint32_t w, int step, uint32_t& e, uint32_t& o,
+                                                const Magic& mg) {
     const uint32_t v = step ? (w >> 8) : w;
-    e = (v & 0x000F000Fu) ^ 0x64086408u;
-    o = (v & 0x00F000F0u) ^ 0x64806480u;
+    e = and_xor(v, mg.lo_mask, mg.lo_bias);
+    o = and_xor(v, mg.hi_mask, mg.hi_bias);
 }
 
 // The same, exact: e = q_even, o = q_odd as fp16.
-__device__ __forceinline__ void unpack_exact_step(uint32_t w, int step, uint32_t& e, uint32_t& o) {
+__device__ __forceinline__ void unpack_exact_step(uint32_t w, int step, uint32_t& e, uint32_t& o,
+                                                  const Magic& mg) {
     uint32_t re, ro;
-    unpack_raw_step(w, step, re, ro);
-    const __half2 v0 = __hsub2(*reinterpret_cast<__half2*>(&re), __floats2half2_rn(1032.f, 1032.f));
-    const __half2 v1 = __hfma2(*reinterpret_cast<__half2*>(&ro), __floats2half2_rn(0.0625f, 0.0625f),
-                               __floats2half2_rn(-72.f, -72.f));
-    e = *reinterpret_cast<const uint32_t*>(&v0);
-    o = *reinterpret_cast<const uint32_t*>(&v1);
+    unpack_raw_step(w, step, re, ro, mg);
+    // fp16 pairs (1032, 1032), (1/16, 1/16), (-72, -72) as bit patterns
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(e) : "r"(re), "r"(0x64086408u));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(o) : "r"(ro), "r"(0x2C002C00u), "r"(0xD480D480u));
 }
 
 __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t a0, uint32_t a1,
@@ -239,17 +258,21 @@ struct Smem {
     uint64_t* tbl_ready;
     volatile int* abort_flag;
     volatile int* n_slots;
+    volatile int* stage_item;  // [kStagesD] gate/up item in the stage; -1: a down stage
     int* red_cnt;      // [kRedBufs] partials written into each reduction buffer
     float* red;        // reduction buffers; during the prologue, the logits
-    float* corr;       // [groups][8] negated offset sums of the 8 token columns
+    float* corr;       // [groups][4 lanes][4]: negated offset sums, C-fragment order
     int* s_idx;        // [T*k] routing
     float* s_w;
     int* s_aux;
     SlotEntry* table;
+    int* done_local;     // [slots] gate/up tiles finished in this CTA (consumers count)
+    int* pub_local;      // [slots] of those, published to the slot counters (producer)
+    int* issued_local;   // [slots] gate/up tiles of a valid slot this CTA was given
     uint8_t* stage0;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L) {
+__device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L, int max_slots) {
     Smem S;
     S.full = reinterpret_cast<uint64_t*>(smem);
     S.empty = S.full + kStagesD;
@@ -258,12 +281,16 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L) {
     S.abort_flag = reinterpret_cast<volatile int*>(smem + 512);
     S.n_slots = S.abort_flag + 1;
     S.red_cnt = reinterpret_cast<int*>(smem + 528);
+    S.stage_item = reinterpret_cast<volatile int*>(smem + 560);
     S.red = reinterpret_cast<float*>(smem + L.red_off);
     S.corr = reinterpret_cast<float*>(smem + L.corr_off);
     S.s_idx = reinterpret_cast<int*>(smem + L.route_off);
     S.s_w = reinterpret_cast<float*>(S.s_idx + kMaxPairs);
     S.s_aux = S.s_idx + 2 * kMaxPairs;
     S.table = reinterpret_cast<SlotEntry*>(smem + L.table_off);
+    S.done_local = reinterpret_cast<int*>(smem + L.cnt_off);
+    S.pub_local = S.done_local + max_slots;
+    S.issued_local = S.pub_local + max_slots;
     S.stage0 = smem + L.stage_off;
     return S;
 }
@@ -438,40 +465,28 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
     return 1;
 }
 
-// Make this warp's h' stores of `n` finished gate/up tiles of `slot` visible
-// GPU-wide, then count them on the slot's counter.
-__device__ __forceinline__ void publish(const Ctx& x, int slot, int n) {
-    fence_acq_rel_gpu();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) atomicAdd(x.sync + 1 + slot, n);
-}
-
-// One gate/up item (j = position in the CTA's stage sequence).  Returns
-// false when the kernel must wind down.  A reducing warp publishes its tiles
-// one reduction late (pend_slot / pend_n), so the fence finds its stores
-// long finished instead of stalling on them.
+// One gate/up item, staged in stage j % kStagesD (its full barrier already
+// passed).  Returns false when the kernel must wind down.  The reducing warp
+// writes h' and counts the tile in this CTA's done_local (a CTA-scope
+// release); the producer thread publishes the counts GPU-wide, so the
+// GPU-scope fence stalls no consumer.
 __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, int j,
                                             const uint32_t (&breg)[kMaxGW][8],
-                                            const int (&coff)[kMaxGW], int g_lo,
-                                            int& pend_slot, int& pend_n) {
+                                            const int (&coff)[kMaxGW], int g_lo) {
     const FfnArgs& a = x.a;
     const Layout& L = x.L;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-    if (*x.S.abort_flag) return false;
-    const int stage = j % kStagesD, use = j / kStagesD;
+    const int stage = j % kStagesD;
     const SlotEntry* en = x.S.table + slot;
     const bool valid = en->e >= 0;
 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (!mbar_wait(&x.S.full[stage], use & 1)) {
-        fail(x, lane);
-        return false;
-    }
     const uint32_t st = smem_addr(x.S.stage0) + stage * L.stage_bytes;
     if (valid) {
         const uint32_t scA = st + 2 * L.gu_op + r * L.gGp * 2;
         const uint32_t scB = scA + L.gu_sc;
-        const uint32_t cor = smem_addr(x.S.corr) + c * 8;
+        const uint32_t cor = smem_addr(x.S.corr) + c * 16;
+        const Magic mg = magic();
         // three independent MMA chains at a time.  A group past the end of
         // H (the last warp's) has a zero B fragment, a zero offset sum and a
         // zero scale, and reads real staged codes.
@@ -484,11 +499,11 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, in
                 const int i = i0 + u, grp = g_lo + i;
                 wa[u] = lds_u2(st + coff[i]);
                 wb[u] = lds_u2(st + L.gu_op + coff[i]);
-                const float2 cr = lds_f2(cor + grp * 32);
+                const float4 cr = lds_f4(cor + grp * 64);
                 part[u][0] = cr.x;
                 part[u][1] = cr.y;
-                part[u][2] = cr.x;
-                part[u][3] = cr.y;
+                part[u][2] = cr.z;
+                part[u][3] = cr.w;
                 fa[u] = __uint_as_float(lds_u16(scA + grp * 2) << 16);
                 fb[u] = __uint_as_float(lds_u16(scB + grp * 2) << 16);
             }
@@ -497,8 +512,8 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, in
                 uint32_t ae[3], ao[3], be[3], bo[3];
 #pragma unroll
                 for (int u = 0; u < 3; ++u) {
-                    unpack_raw_step((ks >> 1) ? wa[u].y : wa[u].x, ks & 1, ae[u], ao[u]);
-                    unpack_raw_step((ks >> 1) ? wb[u].y : wb[u].x, ks & 1, be[u], bo[u]);
+                    unpack_raw_step((ks >> 1) ? wa[u].y : wa[u].x, ks & 1, ae[u], ao[u], mg);
+                    unpack_raw_step((ks >> 1) ? wb[u].y : wb[u].x, ks & 1, be[u], bo[u], mg);
                 }
 #pragma unroll
                 for (int u = 0; u < 3; ++u)
@@ -524,10 +539,6 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, in
         return false;
     }
     if (red == 0 || !valid) return true;
-    if (pend_n > 0 && pend_slot != slot) {
-        publish(x, pend_slot, pend_n);
-        pend_n = 0;
-    }
     // ---- epilogue (one warp): h' = w * silu(g) * u for the slot's tokens ----
     const int n = tile * kGuRows + r;
     const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
@@ -546,8 +557,11 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, in
         }
         a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn(h);
     }
-    pend_slot = slot;
-    ++pend_n;
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(x.S.done_local + slot, 1);
+    }
     return true;
 }
 
@@ -574,7 +588,7 @@ __device__ __forceinline__ void load_down_b(const FfnArgs& a, const SlotEntry* e
 // True once all gate/up tiles of slot s are published (an invalid slot has
 // nothing to wait for).  Relaxed read.
 __device__ __forceinline__ bool slot_ready(const Ctx& x, int s) {
-    return x.S.table[s].e < 0 || ld_relaxed(x.sync + 1 + s) >= x.gu_tiles;
+    return x.S.table[s].e < 0 || ld_relaxed(x.sync + kSyncSlots + s) >= x.gu_tiles;
 }
 
 // Move `frontier` (slots [0, frontier) are complete and their h' visible to
@@ -615,6 +629,7 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
     }
     const uint32_t st = smem_addr(x.S.stage0) + stage * L.stage_bytes;
     if (x.S.table[s].e >= 0) {
+        const Magic mg = magic();
         // per group, the three tiles' MMA chains run interleaved.  A group past
         // the end of I has a zero B fragment and a zero scale (padding
         // column) and reads real staged codes, so it adds zero; a tile this
@@ -641,8 +656,8 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
                 uint32_t ae[kMaxMT], ao[kMaxMT], be[kMaxMT], bo[kMaxMT];
 #pragma unroll
                 for (int m = 0; m < kMaxMT; ++m) {
-                    unpack_exact_step((ks >> 1) ? wa[m].y : wa[m].x, ks & 1, ae[m], ao[m]);
-                    unpack_exact_step((ks >> 1) ? wb[m].y : wb[m].x, ks & 1, be[m], bo[m]);
+                    unpack_exact_step((ks >> 1) ? wa[m].y : wa[m].x, ks & 1, ae[m], ao[m], mg);
+                    unpack_exact_step((ks >> 1) ? wb[m].y : wb[m].x, ks & 1, be[m], bo[m], mg);
                 }
 #pragma unroll
                 for (int m = 0; m < kMaxMT; ++m)
@@ -674,7 +689,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     // 1024-byte aligned start, by pointer arithmetic on the shared array (so
     // the compiler keeps it a shared-memory pointer)
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Smem S = carve(smem, L);
+    const Smem S = carve(smem, L, d.max_slots);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -688,6 +703,9 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         }
         mbar_init(S.tbl_ready, 1);
         *S.abort_flag = 0;
+    }
+    for (int i = threadIdx.x; i < 3 * d.max_slots; i += kThreadsD) S.done_local[i] = 0;
+    if (threadIdx.x == 0) {
         fence_barrier_init();
     }
     __syncthreads();
@@ -717,29 +735,89 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                 n_slots = *S.n_slots;
                 return true;
             };
+            // Publishing: the tiles the consumers finished (done_local, a
+            // CTA-scope release by the reducing warp) go to the GPU-wide slot
+            // counters after one GPU-scope fence, which makes their h' stores
+            // visible first.  Runs whenever the producer would otherwise wait.
+            int pub_lo = 0, pub_hi = -1;  // slots this CTA has tiles of, not all published
+            auto pump = [&]() {
+                bool fenced = false;
+                for (int sl = pub_lo; sl <= pub_hi; ++sl) {
+                    const int dn = *reinterpret_cast<volatile int*>(S.done_local + sl);
+                    const int pb = S.pub_local[sl];
+                    if (dn > pb) {
+                        if (!fenced) {
+                            fence_acq_rel_gpu();
+                            fenced = true;
+                        }
+                        atomicAdd(d.sync + kSyncSlots + sl, dn - pb);
+                        S.pub_local[sl] = dn;
+                    }
+                }
+                // a slot below the newest is complete here once all its tiles are out
+                while (pub_lo < pub_hi && S.pub_local[pub_lo] == S.issued_local[pub_lo]) ++pub_lo;
+            };
+            auto all_published = [&]() -> bool {
+                return pub_hi < 0 || (pub_lo == pub_hi && S.pub_local[pub_hi] == S.issued_local[pub_hi]);
+            };
             auto next_stage = [&](uint8_t*& st) -> bool {
                 const int stage = j % kStagesD, use = j / kStagesD;
-                if (use > 0 && !mbar_wait(&S.empty[stage], (use - 1) & 1)) {
-                    report(a.status, COLI_ERR_TIMEOUT);
-                    *S.abort_flag = 1;
-                    return false;
+                if (use > 0 && !mbar_test_wait(&S.empty[stage], (use - 1) & 1)) {
+                    const uint64_t t0 = global_timer_ns();
+                    for (;;) {
+                        pump();
+                        if (mbar_try_wait_sleep(&S.empty[stage], (use - 1) & 1, 400u)) break;
+                        if (global_timer_ns() - t0 > kWaitLimitNs) {
+                            report(a.status, COLI_ERR_TIMEOUT);
+                            *S.abort_flag = 1;
+                            return false;
+                        }
+                    }
                 }
                 st = S.stage0 + (size_t)stage * L.stage_bytes;
                 return true;
             };
-            for (int item = b;; item += G) {
-                if (item >= n_gu_shared && !table_known()) {
-                    stop = true;
-                    break;
-                }
-                if (n_slots >= 0 && item >= n_slots * gu_tiles) break;
+            // gate/up: item b first, then items handed out by a counter (after
+            // the previous grid has finished and zeroed it), so faster CTAs
+            // take more.  A CTA with one more down tile than others stops
+            // taking items R before the end, R = the extra down work in items.
+            int* item_ctr = d.sync + kSyncItems;
+            int cur = b;
+            bool pdl_done = false;
+            int last_taken = INT_MAX;  // set once the table is known
+            for (;;) {
                 uint8_t* st;
                 if (*S.abort_flag || !next_stage(st)) {
                     stop = true;
                     break;
                 }
-                uint64_t* bar = &S.full[j % kStagesD];
+                if (cur >= n_gu_shared && cur != INT_MAX && !table_known()) {
+                    stop = true;
+                    break;
+                }
+                if (n_slots >= 0 && last_taken == INT_MAX) {
+                    const int t_hi = (n_mt + G - 1) / G;
+                    const int n_hi = n_mt - (t_hi - 1) * G;
+                    const int lo = G - n_hi;
+                    const float extra =
+                        (float)lo * n_slots * (float)(L.dn_op + L.dn_sc) / (float)L.gu_tx;
+                    last_taken = n_slots * gu_tiles - ((my_mt == t_hi && lo > 0) ? (int)extra : 0);
+                }
+                if (cur >= (n_slots >= 0 ? n_slots * gu_tiles : INT_MAX)) break;  // stage j stays free
+                int nxt = INT_MAX;
+                if (cur < last_taken) {
+                    if (!pdl_done) {
+                        pdl_wait();
+                        pdl_done = true;
+                    }
+                    nxt = G + atomicAdd(item_ctr, 1);
+                }
+                const int stage = j % kStagesD;
+                uint64_t* bar = &S.full[stage];
+                S.stage_item[stage] = cur;
                 ++j;
+                const int item = cur;
+                cur = nxt;
                 if (item == a.withhold_item) continue;  // test hook: this stage never fills
                 const int slot = item / gu_tiles, tile = item - slot * gu_tiles;
                 const int e = slot < a.n_shared ? a.E + slot : S.table[slot].e;
@@ -747,6 +825,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                     mbar_arrive(bar);
                     continue;
                 }
+                ++S.issued_local[slot];
+                pub_hi = slot;
                 const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
                 const int n0 = tile * kGuRows;
                 mbar_arrive_expect_tx(bar, L.gu_tx);
@@ -755,11 +835,20 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                 tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
                 tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
             }
-            if (!stop && my_mt > 0 && table_known()) {
-                for (int s = 0; s < n_slots; ++s) {
+            // down stages carry item -1, which tells the consumers that gate/up
+            // is over; without down work a single empty stage does
+            if (!stop && table_known()) {
+                if (my_mt == 0) {
+                    S.stage_item[j % kStagesD] = -1;
+                    mbar_arrive(&S.full[j % kStagesD]);
+                    ++j;
+                }
+                for (int s = 0; s < n_slots && my_mt > 0; ++s) {
                     uint8_t* st;
                     if (*S.abort_flag || !next_stage(st)) break;
-                    uint64_t* bar = &S.full[j % kStagesD];
+                    const int stage = j % kStagesD;
+                    uint64_t* bar = &S.full[stage];
+                    S.stage_item[stage] = -1;
                     ++j;
                     const int e = S.table[s].e;
                     if (e < 0) {
@@ -774,6 +863,20 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                         tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0, bar,
                                     policy);
                     }
+                }
+            }
+            // publish the rest (the consumers may still be reducing the last tiles)
+            if (!stop) {
+                const uint64_t t0 = global_timer_ns();
+                for (;;) {
+                    pump();
+                    if (all_published() || *S.abort_flag) break;
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        report(a.status, COLI_ERR_TIMEOUT);
+                        *S.abort_flag = 1;
+                        break;
+                    }
+                    __nanosleep(200);
                 }
             }
             if (*S.abort_flag) {
@@ -827,10 +930,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         x_fragment(breg[i], amax);
         float cs[4];
         offset_sums(breg[i], cs);
-        if (r == 0) {
-            S.corr[grp * 8 + 2 * c] = -cs[0];  // stored negated: the MMA's initial value
-            S.corr[grp * 8 + 2 * c + 1] = -cs[1];
-        }
+        if (r == 0)  // stored negated, as the MMA's initial C fragment of lane c
+            reinterpret_cast<float4*>(S.corr)[grp * 4 + c] = make_float4(-cs[0], -cs[1], -cs[0], -cs[1]);
     }
     if (amax > 65504.f) report(a.status, COLI_ERR_RANGE);
     if (d.logits) cp_async_wait_all();
@@ -846,18 +947,24 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     // phase 1: gate/up items
     int j = 0;
     bool alive = true;
-    const int n_gu = n_slots * gu_tiles;
-    int pend_slot = -1, pend_n = 0;
-    int slot = b / gu_tiles, tile = b - slot * gu_tiles;  // of item b + j * G
-    for (int item = b; item < n_gu && alive; item += G, ++j) {
-        alive = gateup_item(ctx, slot, tile, j, breg, coff, gg_lo, pend_slot, pend_n);
-        tile += G;
-        while (tile >= gu_tiles) {
-            tile -= gu_tiles;
-            ++slot;
+    for (;;) {  // the producer names each stage's item; -1 ends gate/up
+        const int stage = j % kStagesD;
+        if (*S.abort_flag) {
+            alive = false;
+            break;
         }
+        if (!mbar_wait(&S.full[stage], (j / kStagesD) & 1)) {
+            fail(ctx, lane);
+            alive = false;
+            break;
+        }
+        const int item = S.stage_item[stage];
+        if (item < 0) break;
+        const int slot = item / gu_tiles;
+        alive = gateup_item(ctx, slot, item - slot * gu_tiles, j, breg, coff, gg_lo);
+        ++j;
+        if (!alive) break;
     }
-    if (pend_n > 0) publish(ctx, pend_slot, pend_n);
 
     // phase 2: down + combine over this CTA's output tiles, slot by slot;
     // h' fragments of the next slot are loaded while this one is computed
@@ -926,10 +1033,11 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     // the last CTA to get here returns the counters to zero
     if (threadIdx.x == 0) {
         fence_acq_rel_gpu();
-        if (atomicAdd(d.sync, 1) == G - 1) {
+        if (atomicAdd(d.sync + kSyncDone, 1) == G - 1) {
             fence_acq_rel_gpu();
-            for (int s = 0; s < n_slots; ++s) d.sync[1 + s] = 0;
-            d.sync[0] = 0;
+            for (int s = 0; s < n_slots; ++s) d.sync[kSyncSlots + s] = 0;
+            d.sync[kSyncItems] = 0;
+            d.sync[kSyncDone] = 0;
         }
     }
 }
@@ -961,8 +1069,8 @@ int max_slots_for(int E, int k, int T, int n_shared) {
 bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_sms) {
     if (T < 1 || T > 8 || T * k > kMaxPairs || H % 512 || I % 512 || num_sms < 1) return false;
     // the slot counters live between the two counter offsets of the header
-    if (1 + max_slots_for(E, k, T, n_shared) > (int)((kTileCntOffset - kSlotCntOffset) / 4))
-        return false;
+    const int counters = (int)((kTileCntOffset - kSlotCntOffset) / 4);
+    if (kSyncSlots + max_slots_for(E, k, T, n_shared) > counters) return false;
     const Layout L = make_layout(H, I, max_slots_for(E, k, T, n_shared));
     if (L.smem > kSmemLimitD) return false;
     if (H / kGroup > kCW * kMaxGW || I / kGroup > kCW * kMaxDW) return false;
