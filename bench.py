@@ -254,7 +254,7 @@ def run_ours(args, rank, world, local):
     ws = layer.workspace(T, dev)
     out = torch.empty(T, H, dtype=torch.float32, device=dev)
     idx = torch.empty(T, k, dtype=torch.int32, device=dev)
-    flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     fence_buf = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def flush_l2():

@@ -322,16 +322,14 @@ __device__ void table_init(const FfnArgs& a, const Smem& S, int max_slots) {
     }
 }
 
-// Route the T tokens and build the slot table from the routing: the union
-// of the pairs p = t * k + j, experts ascending, tokens ascending inside an
-// expert (the lists the batch-union step defines).
-template <int NV>
-__device__ void table_from_logits(const DecodeArgs& d, const Smem& S, const float* lg) {
+// The slot table from the routing (s_idx / s_w, written by the routing
+// warps before this): the union of the pairs p = t * k + j, experts
+// ascending, tokens ascending inside an expert (the lists the batch-union
+// step defines).
+__device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
     const FfnArgs& a = d.f;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int P = a.T * a.k;
-    if (warp < a.T)
-        route_row<NV>(lg + warp * a.E, a.E, a.k, lane, S.s_idx + warp * a.k, S.s_w + warp * a.k);
     table_init(a, S, d.max_slots);
     consumers_sync();
     if (blockIdx.x == 0) {
@@ -892,12 +890,17 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
 
     // -------------------------------- consumers --------------------------------
     pdl_wait();
-    // logits -> shared memory (the reduction buffers are free until the first
-    // item); they land while the activation operand is built
-    if (d.logits) {
-        const int n = a.T * a.E;
-        for (int i = threadIdx.x; i < n; i += kConsumerThreads) cp_async4(S.red + i, d.logits + i);
+    // routing first: warp t < T copies token t's logits into shared memory
+    // (the reduction buffers are free until the first item) and routes it,
+    // while the other warps build the activation operand
+    if (d.logits && warp < a.T) {
+        const float* src = d.logits + (int64_t)warp * a.E;
+        float* dst = S.red + warp * a.E;
+        for (int i = lane; i < a.E; i += 32) cp_async4(dst + i, src + i);
         cp_async_commit();
+        cp_async_wait_all();
+        __syncwarp();
+        route_row<NV>(dst, a.E, a.k, lane, S.s_idx + warp * a.k, S.s_w + warp * a.k);
     }
     const int r = lane >> 2, c = lane & 3;
 
@@ -934,10 +937,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             reinterpret_cast<float4*>(S.corr)[grp * 4 + c] = make_float4(-cs[0], -cs[1], -cs[0], -cs[1]);
     }
     if (amax > 65504.f) report(a.status, COLI_ERR_RANGE);
-    if (d.logits) cp_async_wait_all();
-    consumers_sync();
 
-    if (d.logits) table_from_logits<NV>(d, S, S.red);
+    if (d.logits) table_from_logits(d, S);
     else table_from_union(d, S);
     consumers_sync();
     if (threadIdx.x == 0) mbar_arrive(S.tbl_ready);
