@@ -57,7 +57,8 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one fused decode launch, from the ncu capture
 # summarised in profiles/decode_fused_kernel_glm_t1.md (tokens per step ->
 # bytes); a workload without a capture of the current kernel reports null.
-FUSED_DECODE_DRAM_BYTES = {}
+FUSED_DECODE_DRAM_BYTES = {1: 180_608_000 + 3_382_528}
+PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 
 
 def expert_bytes(H, I):
@@ -359,10 +360,24 @@ def run_ours(args, rank, world, local):
     # down and combine; it streams every active expert whole), otherwise the
     # gate/up kernel of the streaming or tensor-core path
     fused = T <= 8
+    tensor = kind == "uniform"  # prefill: the tensor-core grouped GEMM
     k_ms = phase_ms[1] / max(n_calls, 1)
-    k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
-    achieved = k_bytes / (k_ms / 1e3) / 1e9
-    traffic = FUSED_DECODE_DRAM_BYTES.get(T) if fused else None
+    if tensor:
+        # gate/up GEMM: 2/3 of the pair FLOPs over all (token, expert) pairs + shared
+        k_work = (T * k + T * n_sh) * PAIR_FLOP * 2 / 3
+        achieved = k_work / (k_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": "prefill_gemm_kernel<gate/up>",
+                "achieved": achieved, "peak": P["bf16"], "unit": "TFLOP/s",
+                "frac": achieved / P["bf16"], "peak_source": P["src"] + " (bf16 burst; fp16 taken equal)",
+                "traffic": None, "algorithmic_flop_per_launch": k_work, "avg_launch_ms": k_ms}
+    else:
+        k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
+        achieved = k_bytes / (k_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": "decode_fused_kernel" if fused else "gateup_kernel",
+                "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
+                "frac": achieved / P["hbm"], "peak_source": P["src"],
+                "traffic": FUSED_DECODE_DRAM_BYTES.get(T) if fused else None,
+                "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -374,11 +389,7 @@ def run_ours(args, rank, world, local):
                    "l2": "flushed between timed steps (256 MiB read), steps timed alone",
                    "parallelism": f"replicas x{world}"},
         "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
-        "roofline": {"bound": "hbm",
-                     "kernel": "decode_fused_kernel" if fused else "gateup_kernel",
-                     "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
-                     "frac": achieved / P["hbm"], "peak_source": P["src"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
+        "roofline": roof,
         "phase_ms_per_step": {"before": phase_ms[0] / max(n_calls, 1), "main": k_ms,
                               "after": phase_ms[2] / max(n_calls, 1)},
         "cpu_baseline": cpu,
