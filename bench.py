@@ -51,7 +51,10 @@ WORKLOADS = {
     "batch32": (32, "zipf", "GLM-5.2-shaped small-batch decode: T=32, Zipf-1.1 routing, "
                             "71.6% step-to-step expert repeats"),
     "prefill": (4096, "uniform", "GLM-5.2-shaped prefill: T=4096, logits U[0,1)"),
+    "stack": (64, "zipf", "16 independent GLM-5.2-shaped layers (16 x 257 experts resident), "
+                          "T=64, per-layer Zipf-1.1 routing, x_(l+1) = x_l + MoE_l(x_l) in bf16"),
 }
+STACK_LAYERS = 16
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one fused decode launch, from the ncu capture
@@ -203,12 +206,63 @@ def oracle_steps(bank, xs, lgs, n_threads):
     return time.perf_counter() - t0, X.shape[0]
 
 
+def run_reference_stack(args):
+    """The CPU oracle on the stack: each step takes a 2-token sample through
+    all 16 layers (each layer's bf16 output feeds the next), timed on the
+    host cores; the layers' weights are generated one at a time."""
+    import oracle
+    T, _, desc = WORKLOADS["stack"]
+    H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    cores = os.cpu_count() or 1
+    n = args.warmup + args.steps
+    tok = 2
+    xs, lgs = stack_inputs(n, seed=7, device="cpu")
+    x = [xs[i][:tok].clone() for i in range(n)]
+    sec = 0.0
+    for l in range(STACK_LAYERS):
+        bank = synth.make_expert_bank(H, I, E + n_sh, seed=7000 + l, device=dev,
+                                      scale_range=synth.STACK_SCALE_RANGE,
+                                      code_range=synth.STACK_CODE_RANGE)
+        routes = [oracle.route(lgs[l][i][:tok].float().numpy(), k) for i in range(n)]
+        needed = set(range(E, E + n_sh))
+        for idx, _ in routes:
+            needed |= set(idx.ravel().tolist())
+        ex = oracle.Experts([bank.expert_numpy(e) if e in needed else None for e in range(bank.n)])
+        del bank
+        for i in range(n):
+            xb = x[i].view(torch.int16).numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            y = oracle.layer(H, I, E, k, n_sh, ex, xb, routes[i][0], routes[i][1],
+                             n_threads=cores)
+            if i >= args.warmup:
+                sec += time.perf_counter() - t0
+            x[i] = (x[i].double() + torch.from_numpy(np.asarray(y))).to(torch.bfloat16)
+    value = tok * args.steps / sec
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": desc, "tokens_per_step": tok, "layers": STACK_LAYERS},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {tok} tokens through all "
+                                   f"{STACK_LAYERS} layers, every routed + shared expert"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, rank, world):
     """The CPU oracle on the same workload: each step is one full layer step
     of the workload (all its tokens), timed on the host cores."""
     if rank != 0:
         return
     name = args.workload
+    if name == "stack":
+        run_reference_stack(args)
+        return
     T, _, desc = WORKLOADS[name]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     bank = synth.make_expert_bank(GLM["H"], GLM["I"], GLM["E"] + 1, seed=1, device=dev)
@@ -242,6 +296,143 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------------------
+def stack_inputs(n, seed, device):
+    """Per-step layer-0 activations and per-layer, per-step Zipf logits."""
+    T = WORKLOADS["stack"][0]
+    xs = [synth.make_activations(T, GLM["H"], seed=seed * 100003 + s, device=device)
+          for s in range(n)]
+    lgs = []
+    for l in range(STACK_LAYERS):
+        _, lg_np = synth.zipf_routing(T, GLM["E"], GLM["k"], steps=n, seed=seed * 1009 + l)
+        lgs.append([torch.from_numpy(lg_np[s]).to(device) for s in range(n)])
+    return xs, lgs
+
+
+def run_stack(args, rank, world, local):
+    """Config 5: 16 independent layers, each step runs them in sequence on
+    one token batch, x_(l+1) = x_l + MoE_l(x_l) (bf16 stream, residual added
+    in fp32 by the combine)."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    T, _, desc = WORKLOADS["stack"]
+    H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
+    L = STACK_LAYERS
+    dev = torch.device("cuda", local if world > 1 else 0)
+    banks = [synth.make_expert_bank(H, I, E + n_sh, seed=7000 + l, device=dev,
+                                    scale_range=synth.STACK_SCALE_RANGE,
+                                    code_range=synth.STACK_CODE_RANGE) for l in range(L)]
+    layers = [c.MoELayer(b, n_routed=E, top_k=k, n_shared=n_sh) for b in banks]
+    n = args.warmup + args.steps
+    xs, lgs = stack_inputs(n, seed=7 + rank, device=dev)
+    ws = layers[0].workspace(T, dev)
+    acts = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    fence_buf = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def flush_l2():
+        flush_buf.sum()
+        fence_buf.zero_()
+
+    def step(i, x0, out_last=None):
+        x = x0
+        for l in range(L):
+            out = acts[l] if (l < L - 1 or out_last is None) else out_last
+            c.coli_moe_layer(layers[l].handle, T, x, lgs[l][i], None, x, out, c.COLI_OUT_BF16,
+                             None, None, ws, stream)
+            x = out
+        return x
+
+    for i in range(args.warmup):
+        step(i, xs[i])
+        flush_l2()
+    torch.cuda.synchronize(dev)
+    if c.coli_moe_get_status(ws) != c.COLI_OK:
+        raise RuntimeError("device status after warm-up: " + c.status_string(c.coli_moe_get_status(ws)))
+    uniq = [[len(set(torch.topk(lgs[l][i], k, dim=1).indices.flatten().tolist()))
+             for l in range(L)] for i in range(args.warmup, n)]
+
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for j in range(args.steps):
+        ev[j][0].record(stream)
+        step(args.warmup + j, xs[args.warmup + j])
+        ev[j][1].record(stream)
+        flush_l2()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    if c.coli_moe_get_status(ws) != c.COLI_OK:
+        raise RuntimeError("device status: " + c.status_string(c.coli_moe_get_status(ws)))
+
+    torch.cuda.synchronize(dev)
+    c.coli_moe_profile_enable(True)
+    for j in range(args.steps):
+        step(args.warmup + j, xs[args.warmup + j])
+        flush_l2()
+    torch.cuda.synchronize(dev)
+    c.coli_moe_profile_enable(False)
+    phase_ms, n_calls = c.coli_moe_profile_read()
+
+    # end to end: layer-0 input from pinned host memory, last output back
+    x_host = torch.stack([x.cpu() for x in xs[args.warmup:]]).pin_memory()
+    out_host = torch.empty(args.steps, T, H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    out_dev = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for j in range(args.steps):
+        ev2[j][0].record(stream)
+        x_dev.copy_(x_host[j], non_blocking=True)
+        step(args.warmup + j, x_dev, out_last=out_dev)
+        out_host[j].copy_(out_dev, non_blocking=True)
+        ev2[j][1].record(stream)
+        flush_l2()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world)
+
+    if rank != 0:
+        return
+    P = peaks()
+    tokens = T * args.steps * world
+    value = tokens / (total_ms / 1e3)
+    step_bytes = statistics.mean(sum(u + n_sh for u in us) for us in uniq) * expert_bytes(H, I)
+    k_ms = phase_ms[1] / max(n_calls, 1)
+    k_bytes = statistics.mean(statistics.mean(us) for us in uniq) * gateup_bytes(H, I) + \
+        n_sh * gateup_bytes(H, I)
+    achieved = k_bytes / (k_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4xbf16/f16->f32", "data": "synthetic",
+        "config": {"workload": desc, "tokens_per_step": T, "layers": L, "hidden": H, "inter": I,
+                   "routed_experts": E, "top_k": k, "shared_experts": n_sh,
+                   "resident_bytes": L * (E + n_sh) * expert_bytes(H, I),
+                   "unique_routed_experts_per_layer": statistics.mean(
+                       statistics.mean(us) for us in uniq),
+                   "l2": "flushed between timed steps (256 MiB read); the stack itself "
+                         "streams far more than L2 per step",
+                   "parallelism": f"replicas x{world}"},
+        "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": achieved,
+                     "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
+                     "peak_source": P["src"], "traffic": None,
+                     "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
+        "cpu_baseline": None,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": 4 * L * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args, rank, world, local):
     from int4_routed_expert_coli_b200 import coli_moe as c
     name = args.workload
@@ -425,6 +616,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "stack":
+            run_stack(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -75,20 +75,43 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
+# Generator settings of the stacked-layers workload.  Untrained experts drawn
+# as for a single layer make x_(l+1) = x_l + MoE_l(x_l) blow up: codes
+# uniform over [-8, 7] have mean -1/2, so every layer adds the same offset to
+# all H elements and the next layer's dot products grow with it, and U(.005,
+# .02) scales multiply the stream's RMS by ~50 per layer.  Zero-mean codes
+# over [-7, 7] and one eighth of the scales keep every layer's update near
+# 7 % of an O(1) stream.
+STACK_SCALE_RANGE = (0.005 / 8, 0.02 / 8)
+STACK_CODE_RANGE = (-7, 7)
+
+
 def make_expert_bank(hidden: int, inter: int, n_experts: int, seed: int,
-                     device="cpu") -> ExpertBank:
-    """Random int4 gs64 experts: codes uniform over [-8, 7], scales U(.005,.02)."""
+                     device="cpu", scale_range=(0.005, 0.02),
+                     code_range=(-8, 7)) -> ExpertBank:
+    """Random int4 gs64 experts: codes uniform over code_range (default
+    [-8, 7]: every nibble value), scales U(scale_range) rounded to bf16
+    (default U(.005, .02))."""
     if hidden % (2 * GROUP) or inter % (2 * GROUP):
         raise ValueError("hidden and inter must be multiples of 128")
     g = _gen(seed, device)
     kw = dict(dtype=torch.uint8, device=device)
-    gate_q = torch.empty(n_experts, inter, hidden // 2, **kw).random_(0, 256, generator=g)
-    up_q = torch.empty(n_experts, inter, hidden // 2, **kw).random_(0, 256, generator=g)
-    down_q = torch.empty(n_experts, hidden, inter // 2, **kw).random_(0, 256, generator=g)
+
+    def codes(rows, cols):
+        if tuple(code_range) == (-8, 7):  # all 16 nibble values: uniform bytes
+            return torch.empty(n_experts, rows, cols, **kw).random_(0, 256, generator=g)
+        lo, hi = code_range
+        q = torch.empty(2, n_experts, rows, cols, **kw).random_(0, hi - lo + 1, generator=g)
+        q = (q.to(torch.int16) + lo).bitwise_and(0xF).to(torch.uint8)
+        return q[0] | (q[1] << 4)
+
+    gate_q = codes(inter, hidden // 2)
+    up_q = codes(inter, hidden // 2)
+    down_q = codes(hidden, inter // 2)
 
     def scales(rows, cols):
         s = torch.empty(n_experts, rows, cols, dtype=torch.float32, device=device)
-        s.uniform_(0.005, 0.02, generator=g)
+        s.uniform_(scale_range[0], scale_range[1], generator=g)
         return s.to(torch.bfloat16)
 
     gate_s = scales(inter, hidden // GROUP)
