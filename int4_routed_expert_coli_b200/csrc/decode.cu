@@ -438,9 +438,9 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rb = j % kRedBufs, ruse = j / kRedBufs;
     if (ruse > 0 && !mbar_wait(&x.S.red_empty[rb], (ruse - 1) & 1)) return -1;
-    const uint32_t rbuf = smem_addr(x.S.red) + (rb * (kCW * 4 * 32) + lane) * 4;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sts_f(rbuf + (warp * 4 + q) * 128, acc[q]);
+    // [warp][lane] float4 per buffer: one 16-byte store per lane
+    const uint32_t rbuf = smem_addr(x.S.red) + (rb * (kCW * 4 * 32) + lane * 4) * 4;
+    sts_f4(rbuf + warp * 512, make_float4(acc[0], acc[1], acc[2], acc[3]));
     __threadfence_block();
     __syncwarp();
     int arrived = 0;
@@ -448,13 +448,19 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
     arrived = __shfl_sync(0xffffffffu, arrived, 0);
     if (arrived != kCW - 1) return 0;
     __threadfence_block();
+    float4 sum = lds_f4(rbuf);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kCW; ++w) s += lds_f(rbuf + (w * 4 + q) * 128);
-        v[q] = s;
+    for (int w = 1; w < kCW; ++w) {
+        const float4 p = lds_f4(rbuf + w * 512);
+        sum.x += p.x;
+        sum.y += p.y;
+        sum.z += p.z;
+        sum.w += p.w;
     }
+    v[0] = sum.x;
+    v[1] = sum.y;
+    v[2] = sum.z;
+    v[3] = sum.w;
     __syncwarp();
     if (lane == 0) {
         x.S.red_cnt[rb] = 0;
