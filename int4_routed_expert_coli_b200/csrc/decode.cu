@@ -330,6 +330,54 @@ __device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
     const FfnArgs& a = d.f;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int P = a.T * a.k;
+    if (P <= 32) {
+        // one warp, one pair per lane: leaders by match_any, ranks by shuffles
+        if (a.T > 1) consumers_sync();  // the other routing warps' pairs
+        if (warp != 0) return;
+        __syncwarp();
+        const bool on = lane < P;
+        const int e = on ? S.s_idx[lane] : INT_MAX;
+        const float w = on ? S.s_w[lane] : 0.f;
+        const unsigned below = (1u << lane) - 1u;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const bool lead = on && (peers & below) == 0u;
+        const unsigned leads = __ballot_sync(0xffffffffu, lead);
+        int before = 0, rank = 0;
+        for (int q = 0; q < P; ++q) {
+            const int eq = __shfl_sync(0xffffffffu, e, q);
+            before += eq < e;
+            rank += (eq < e) & (int)((leads >> q) & 1u);
+        }
+        const int n_slots = a.n_shared + __popc(leads);
+        for (int i = lane; i < n_slots; i += 32) {
+            SlotEntry& en = S.table[i];
+            const bool sh = i < a.n_shared;
+            en.e = sh ? a.E + i : -1;
+            en.list_begin = sh ? P + i * a.T : 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                en.pos[t] = (int8_t)((sh && t < a.T) ? t : -1);
+                en.w[t] = (sh && t < a.T) ? 1.f : 0.f;
+            }
+        }
+        __syncwarp();
+        if (on) {
+            SlotEntry& en = S.table[a.n_shared + rank];
+            if (lead) {
+                en.e = e;
+                en.list_begin = before;
+            }
+            const int t = lane / a.k;
+            en.pos[t] = (int8_t)__popc(peers & below);
+            en.w[t] = w;
+            if (blockIdx.x == 0) {
+                if (d.idx_out) d.idx_out[lane] = e;
+                if (d.w_out) d.w_out[lane] = w;
+            }
+        }
+        if (lane == 0) *S.n_slots = n_slots;
+        return;
+    }
     table_init(a, S, d.max_slots);
     consumers_sync();
     if (blockIdx.x == 0) {
