@@ -438,6 +438,8 @@ def run_ours(args, rank, world, local):
     name = args.workload
     T, kind, desc = WORKLOADS[name]
     H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
+    if E != 256:  # a smaller resident bank (profiling runs) says so in the label
+        desc = desc.replace("256 routed", f"{E} routed") + f", {E} routed experts resident"
     dev = torch.device("cuda", local if world > 1 else 0)
     bank = synth.make_expert_bank(H, I, E + n_sh, seed=1, device=dev)
     layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=n_sh)

@@ -6,23 +6,35 @@
 // "yunpan.plus/t/30351-1-1", capability two), gate/up is
 //   [2 x I rows of int4 codes] x [n_e tokens x H]  -> h [n_e][I]
 // and down is [H rows] x [n_e x I] -> y [n_e][H].  The weight rows are the MMA
-// M dimension (tiles of 128), the tokens the N dimension (tiles of up to 128,
-// rounded to 16), K is walked in 64-element blocks (one gs64 scale group).
+// M dimension (128 per tile; for gate/up 64 gate rows + the up rows of the
+// same 64 features, so one MMA covers both and reads the activation tile
+// once), the tokens the N dimension (tiles of up to 192, rounded to 16, so a
+// routed expert of a 4096-token prefill is one tile and its weights are
+// dequantised once per M tile), K is walked in 64-element blocks (one gs64
+// scale group).
 //
 // Pipeline (one CTA per SM, persistent over a flattened list of tiles):
-//   warp 0      TMA producer: packed int4 codes of the tile rows (a 2-D tensor
-//               map per expert matrix, 32 bytes x 128 rows per K-block) and the
-//               activation tile (128-byte swizzled, fp16);
+//   warp 0      TMA producer: packed int4 codes of the tile rows (2-D tensor
+//               maps per expert matrix, 32 bytes x 64 or 128 rows per K-block)
+//               and the activation rows the tile has (128-byte swizzled fp16,
+//               32-row boxes);
 //   warps 4-7   dequant: each thread owns one weight row, turns its 64 codes
 //               into fp16 q * s (exact: a 3-bit code magnitude times an 8-bit
-//               bf16 scale fits fp16's 11 bits) and writes the 128-byte
-//               swizzled K-major operand tile;
-//   warp 1      one thread issues tcgen05.mma (kind::f16, fp32 accumulate in
-//               tensor memory; gate and up share the activation tile and have
-//               two accumulators) and commits stage release / tile completion;
+//               bf16 scale fits fp16's 11 bits) and stores them straight into
+//               tensor memory (tcgen05.st, lane = weight row, two fp16 per
+//               column): the weight operand never passes through shared
+//               memory, whose bandwidth the activation tile and the TMA
+//               copies need;
+//   warp 1      one thread issues tcgen05.mma (kind::f16, A from tensor
+//               memory, B from shared memory, fp32 accumulate in tensor
+//               memory) and commits stage / operand release and tile
+//               completion;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator (each warp its 32
 //               lanes), SwiGLU to fp16 h, or the fp32 y rows of the down GEMM.
-//   Two accumulator buffers let the epilogue of one tile overlap the next.
+//   Tensor memory (512 columns): two 192-column accumulators (the epilogue of
+//   one tile overlaps the next tile's MMAs) and a 4-deep ring of 32-column
+//   weight operands.  The shared-memory ring of code and activation tiles is
+//   deeper than the operand ring; each has its own release barrier.
 // Every wait is bounded (COLI_ERR_TIMEOUT) so nothing can hang the GPU.
 //
 // K order.  Within each group of 8 consecutive K elements the dequant unpack
@@ -44,8 +56,12 @@
 namespace coli {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int BM = 128, BN = 192, BK = 64;
+constexpr int kBRowQuant = 32;      // activation rows are loaded in multiples of 32
 constexpr int kThreadsP = 384;
+constexpr uint32_t kTmemColsP = 512;
+constexpr uint32_t kAccCols = 2 * BN;  // two accumulators; the operand ring follows
+constexpr int kXchBytes = 64 * 33 * 4;  // gate/up epilogue exchange block
 constexpr int kHeaderP = 2048;
 constexpr int kSmemLimitP = 227 * 1024;
 
@@ -70,12 +86,13 @@ __device__ __forceinline__ uint32_t idesc_f16(int n) {
            | ((uint32_t)(BM >> 4) << 24);     // M = 128; A, B: f16, K-major
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate) {
+// A (the dequantised weights) from tensor memory, B from shared memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -104,6 +121,36 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t v[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 consecutive columns of this warp's 32 lanes <- v (lane i writes its own row).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+// bar.red.and over `count` threads of named barrier `id`: true iff every
+// participating thread passed true.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1,
                                             uint64_t* bar) {
     asm volatile(
@@ -121,6 +168,18 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, in
         "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
+
+// Position in a ring of barriers: slot index and how many times it wrapped
+// (the parity of the phase to wait for), advanced without a division.
+struct Ring {
+    int i = 0, pass = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++i == n) {
+            i = 0;
+            ++pass;
+        }
+    }
+};
 
 // ---- tile bookkeeping --------------------------------------------------------
 struct TileInfo {
@@ -174,34 +233,45 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_
 }
 
 // ---- the GEMM kernel -------------------------------------------------------
+// kGU: gate/up.  A tile's 128 MMA rows are 64 gate rows and the up rows of the
+// same 64 features (K = H), so one MMA per K step covers both and the
+// activation tile is read once; the epilogue pairs lane f (gate) with lane
+// 64 + f (up) through shared memory.  Otherwise down: 128 rows of W_d, K = I.
 template <bool kGU>
 __global__ void __launch_bounds__(kThreadsP, 1)
-prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, int stages) {
-    constexpr int NA = kGU ? 2 : 1;                          // weight matrices per tile
-    constexpr int kDqBytes = BM * BK * 2;                    // 16 KB per matrix
-    constexpr int kBBytes = BN * BK * 2;                     // 16 KB
-    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
-    constexpr int kStage = NA * kDqBytes + kBBytes + NA * kPkBytes;
-    constexpr uint32_t kTmemCols = kGU ? 512 : 256;          // 2 buffers x NA x 128
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
+                    const __grid_constant__ CUtensorMap bmap64,
+                    const __grid_constant__ CUtensorMap bmap32, const GemmArgs a, int stages) {
+    constexpr int kFeat = kGU ? BM / 2 : BM;                 // output features per tile
+    constexpr int kBBytes = BN * BK * 2;                     // 24 KB
+    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB
+    constexpr int kStage = kBBytes + kPkBytes;
+    constexpr int kACols = BK / 2;                           // operand columns per K-block
+    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 4
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // TMA landed
-    uint64_t* dq_full = full + 16;                             // operand tile written
+    uint64_t* dq_full = full + 16;                             // operand written to TMEM
     uint64_t* empty = full + 32;                               // MMAs done reading the stage
     uint64_t* acc_full = full + 48;                            // [2] accumulator ready
     uint64_t* acc_empty = full + 50;                           // [2] accumulator drained
+    uint64_t* a_empty = full + 52;                             // [8] MMAs done with an operand
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 512);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
     uint8_t* stage0 = smem + kHeaderP;
+    float* xch = reinterpret_cast<float*>(stage0 + (size_t)stages * kStage);  // gate/up only
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&dq_full[s], 4);
             mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&dq_full[s], 4);
+            mbar_init(&a_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -213,7 +283,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr((const void*)tmem_slot)),
-                     "r"(kTmemCols)
+                     "r"(kTmemColsP)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -230,7 +300,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
         n_act = 0;
     }
     const int n_slots = n_act + a.n_shared;
-    const int m_tiles = kGU ? a.I / BM : a.H / BM;
+    const int m_tiles = (kGU ? a.I : a.H) / kFeat;
     const int K = kGU ? a.H : a.I;
     const int KB = K / BK;
     const int G = K / kGroup;
@@ -246,32 +316,50 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
             const uint64_t policy = policy_evict_first();
-            int64_t it = 0;
+            Ring rs;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-                const CUtensorMap* m0 = a.wmaps + (size_t)ti.e * 3 + (kGU ? 0 : 2);
-                for (int kb = 0; kb < KB; ++kb, ++it) {
-                    const int s = (int)(it % stages);
-                    const uint32_t use = (uint32_t)(it / stages);
-                    if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
+                const CUtensorMap* wm = a.wmaps + (size_t)ti.e * 3;
+                const int f0 = ti.m_tile * kFeat;
+                // only the token rows the tile has, rounded up to 32, in at
+                // most two boxes (128 + 64 / 128 + 32 / 64 + 32 / one)
+                const int brows = (max(ti.ntok, 1) + kBRowQuant - 1) / kBRowQuant * kBRowQuant;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const int s = rs.i;
+                    if (rs.pass > 0 && !mbar_wait(&empty[s], (uint32_t)(rs.pass - 1) & 1)) {
                         timeout();
                         break;
                     }
+                    rs.next(stages);
                     uint8_t* st = stage_ptr(s);
-                    mbar_arrive_expect_tx(&full[s], NA * kPkBytes + kBBytes);
-                    uint8_t* pk = st + NA * kDqBytes + kBBytes;
-                    tma_load_2d_hint(pk, m0, kb * (BK / 2), ti.m_tile * BM, &full[s], policy);
-                    if constexpr (kGU)
-                        tma_load_2d_hint(pk + kPkBytes, a.wmaps + (size_t)ti.e * 3 + 1, kb * (BK / 2),
-                                         ti.m_tile * BM, &full[s], policy);
-                    tma_load_2d(st + NA * kDqBytes, &bmap, kb * BK, ti.b_row0, &full[s]);
+                    mbar_arrive_expect_tx(&full[s], kPkBytes + brows * BK * 2);
+                    uint8_t* pk = st + kBBytes;
+                    if constexpr (kGU) {
+                        tma_load_2d_hint(pk, wm + 0, kb * (BK / 2), f0, &full[s], policy);
+                        tma_load_2d_hint(pk + kPkBytes / 2, wm + 1, kb * (BK / 2), f0, &full[s],
+                                         policy);
+                    } else {
+                        tma_load_2d_hint(pk, wm + 2, kb * (BK / 2), f0, &full[s], policy);
+                    }
+                    int r0 = 0;
+                    if (brows - r0 >= 128) {
+                        tma_load_2d(st, &bmap128, kb * BK, ti.b_row0, &full[s]);
+                        r0 += 128;
+                    }
+                    if (brows - r0 >= 64) {
+                        tma_load_2d(st + r0 * (BK * 2), &bmap64, kb * BK, ti.b_row0 + r0, &full[s]);
+                        r0 += 64;
+                    }
+                    if (brows - r0 >= 32)
+                        tma_load_2d(st + r0 * (BK * 2), &bmap32, kb * BK, ti.b_row0 + r0, &full[s]);
                 }
             }
         }
     } else if (warp == 1) {
         // -------------------------------- MMA --------------------------------
         if (lane == 0) {
-            int64_t it = 0, lt = 0;
+            Ring rs, ra;
+            int64_t lt = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
@@ -283,27 +371,26 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
                 }
                 tc_fence_after();
                 const uint32_t idesc = idesc_f16(ti.n_mma);
-                const uint32_t d0 = tmem_base + (uint32_t)(buf * NA * BM);
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * BN);
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb, ++it) {
-                    const int s = (int)(it % stages);
-                    if (!mbar_wait(&dq_full[s], (uint32_t)(it / stages) & 1)) {
+                for (int kb = 0; kb < KB; ++kb) {
+                    const int s = rs.i, as = ra.i;
+                    if (!mbar_wait(&dq_full[as], (uint32_t)ra.pass & 1)) {
                         timeout();
                         ok = false;
                         break;
                     }
+                    rs.next(stages);
+                    ra.next(kAStages);
                     tc_fence_after();
-                    const uint8_t* st = stage_ptr(s);
-                    const uint32_t b_addr = smem_addr(st + NA * kDqBytes);
+                    const uint32_t b_addr = smem_addr(stage_ptr(s));
+                    const uint32_t a0 = tmem_base + kAccCols + (uint32_t)(as * kACols);
 #pragma unroll
-                    for (int m = 0; m < NA; ++m) {
-                        const uint32_t a_addr = smem_addr(st + m * kDqBytes);
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_f16(d0 + m * BM, desc_sw128(a_addr + kk * 32),
-                                    desc_sw128(b_addr + kk * 32), idesc, (kb | kk) != 0);
-                    }
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_f16_ts(d0, a0 + kk * 8, desc_sw128(b_addr + kk * 32), idesc,
+                                   (kb | kk) != 0);
                     mma_commit(&empty[s]);
+                    mma_commit(&a_empty[as]);
                 }
                 if (!ok) break;
                 mma_commit(&acc_full[buf]);
@@ -311,106 +398,126 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------- dequant -------------------------------
-        const int row = threadIdx.x - 128;  // weight row of the tile owned by this thread
-        int64_t it = 0;
+        const int row = threadIdx.x - 128;  // MMA row of the tile owned by this thread
+        // this warp's 32 lanes of the operand ring
+        const uint32_t ta = tmem_base + ((uint32_t)(warp & 3) << 21) + kAccCols;
+        Ring rs, ra;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
             const DevExpert ex = a.experts[ti.e];
-            const int64_t srow = (int64_t)(ti.m_tile * BM + row) * G;
-            const uint16_t* sc0 = (kGU ? ex.gate_s : ex.down_s) + srow;
-            const uint16_t* sc1 = kGU ? ex.up_s + srow : nullptr;
-            uint16_t nxt0 = __ldg(sc0), nxt1 = kGU ? __ldg(sc1) : 0;
+            const int f0 = ti.m_tile * kFeat;
+            const uint16_t* sc;
+            if constexpr (kGU)
+                sc = row < kFeat ? ex.gate_s + (int64_t)(f0 + row) * G
+                                 : ex.up_s + (int64_t)(f0 + row - kFeat) * G;
+            else
+                sc = ex.down_s + (int64_t)(f0 + row) * G;
+            uint16_t nxt = __ldg(sc);
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const uint16_t cur[2] = {nxt0, nxt1};
-                if (kb + 1 < KB) {
-                    nxt0 = __ldg(sc0 + kb + 1);
-                    if (kGU) nxt1 = __ldg(sc1 + kb + 1);
-                }
-                const int s = (int)(it % stages);
-                if (!mbar_wait(&full[s], (uint32_t)(it / stages) & 1)) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const uint16_t cur = nxt;
+                if (kb + 1 < KB) nxt = __ldg(sc + kb + 1);
+                const int s = rs.i, as = ra.i;
+                if (!mbar_wait(&full[s], (uint32_t)rs.pass & 1) ||
+                    (ra.pass > 0 && !mbar_wait(&a_empty[as], (uint32_t)(ra.pass - 1) & 1))) {
                     if (lane == 0) timeout();
                     ok = false;
                     break;
                 }
-                uint8_t* st = stage_ptr(s);
+                rs.next(stages);
+                ra.next(kAStages);
+                tc_fence_after();
+                const uint4* pk = reinterpret_cast<const uint4*>(stage_ptr(s) + kBBytes + row * 32);
+                const uint4 p0 = pk[0], p1 = pk[1];
+                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                // bf16 scale -> fp16 (exact for scales in fp16's normal range)
+                const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur << 16));
+                const __half2 s2 = __halves2half2(sh, sh);
+                uint32_t cols[32];  // column 4c + i: elements i, i + 4 of 8-group c
 #pragma unroll
-                for (int m = 0; m < NA; ++m) {
-                    const uint4* pk = reinterpret_cast<const uint4*>(st + NA * kDqBytes + kBBytes +
-                                                                     m * kPkBytes + row * 32);
-                    const uint4 p0 = pk[0], p1 = pk[1];
-                    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    // bf16 scale -> fp16 (exact for scales in fp16's normal range)
-                    const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur[m] << 16));
-                    const __half2 s2 = __halves2half2(sh, sh);
-                    uint8_t* dq = st + m * kDqBytes + row * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t w = words[c], w8 = w >> 8;
-                        uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
-                        uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
-                        uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
-                        uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
-                        const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
-                        const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
-                        const __half2 hi = __floats2half2_rn(-72.f, -72.f);
-                        __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
-                        __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
-                        __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
-                        __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
-                        uint4 out;
-                        out.x = *reinterpret_cast<uint32_t*>(&v0);
-                        out.y = *reinterpret_cast<uint32_t*>(&v1);
-                        out.z = *reinterpret_cast<uint32_t*>(&v2);
-                        out.w = *reinterpret_cast<uint32_t*>(&v3);
-                        *reinterpret_cast<uint4*>(dq + ((c ^ (row & 7)) << 4)) = out;
-                    }
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t w = words[c], w8 = w >> 8;
+                    uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
+                    uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
+                    uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
+                    uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
+                    const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
+                    const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
+                    const __half2 hi = __floats2half2_rn(-72.f, -72.f);
+                    __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
+                    __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
+                    __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
+                    __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
+                    cols[4 * c + 0] = *reinterpret_cast<uint32_t*>(&v0);
+                    cols[4 * c + 1] = *reinterpret_cast<uint32_t*>(&v1);
+                    cols[4 * c + 2] = *reinterpret_cast<uint32_t*>(&v2);
+                    cols[4 * c + 3] = *reinterpret_cast<uint32_t*>(&v3);
                 }
-                fence_proxy_async();
+                tmem_st32(ta + (uint32_t)(as * kACols), cols);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dq_full[s]);
+                if (lane == 0) mbar_arrive(&dq_full[as]);
             }
             if (!ok) break;
         }
     } else if (warp >= 8) {
         // ------------------------------- epilogue ------------------------------
         const int q = warp & 3;
-        const int row = q * 32 + lane;  // accumulator lane = weight row of the tile
+        const int row = q * 32 + lane;  // accumulator lane = MMA row of the tile
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
             const int buf = (int)(lt & 1);
-            if (!mbar_wait(&acc_full[buf], (uint32_t)(lt >> 1) & 1)) {
-                if (lane == 0) timeout();
+            const bool got = mbar_wait(&acc_full[buf], (uint32_t)(lt >> 1) & 1);
+            // gate/up: the four warps agree before they meet at the exchange
+            // barriers (a wait that ran out in one of them ends all four)
+            if (kGU ? !named_barrier_and(1, 128, got) : !got) {
+                if (lane == 0 && !got) timeout();
                 break;
             }
             tc_fence_after();
-            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BM);
-            const int feat = ti.m_tile * BM + row;
-            for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
-                uint32_t v0[32];
-                tmem_ld32(tq + c0, v0);
-                if constexpr (kGU) {
-                    uint32_t v1[32];
-                    tmem_ld32(tq + BM + c0, v1);
-                    const int col = perm_col(feat);
+            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+            if constexpr (kGU) {
+                // lanes 0-63 hold gate, 64-127 up of features f0 + (row & 63):
+                // the up warps pass their values through shared memory (a
+                // 64 x 33 float block per 32 tokens, conflict-free both ways)
+                const bool gate_lane = row < kFeat;
+                const int col = perm_col(ti.m_tile * kFeat + (row & (kFeat - 1)));
+                for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tq + c0, v);
+                    if (!gate_lane) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (c0 + j < ti.ntok) {
-                            const float g = __uint_as_float(v0[j]), u = __uint_as_float(v1[j]);
-                            float hv = g / (1.f + expf(-g)) * u;
-                            if (fabsf(hv) > 65504.f) {
-                                report(a.status, COLI_ERR_RANGE);
-                                hv = copysignf(65504.f, hv);
+                        for (int j = 0; j < 32; ++j) xch[(row - kFeat) * 33 + j] = __uint_as_float(v[j]);
+                    }
+                    named_barrier(1, 128);
+                    if (gate_lane) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            if (c0 + j < ti.ntok) {
+                                const float g = __uint_as_float(v[j]), u = xch[row * 33 + j];
+                                float hv = g / (1.f + expf(-g)) * u;
+                                if (fabsf(hv) > 65504.f) {
+                                    report(a.status, COLI_ERR_RANGE);
+                                    hv = copysignf(65504.f, hv);
+                                }
+                                a.hbuf[(int64_t)(ti.out_row0 + c0 + j) * a.I + col] =
+                                    __float2half_rn(hv);
                             }
-                            a.hbuf[(int64_t)(ti.out_row0 + c0 + j) * a.I + col] = __float2half_rn(hv);
                         }
                     }
-                } else {
+                    named_barrier(1, 128);
+                }
+            } else {
+                const int feat = ti.m_tile * kFeat + row;
+                for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tq + c0, v);
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (c0 + j < ti.ntok)
-                            a.y[(int64_t)(ti.out_row0 + c0 + j) * a.H + feat] = __uint_as_float(v0[j]);
+                            a.y[(int64_t)(ti.out_row0 + c0 + j) * a.H + feat] = __uint_as_float(v[j]);
                 }
             }
             tc_fence_before();
@@ -424,7 +531,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const GemmArgs a, 
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kTmemCols)
+                     "r"(kTmemColsP)
                      : "memory");
     }
 }
@@ -528,17 +635,17 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 
 template <bool kGU>
 int gemm_stages() {
-    constexpr int NA = kGU ? 2 : 1;
-    constexpr int kStage = NA * BM * BK * 2 + BN * BK * 2 + NA * BM * BK / 2;
-    return std::min(16, (kSmemLimitP - kHeaderP - 1024) / kStage);
+    constexpr int kStage = BN * BK * 2 + BM * BK / 2;
+    const int extra = kGU ? kXchBytes : 0;
+    return std::min(16, (kSmemLimitP - kHeaderP - 1024 - extra) / kStage);
 }
 
 template <bool kGU>
-cudaError_t launch_gemm(const CUtensorMap& bmap, const GemmArgs& a, int num_sms, cudaStream_t st) {
-    constexpr int NA = kGU ? 2 : 1;
-    constexpr int kStage = NA * BM * BK * 2 + BN * BK * 2 + NA * BM * BK / 2;
+cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num_sms,
+                        cudaStream_t st) {
+    constexpr int kStage = BN * BK * 2 + BM * BK / 2;
     const int stages = gemm_stages<kGU>();
-    const int smem = kHeaderP + 1024 + stages * kStage;
+    const int smem = kHeaderP + 1024 + stages * kStage + (kGU ? kXchBytes : 0);
     cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
@@ -552,7 +659,8 @@ cudaError_t launch_gemm(const CUtensorMap& bmap, const GemmArgs& a, int num_sms,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<kGU>, bmap, a, stages);
+    return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<kGU>, bmap[0], bmap[1], bmap[2], a,
+                              stages);
 }
 
 }  // namespace
@@ -566,9 +674,9 @@ cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I
         const DevExpert& x = host_experts[e];
         const bool ok =
             encode_2d(&maps[e * 3 + 0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.gate_q, H / 2, I, H / 2,
-                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      BK / 2, BM / 2, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.up_q, H / 2, I, H / 2,
-                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      BK / 2, BM / 2, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.down_q, I / 2, H, I / 2,
                       BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (!ok) {
@@ -636,12 +744,16 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
     a.hbuf = f.hp;
     a.y = f.y;
     a.status = f.status;
-    CUtensorMap xmap, hmap;
-    if (!encode_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xg, f.H, (uint64_t)(P + f.T),
-                   (uint64_t)f.H * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, f.hp, f.I, (uint64_t)S,
-                   (uint64_t)f.I * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+    // activation / h tiles as 128-, 64- and 32-row boxes
+    CUtensorMap xmap[3], hmap[3];
+    for (int b = 0; b < 3; ++b) {
+        const uint32_t rows = 128u >> b;
+        if (!encode_2d(&xmap[b], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xg, f.H, (uint64_t)(P + f.T),
+                       (uint64_t)f.H * 2, BK, rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_2d(&hmap[b], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, f.hp, f.I, (uint64_t)S,
+                       (uint64_t)f.I * 2, BK, rows, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     profile_mark(1, st);
     cudaError_t err = launch_gemm<true>(xmap, a, num_sms, st);
     if (err != cudaSuccess) return err;
