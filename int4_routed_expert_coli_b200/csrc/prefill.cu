@@ -6,35 +6,35 @@
 // "yunpan.plus/t/30351-1-1", capability two), gate/up is
 //   [2 x I rows of int4 codes] x [n_e tokens x H]  -> h [n_e][I]
 // and down is [H rows] x [n_e x I] -> y [n_e][H].  The weight rows are the MMA
-// M dimension (128 per tile; for gate/up 64 gate rows + the up rows of the
-// same 64 features, so one MMA covers both and reads the activation tile
-// once), the tokens the N dimension (tiles of up to 192, rounded to 16, so a
-// routed expert of a 4096-token prefill is one tile and its weights are
-// dequantised once per M tile), K is walked in 64-element blocks (one gs64
-// scale group).
+// M dimension (tiles of 128 features; gate/up runs the gate and the up MMA of
+// a tile on the same activation tile, so each activation tile is loaded from
+// L2 once per 128 features), the tokens the N dimension (tiles of up to 192,
+// rounded to 16, so a routed expert of a 4096-token prefill is one tile and
+// its weights are dequantised once per M tile), K is walked in 64-element
+// blocks (one gs64 scale group).
 //
 // Pipeline (one CTA per SM, persistent over a flattened list of tiles):
-//   warp 0      TMA producer: packed int4 codes of the tile rows (2-D tensor
-//               maps per expert matrix, 32 bytes x 64 or 128 rows per K-block)
-//               and the activation rows the tile has (128-byte swizzled fp16,
-//               32-row boxes);
-//   warps 4-7   dequant: each thread owns one weight row, turns its 64 codes
-//               into fp16 q * s (exact: a 3-bit code magnitude times an 8-bit
-//               bf16 scale fits fp16's 11 bits) and stores them straight into
-//               tensor memory (tcgen05.st, lane = weight row, two fp16 per
-//               column): the weight operand never passes through shared
-//               memory, whose bandwidth the activation tile and the TMA
-//               copies need;
+//   warp 0      TMA producer: packed int4 codes of the tile rows (a 2-D tensor
+//               map per expert matrix, 32 bytes x 128 rows per K-block) and the
+//               activation rows the tile has (128-byte swizzled fp16, at most
+//               two boxes of 128/64/32 rows);
+//   warps 4-7   dequant: each thread owns one weight row (of gate and of up),
+//               turns its 64 codes into fp16 q * s (exact: a 3-bit code
+//               magnitude times an 8-bit bf16 scale fits fp16's 11 bits) and
+//               stores them straight into tensor memory (tcgen05.st, lane =
+//               weight row, two fp16 per column): the weight operand never
+//               passes through shared memory;
 //   warp 1      one thread issues tcgen05.mma (kind::f16, A from tensor
 //               memory, B from shared memory, fp32 accumulate in tensor
 //               memory) and commits stage / operand release and tile
 //               completion;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator (each warp its 32
 //               lanes), SwiGLU to fp16 h, or the fp32 y rows of the down GEMM.
-//   Tensor memory (512 columns): two 192-column accumulators (the epilogue of
-//   one tile overlaps the next tile's MMAs) and a 4-deep ring of 32-column
-//   weight operands.  The shared-memory ring of code and activation tiles is
-//   deeper than the operand ring; each has its own release barrier.
+//   Tensor memory (512 columns): accumulators in [0, 384) -- gate/up one
+//   buffer of gate (192) + up (192), drained by the epilogue before the next
+//   tile; down two 192-column buffers, so its epilogue overlaps the next
+//   tile -- and a ring of weight operands in [384, 512) (2 gate/up K-blocks
+//   of 64 columns, 4 down K-blocks of 32).
 // Every wait is bounded (COLI_ERR_TIMEOUT) so nothing can hang the GPU.
 //
 // K order.  Within each group of 8 consecutive K elements the dequant unpack
@@ -60,8 +60,7 @@ constexpr int BM = 128, BN = 192, BK = 64;
 constexpr int kBRowQuant = 32;      // activation rows are loaded in multiples of 32
 constexpr int kThreadsP = 384;
 constexpr uint32_t kTmemColsP = 512;
-constexpr uint32_t kAccCols = 2 * BN;  // two accumulators; the operand ring follows
-constexpr int kXchBytes = 64 * 33 * 4;  // gate/up epilogue exchange block
+constexpr uint32_t kAccCols = 2 * BN;  // accumulators; the operand ring follows
 constexpr int kHeaderP = 2048;
 constexpr int kSmemLimitP = 227 * 1024;
 
@@ -132,19 +131,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t v[32]) 
         "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
         "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
-}
-
-// bar.red.and over `count` threads of named barrier `id`: true iff every
-// participating thread passed true.
-__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "barrier.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
@@ -233,21 +219,21 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_
 }
 
 // ---- the GEMM kernel -------------------------------------------------------
-// kGU: gate/up.  A tile's 128 MMA rows are 64 gate rows and the up rows of the
-// same 64 features (K = H), so one MMA per K step covers both and the
-// activation tile is read once; the epilogue pairs lane f (gate) with lane
-// 64 + f (up) through shared memory.  Otherwise down: 128 rows of W_d, K = I.
+// kGU: gate/up (two MMAs per K step, gate rows and up rows of the same 128
+// features, on one activation tile; K = H).  Otherwise down: 128 rows of W_d,
+// K = I.
 template <bool kGU>
 __global__ void __launch_bounds__(kThreadsP, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     const __grid_constant__ CUtensorMap bmap64,
                     const __grid_constant__ CUtensorMap bmap32, const GemmArgs a, int stages) {
-    constexpr int kFeat = kGU ? BM / 2 : BM;                 // output features per tile
+    constexpr int NA = kGU ? 2 : 1;                          // weight matrices per tile
+    constexpr int kAccBufs = kGU ? 1 : 2;                    // x NA x BN = 384 columns
     constexpr int kBBytes = BN * BK * 2;                     // 24 KB
-    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB
-    constexpr int kStage = kBBytes + kPkBytes;
-    constexpr int kACols = BK / 2;                           // operand columns per K-block
-    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 4
+    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
+    constexpr int kStage = kBBytes + NA * kPkBytes;
+    constexpr int kACols = NA * BK / 2;                      // operand columns per K-block
+    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 2 gate/up, 4 down
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -261,7 +247,6 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 512);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
     uint8_t* stage0 = smem + kHeaderP;
-    float* xch = reinterpret_cast<float*>(stage0 + (size_t)stages * kStage);  // gate/up only
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -300,7 +285,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         n_act = 0;
     }
     const int n_slots = n_act + a.n_shared;
-    const int m_tiles = (kGU ? a.I : a.H) / kFeat;
+    const int m_tiles = (kGU ? a.I : a.H) / BM;
     const int K = kGU ? a.H : a.I;
     const int KB = K / BK;
     const int G = K / kGroup;
@@ -320,7 +305,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
                 const CUtensorMap* wm = a.wmaps + (size_t)ti.e * 3;
-                const int f0 = ti.m_tile * kFeat;
+                const int f0 = ti.m_tile * BM;
                 // only the token rows the tile has, rounded up to 32, in at
                 // most two boxes (128 + 64 / 128 + 32 / 64 + 32 / one)
                 const int brows = (max(ti.ntok, 1) + kBRowQuant - 1) / kBRowQuant * kBRowQuant;
@@ -332,11 +317,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     }
                     rs.next(stages);
                     uint8_t* st = stage_ptr(s);
-                    mbar_arrive_expect_tx(&full[s], kPkBytes + brows * BK * 2);
+                    mbar_arrive_expect_tx(&full[s], NA * kPkBytes + brows * BK * 2);
                     uint8_t* pk = st + kBBytes;
                     if constexpr (kGU) {
                         tma_load_2d_hint(pk, wm + 0, kb * (BK / 2), f0, &full[s], policy);
-                        tma_load_2d_hint(pk + kPkBytes / 2, wm + 1, kb * (BK / 2), f0, &full[s],
+                        tma_load_2d_hint(pk + kPkBytes, wm + 1, kb * (BK / 2), f0, &full[s],
                                          policy);
                     } else {
                         tma_load_2d_hint(pk, wm + 2, kb * (BK / 2), f0, &full[s], policy);
@@ -363,15 +348,15 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-                const int buf = (int)(lt & 1);
-                const uint32_t ause = (uint32_t)(lt >> 1);
+                const int buf = (int)(lt % kAccBufs);
+                const uint32_t ause = (uint32_t)(lt / kAccBufs);
                 if (ause > 0 && !mbar_wait(&acc_empty[buf], (ause - 1) & 1)) {
                     timeout();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t idesc = idesc_f16(ti.n_mma);
-                const uint32_t d0 = tmem_base + (uint32_t)(buf * BN);
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * NA * BN);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     const int s = rs.i, as = ra.i;
@@ -386,9 +371,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     const uint32_t b_addr = smem_addr(stage_ptr(s));
                     const uint32_t a0 = tmem_base + kAccCols + (uint32_t)(as * kACols);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_f16_ts(d0, a0 + kk * 8, desc_sw128(b_addr + kk * 32), idesc,
-                                   (kb | kk) != 0);
+                    for (int m = 0; m < NA; ++m)
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_f16_ts(d0 + m * BN, a0 + m * (BK / 2) + kk * 8,
+                                       desc_sw128(b_addr + kk * 32), idesc, (kb | kk) != 0);
                     mma_commit(&empty[s]);
                     mma_commit(&a_empty[as]);
                 }
@@ -405,18 +392,17 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
             const DevExpert ex = a.experts[ti.e];
-            const int f0 = ti.m_tile * kFeat;
-            const uint16_t* sc;
-            if constexpr (kGU)
-                sc = row < kFeat ? ex.gate_s + (int64_t)(f0 + row) * G
-                                 : ex.up_s + (int64_t)(f0 + row - kFeat) * G;
-            else
-                sc = ex.down_s + (int64_t)(f0 + row) * G;
-            uint16_t nxt = __ldg(sc);
+            const int64_t srow = (int64_t)(ti.m_tile * BM + row) * G;
+            const uint16_t* sc0 = (kGU ? ex.gate_s : ex.down_s) + srow;
+            const uint16_t* sc1 = kGU ? ex.up_s + srow : nullptr;
+            uint16_t nxt0 = __ldg(sc0), nxt1 = kGU ? __ldg(sc1) : 0;
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
-                const uint16_t cur = nxt;
-                if (kb + 1 < KB) nxt = __ldg(sc + kb + 1);
+                const uint16_t cur[2] = {nxt0, nxt1};
+                if (kb + 1 < KB) {
+                    nxt0 = __ldg(sc0 + kb + 1);
+                    if (kGU) nxt1 = __ldg(sc1 + kb + 1);
+                }
                 const int s = rs.i, as = ra.i;
                 if (!mbar_wait(&full[s], (uint32_t)rs.pass & 1) ||
                     (ra.pass > 0 && !mbar_wait(&a_empty[as], (uint32_t)(ra.pass - 1) & 1))) {
@@ -427,33 +413,37 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                 rs.next(stages);
                 ra.next(kAStages);
                 tc_fence_after();
-                const uint4* pk = reinterpret_cast<const uint4*>(stage_ptr(s) + kBBytes + row * 32);
-                const uint4 p0 = pk[0], p1 = pk[1];
-                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                // bf16 scale -> fp16 (exact for scales in fp16's normal range)
-                const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur << 16));
-                const __half2 s2 = __halves2half2(sh, sh);
-                uint32_t cols[32];  // column 4c + i: elements i, i + 4 of 8-group c
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t w = words[c], w8 = w >> 8;
-                    uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
-                    uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
-                    uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
-                    uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
-                    const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
-                    const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
-                    const __half2 hi = __floats2half2_rn(-72.f, -72.f);
-                    __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
-                    __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
-                    __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
-                    __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
-                    cols[4 * c + 0] = *reinterpret_cast<uint32_t*>(&v0);
-                    cols[4 * c + 1] = *reinterpret_cast<uint32_t*>(&v1);
-                    cols[4 * c + 2] = *reinterpret_cast<uint32_t*>(&v2);
-                    cols[4 * c + 3] = *reinterpret_cast<uint32_t*>(&v3);
+                for (int m = 0; m < NA; ++m) {
+                    const uint4* pk = reinterpret_cast<const uint4*>(stage_ptr(s) + kBBytes +
+                                                                     m * kPkBytes + row * 32);
+                    const uint4 p0 = pk[0], p1 = pk[1];
+                    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    // bf16 scale -> fp16 (exact for scales in fp16's normal range)
+                    const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur[m] << 16));
+                    const __half2 s2 = __halves2half2(sh, sh);
+                    uint32_t cols[32];  // column 4c + i: elements i, i + 4 of 8-group c
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t w = words[c], w8 = w >> 8;
+                        uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
+                        uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
+                        uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
+                        uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
+                        const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
+                        const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
+                        const __half2 hi = __floats2half2_rn(-72.f, -72.f);
+                        __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
+                        __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
+                        __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
+                        __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
+                        cols[4 * c + 0] = *reinterpret_cast<uint32_t*>(&v0);
+                        cols[4 * c + 1] = *reinterpret_cast<uint32_t*>(&v1);
+                        cols[4 * c + 2] = *reinterpret_cast<uint32_t*>(&v2);
+                        cols[4 * c + 3] = *reinterpret_cast<uint32_t*>(&v3);
+                    }
+                    tmem_st32(ta + (uint32_t)(as * kACols + m * (BK / 2)), cols);
                 }
-                tmem_st32(ta + (uint32_t)(as * kACols), cols);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -468,49 +458,38 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-            const int buf = (int)(lt & 1);
-            const bool got = mbar_wait(&acc_full[buf], (uint32_t)(lt >> 1) & 1);
-            // gate/up: the four warps agree before they meet at the exchange
-            // barriers (a wait that ran out in one of them ends all four)
-            if (kGU ? !named_barrier_and(1, 128, got) : !got) {
-                if (lane == 0 && !got) timeout();
+            const int buf = (int)(lt % kAccBufs);
+            if (!mbar_wait(&acc_full[buf], (uint32_t)(lt / kAccBufs) & 1)) {
+                if (lane == 0) timeout();
                 break;
             }
             tc_fence_after();
-            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BN);
+            const int feat = ti.m_tile * BM + row;
             if constexpr (kGU) {
-                // lanes 0-63 hold gate, 64-127 up of features f0 + (row & 63):
-                // the up warps pass their values through shared memory (a
-                // 64 x 33 float block per 32 tokens, conflict-free both ways)
-                const bool gate_lane = row < kFeat;
-                const int col = perm_col(ti.m_tile * kFeat + (row & (kFeat - 1)));
+                // gate and up of this lane's feature sit in the same lane; the
+                // next tile's MMAs wait for this (single accumulator buffer),
+                // so SiLU uses the fast exponential and division
+                const int col = perm_col(feat);
+                __half* hcol = a.hbuf + (int64_t)ti.out_row0 * a.I + col;
                 for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tq + c0, v);
-                    if (!gate_lane) {
+                    uint32_t vg[32], vu[32];
+                    tmem_ld32(tq + c0, vg);
+                    tmem_ld32(tq + BN + c0, vu);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) xch[(row - kFeat) * 33 + j] = __uint_as_float(v[j]);
-                    }
-                    named_barrier(1, 128);
-                    if (gate_lane) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            if (c0 + j < ti.ntok) {
-                                const float g = __uint_as_float(v[j]), u = xch[row * 33 + j];
-                                float hv = g / (1.f + expf(-g)) * u;
-                                if (fabsf(hv) > 65504.f) {
-                                    report(a.status, COLI_ERR_RANGE);
-                                    hv = copysignf(65504.f, hv);
-                                }
-                                a.hbuf[(int64_t)(ti.out_row0 + c0 + j) * a.I + col] =
-                                    __float2half_rn(hv);
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < ti.ntok) {
+                            const float g = __uint_as_float(vg[j]), u = __uint_as_float(vu[j]);
+                            float hv = __fdividef(g, 1.f + __expf(-g)) * u;
+                            if (!(fabsf(hv) <= 65504.f)) {
+                                report(a.status, COLI_ERR_RANGE);
+                                hv = copysignf(65504.f, hv);
                             }
+                            hcol[(int64_t)(c0 + j) * a.I] = __float2half_rn(hv);
                         }
                     }
-                    named_barrier(1, 128);
                 }
             } else {
-                const int feat = ti.m_tile * kFeat + row;
                 for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld32(tq + c0, v);
@@ -635,17 +614,16 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 
 template <bool kGU>
 int gemm_stages() {
-    constexpr int kStage = BN * BK * 2 + BM * BK / 2;
-    const int extra = kGU ? kXchBytes : 0;
-    return std::min(16, (kSmemLimitP - kHeaderP - 1024 - extra) / kStage);
+    constexpr int kStage = BN * BK * 2 + (kGU ? 2 : 1) * BM * BK / 2;
+    return std::min(16, (kSmemLimitP - kHeaderP - 1024) / kStage);
 }
 
 template <bool kGU>
 cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num_sms,
                         cudaStream_t st) {
-    constexpr int kStage = BN * BK * 2 + BM * BK / 2;
+    constexpr int kStage = BN * BK * 2 + (kGU ? 2 : 1) * BM * BK / 2;
     const int stages = gemm_stages<kGU>();
-    const int smem = kHeaderP + 1024 + stages * kStage + (kGU ? kXchBytes : 0);
+    const int smem = kHeaderP + 1024 + stages * kStage;
     cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
@@ -674,9 +652,9 @@ cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I
         const DevExpert& x = host_experts[e];
         const bool ok =
             encode_2d(&maps[e * 3 + 0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.gate_q, H / 2, I, H / 2,
-                      BK / 2, BM / 2, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.up_q, H / 2, I, H / 2,
-                      BK / 2, BM / 2, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.down_q, I / 2, H, I / 2,
                       BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (!ok) {
