@@ -28,8 +28,10 @@
 //               memory, B from shared memory, fp32 accumulate in tensor
 //               memory) and commits stage / operand release and tile
 //               completion;
-//   warps 8-11  epilogue: tcgen05.ld of the accumulator (each warp its 32
-//               lanes), SwiGLU to fp16 h, or the fp32 y rows of the down GEMM.
+//   warps 8-15  epilogue: tcgen05.ld of the accumulator (a warp reads the 32
+//               lanes of its quarter, the two warps of a quarter alternate
+//               32-token chunks), SwiGLU to fp16 h, or the fp32 y rows of the
+//               down GEMM.
 //   Tensor memory (512 columns): accumulators in [0, 384) -- gate/up one
 //   buffer of gate (192) + up (192), drained by the epilogue before the next
 //   tile; down two 192-column buffers, so its epilogue overlaps the next
@@ -58,7 +60,8 @@ namespace {
 
 constexpr int BM = 128, BN = 192, BK = 64;
 constexpr int kBRowQuant = 32;      // activation rows are loaded in multiples of 32
-constexpr int kThreadsP = 384;
+constexpr int kThreadsP = 512;
+constexpr int kEpiWarps = 8;  // warps 8-15: two per tensor-memory lane quarter
 constexpr uint32_t kTmemColsP = 512;
 constexpr uint32_t kAccCols = 2 * BN;  // accumulators; the operand ring follows
 constexpr int kHeaderP = 2048;
@@ -85,13 +88,21 @@ __device__ __forceinline__ uint32_t idesc_f16(int n) {
            | ((uint32_t)(BM >> 4) << 24);     // M = 128; A, B: f16, K-major
 }
 
-// A (the dequantised weights) from tensor memory, B from shared memory.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                           uint32_t idesc, uint32_t accumulate) {
+// The four K=16 MMAs of one 64-wide K-block: A columns a, a + 8, a + 16,
+// a + 24; the B descriptor advanced by 32 bytes (two 16-byte units) each.
+// The first accumulates into d unless `accumulate` is 0, the others always.
+__device__ __forceinline__ void mma_kblock_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+        "{\n\t.reg .pred p, t;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a1, a2, a3;\n\t"
+        "setp.ne.u32 p, %4, 0;\n\tsetp.ne.u32 t, %5, 0;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(1u));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -260,7 +271,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], kEpiWarps);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -368,14 +379,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     rs.next(stages);
                     ra.next(kAStages);
                     tc_fence_after();
-                    const uint32_t b_addr = smem_addr(stage_ptr(s));
+                    const uint64_t bdesc = desc_sw128(smem_addr(stage_ptr(s)));
                     const uint32_t a0 = tmem_base + kAccCols + (uint32_t)(as * kACols);
 #pragma unroll
                     for (int m = 0; m < NA; ++m)
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_f16_ts(d0 + m * BN, a0 + m * (BK / 2) + kk * 8,
-                                       desc_sw128(b_addr + kk * 32), idesc, (kb | kk) != 0);
+                        mma_kblock_ts(d0 + m * BN, a0 + m * (BK / 2), bdesc, idesc, kb != 0);
                     mma_commit(&empty[s]);
                     mma_commit(&a_empty[as]);
                 }
@@ -454,6 +462,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     } else if (warp >= 8) {
         // ------------------------------- epilogue ------------------------------
         const int q = warp & 3;
+        const int c_first = ((warp - 8) >> 2) * 32;  // the two warps of a quarter take
+                                                     // alternate 32-token chunks
         const int row = q * 32 + lane;  // accumulator lane = MMA row of the tile
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
@@ -472,7 +482,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                 // so SiLU uses the fast exponential and division
                 const int col = perm_col(feat);
                 __half* hcol = a.hbuf + (int64_t)ti.out_row0 * a.I + col;
-                for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
+                for (int c0 = c_first; c0 < ti.ntok; c0 += 64) {
                     uint32_t vg[32], vu[32];
                     tmem_ld32(tq + c0, vg);
                     tmem_ld32(tq + BN + c0, vu);
@@ -490,7 +500,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     }
                 }
             } else {
-                for (int c0 = 0; c0 < ti.ntok; c0 += 32) {
+                for (int c0 = c_first; c0 < ti.ntok; c0 += 64) {
                     uint32_t v[32];
                     tmem_ld32(tq + c0, v);
 #pragma unroll
