@@ -529,7 +529,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
 // xg[s] = fp16(x[pairs[s] / k]) for s < P (the union's order), xg[P + t] =
 // fp16(x[t]) (the shared experts' rows), columns in operand order.  Block 0
 // also lays out the tile list: ntile_start[slot] = sum over earlier slots of
-// ceil(tokens / 128).
+// ceil(tokens / BN).
 __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
     pdl_wait();
     pdl_launch_dependents();
@@ -558,12 +558,14 @@ __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
         if (s0 + 1 <= n_slots) g.ntile_start[s0 + 1] = base + cnt[0];
         return;
     }
+    // the other blocks: four rows per pass (256 threads per row), no
+    // per-element division; a row's token index is one broadcast load
     const int chunks = g.H / 8;
-    const int64_t n = (int64_t)(P + g.T) * chunks;
-    for (int64_t i = (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)(gridDim.x - 1) * blockDim.x) {
-        const int64_t s = i / chunks;
-        const int c = (int)(i % chunks);
+    const int64_t rows = P + g.T;
+    const int sub = threadIdx.x >> 8, lt = threadIdx.x & 255;
+    for (int64_t s0 = (int64_t)(blockIdx.x - 1) * 4; s0 < rows; s0 += (int64_t)(gridDim.x - 1) * 4) {
+        const int64_t s = s0 + sub;
+        if (s >= rows) continue;
         int t;
         if (s < P) {
             const int p = g.pairs[s];
@@ -571,25 +573,27 @@ __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
         } else {
             t = (int)(s - P);
         }
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (t >= 0) {
-            const uint4 in = *reinterpret_cast<const uint4*>(
-                reinterpret_cast<const uint16_t*>(g.x) + (int64_t)t * g.H + c * 8);
-            const uint16_t* v = reinterpret_cast<const uint16_t*>(&in);
-            uint16_t o[8];
+        for (int c = lt; c < chunks; c += 256) {
+            uint4 out = make_uint4(0, 0, 0, 0);
+            if (t >= 0) {
+                const uint4 in = *reinterpret_cast<const uint4*>(
+                    reinterpret_cast<const uint16_t*>(g.x) + (int64_t)t * g.H + c * 8);
+                const uint16_t* v = reinterpret_cast<const uint16_t*>(&in);
+                uint16_t o[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float f = __uint_as_float((uint32_t)v[j] << 16);
-                if (fabsf(f) > 65504.f) {
-                    report(g.status, COLI_ERR_RANGE);
-                    f = copysignf(65504.f, f);
+                for (int j = 0; j < 8; ++j) {
+                    float f = __uint_as_float((uint32_t)v[j] << 16);
+                    if (fabsf(f) > 65504.f) {
+                        report(g.status, COLI_ERR_RANGE);
+                        f = copysignf(65504.f, f);
+                    }
+                    const __half h = __float2half_rn(f);
+                    o[perm8(j)] = *reinterpret_cast<const uint16_t*>(&h);
                 }
-                const __half h = __float2half_rn(f);
-                o[perm8(j)] = *reinterpret_cast<const uint16_t*>(&h);
+                out = *reinterpret_cast<uint4*>(o);
             }
-            out = *reinterpret_cast<uint4*>(o);
+            *reinterpret_cast<uint4*>(g.xg + s * g.H + c * 8) = out;
         }
-        *reinterpret_cast<uint4*>(g.xg + s * g.H + c * 8) = out;
     }
 }
 
@@ -702,8 +706,8 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
     g.ntile_start = ntile_start;
     g.status = f.status;
     {
-        const int64_t n = (int64_t)(P + f.T) * (f.H / 8);
-        const int blocks = 1 + (int)std::min<int64_t>((n + 1023) / 1024, (int64_t)num_sms * 2);
+        const int64_t rows = P + f.T;
+        const int blocks = 1 + (int)std::min<int64_t>((rows + 3) / 4, (int64_t)num_sms * 2);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(blocks);
         cfg.blockDim = dim3(1024);
