@@ -6,9 +6,10 @@
 // "yunpan.plus/t/30351-1-1", capability two), gate/up is
 //   [2 x I rows of int4 codes] x [n_e tokens x H]  -> h [n_e][I]
 // and down is [H rows] x [n_e x I] -> y [n_e][H].  The weight rows are the MMA
-// M dimension (tiles of 128 features; gate/up runs the gate and the up MMA of
-// a tile on the same activation tile, so each activation tile is loaded from
-// L2 once per 128 features), the tokens the N dimension (tiles of up to 192,
+// M dimension (128 per MMA; a tile runs two MMAs on the same activation tile:
+// gate and up of 128 features, or two 128-row blocks of W_d, so each
+// activation tile is loaded from L2 once per 256 weight rows), the tokens the
+// N dimension (tiles of up to 192,
 // rounded to 16, so a routed expert of a 4096-token prefill is one tile and
 // its weights are dequantised once per M tile), K is walked in 64-element
 // blocks (one gs64 scale group).
@@ -18,7 +19,7 @@
 //               map per expert matrix, 32 bytes x 128 rows per K-block) and the
 //               activation rows the tile has (128-byte swizzled fp16, at most
 //               two boxes of 128/64/32 rows);
-//   warps 4-7   dequant: each thread owns one weight row (of gate and of up),
+//   warps 4-7   dequant: each thread owns one weight row of each block,
 //               turns its 64 codes into fp16 q * s (exact: a 3-bit code
 //               magnitude times an 8-bit bf16 scale fits fp16's 11 bits) and
 //               stores them straight into tensor memory (tcgen05.st, lane =
@@ -32,11 +33,9 @@
 //               lanes of its quarter, the two warps of a quarter alternate
 //               32-token chunks), SwiGLU to fp16 h, or the fp32 y rows of the
 //               down GEMM.
-//   Tensor memory (512 columns): accumulators in [0, 384) -- gate/up one
-//   buffer of gate (192) + up (192), drained by the epilogue before the next
-//   tile; down two 192-column buffers, so its epilogue overlaps the next
-//   tile -- and a ring of weight operands in [384, 512) (2 gate/up K-blocks
-//   of 64 columns, 4 down K-blocks of 32).
+//   Tensor memory (512 columns): one accumulator of two 192-column blocks in
+//   [0, 384), drained by the epilogue before the next tile's MMAs, and a ring
+//   of weight operands in [384, 512) (2 K-blocks of 2 x 32 columns).
 // Every wait is bounded (COLI_ERR_TIMEOUT) so nothing can hang the GPU.
 //
 // K order.  Within each group of 8 consecutive K elements the dequant unpack
@@ -230,16 +229,16 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_
 }
 
 // ---- the GEMM kernel -------------------------------------------------------
-// kGU: gate/up (two MMAs per K step, gate rows and up rows of the same 128
-// features, on one activation tile; K = H).  Otherwise down: 128 rows of W_d,
-// K = I.
+// Two MMAs per K step on one activation tile: kGU gate/up (the gate rows and
+// the up rows of the same 128 features, K = H), otherwise down (two blocks of
+// 128 rows of W_d, 256 output features, K = I).
 template <bool kGU>
 __global__ void __launch_bounds__(kThreadsP, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     const __grid_constant__ CUtensorMap bmap64,
                     const __grid_constant__ CUtensorMap bmap32, const GemmArgs a, int stages) {
-    constexpr int NA = kGU ? 2 : 1;                          // weight matrices per tile
-    constexpr int kAccBufs = kGU ? 1 : 2;                    // x NA x BN = 384 columns
+    constexpr int NA = 2;                                    // weight blocks per tile
+    constexpr int kFeat = kGU ? BM : 2 * BM;                 // output features per tile
     constexpr int kBBytes = BN * BK * 2;                     // 24 KB
     constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
     constexpr int kStage = kBBytes + NA * kPkBytes;
@@ -296,7 +295,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         n_act = 0;
     }
     const int n_slots = n_act + a.n_shared;
-    const int m_tiles = (kGU ? a.I : a.H) / BM;
+    const int m_tiles = kGU ? a.I / BM : (a.H + kFeat - 1) / kFeat;
     const int K = kGU ? a.H : a.I;
     const int KB = K / BK;
     const int G = K / kGroup;
@@ -316,7 +315,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
                 const CUtensorMap* wm = a.wmaps + (size_t)ti.e * 3;
-                const int f0 = ti.m_tile * BM;
+                const int f0 = ti.m_tile * kFeat;
                 // only the token rows the tile has, rounded up to 32, in at
                 // most two boxes (128 + 64 / 128 + 32 / 64 + 32 / one)
                 const int brows = (max(ti.ntok, 1) + kBRowQuant - 1) / kBRowQuant * kBRowQuant;
@@ -335,7 +334,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                         tma_load_2d_hint(pk + kPkBytes, wm + 1, kb * (BK / 2), f0, &full[s],
                                          policy);
                     } else {
+                        // the second block may lie past H (zero-filled codes)
                         tma_load_2d_hint(pk, wm + 2, kb * (BK / 2), f0, &full[s], policy);
+                        tma_load_2d_hint(pk + kPkBytes, wm + 2, kb * (BK / 2), f0 + BM, &full[s],
+                                         policy);
                     }
                     int r0 = 0;
                     if (brows - r0 >= 128) {
@@ -359,8 +361,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-                const int buf = (int)(lt % kAccBufs);
-                const uint32_t ause = (uint32_t)(lt / kAccBufs);
+                const int buf = 0;  // one accumulator (NA x BN = 384 columns)
+                const uint32_t ause = (uint32_t)lt;
                 if (ause > 0 && !mbar_wait(&acc_empty[buf], (ause - 1) & 1)) {
                     timeout();
                     break;
@@ -400,16 +402,21 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
             const DevExpert ex = a.experts[ti.e];
-            const int64_t srow = (int64_t)(ti.m_tile * BM + row) * G;
+            // gate/up: gate and up row of feature f0 + row; down: W_d rows
+            // f0 + row and f0 + 128 + row (the latter past H in a ragged last
+            // tile: scale 0, and its codes are zero-filled)
+            const int f0 = ti.m_tile * kFeat;
+            const int64_t srow = (int64_t)(f0 + row) * G;
+            const bool has1 = kGU || f0 + BM < a.H;
             const uint16_t* sc0 = (kGU ? ex.gate_s : ex.down_s) + srow;
-            const uint16_t* sc1 = kGU ? ex.up_s + srow : nullptr;
-            uint16_t nxt0 = __ldg(sc0), nxt1 = kGU ? __ldg(sc1) : 0;
+            const uint16_t* sc1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * G;
+            uint16_t nxt0 = __ldg(sc0), nxt1 = has1 ? __ldg(sc1) : 0;
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
                 const uint16_t cur[2] = {nxt0, nxt1};
                 if (kb + 1 < KB) {
                     nxt0 = __ldg(sc0 + kb + 1);
-                    if (kGU) nxt1 = __ldg(sc1 + kb + 1);
+                    if (has1) nxt1 = __ldg(sc1 + kb + 1);
                 }
                 const int s = rs.i, as = ra.i;
                 if (!mbar_wait(&full[s], (uint32_t)rs.pass & 1) ||
@@ -468,14 +475,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-            const int buf = (int)(lt % kAccBufs);
-            if (!mbar_wait(&acc_full[buf], (uint32_t)(lt / kAccBufs) & 1)) {
+            const int buf = 0;
+            if (!mbar_wait(&acc_full[buf], (uint32_t)lt & 1)) {
                 if (lane == 0) timeout();
                 break;
             }
             tc_fence_after();
             const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BN);
-            const int feat = ti.m_tile * BM + row;
+            const int feat = ti.m_tile * kFeat + row;
             if constexpr (kGU) {
                 // gate and up of this lane's feature sit in the same lane; the
                 // next tile's MMAs wait for this (single accumulator buffer),
@@ -500,13 +507,19 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     }
                 }
             } else {
+                const bool has1 = feat + BM < a.H;
+                float* yrow = a.y + (int64_t)ti.out_row0 * a.H + feat;
                 for (int c0 = c_first; c0 < ti.ntok; c0 += 64) {
-                    uint32_t v[32];
-                    tmem_ld32(tq + c0, v);
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tq + c0, v0);
+                    tmem_ld32(tq + BN + c0, v1);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < ti.ntok)
-                            a.y[(int64_t)(ti.out_row0 + c0 + j) * a.H + feat] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < ti.ntok) {
+                            yrow[(int64_t)(c0 + j) * a.H] = __uint_as_float(v0[j]);
+                            if (has1) yrow[(int64_t)(c0 + j) * a.H + BM] = __uint_as_float(v1[j]);
+                        }
+                    }
                 }
             }
             tc_fence_before();
@@ -628,14 +641,14 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 
 template <bool kGU>
 int gemm_stages() {
-    constexpr int kStage = BN * BK * 2 + (kGU ? 2 : 1) * BM * BK / 2;
+    constexpr int kStage = BN * BK * 2 + 2 * BM * BK / 2;
     return std::min(16, (kSmemLimitP - kHeaderP - 1024) / kStage);
 }
 
 template <bool kGU>
 cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num_sms,
                         cudaStream_t st) {
-    constexpr int kStage = BN * BK * 2 + (kGU ? 2 : 1) * BM * BK / 2;
+    constexpr int kStage = BN * BK * 2 + 2 * BM * BK / 2;
     const int stages = gemm_stages<kGU>();
     const int smem = kHeaderP + 1024 + stages * kStage;
     cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU>,
