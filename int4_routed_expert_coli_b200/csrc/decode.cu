@@ -51,6 +51,7 @@ constexpr int kCW = 11;                      // consumer warps (12 warps in all)
 constexpr int kThreadsD = (kCW + 1) * 32;    // + producer warp
 constexpr int kStagesD = 3;
 constexpr int kRedBufs = 4;
+constexpr int kRedLag = 2;  // item j is summed by warp j % kCW while it works on item j + 2
 constexpr int kSmemLimitD = 227 * 1024;
 constexpr int kGuRows = 8;                   // gate rows (and up rows) per gate/up item
 constexpr int kDnRows = 16;                  // rows per down tile
@@ -260,6 +261,7 @@ struct Smem {
     volatile int* n_slots;
     volatile int* stage_item;  // [kStagesD] gate/up item in the stage; -1: a down stage
     int* red_cnt;      // [kRedBufs] partials written into each reduction buffer
+    volatile int* red_item;  // [kRedBufs] the item whose partials a buffer holds
     float* red;        // reduction buffers; during the prologue, the logits
     float* corr;       // [groups][4 lanes][4]: negated offset sums, C-fragment order
     int* s_idx;        // [T*k] routing
@@ -282,6 +284,7 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L, int max_sl
     S.n_slots = S.abort_flag + 1;
     S.red_cnt = reinterpret_cast<int*>(smem + 528);
     S.stage_item = reinterpret_cast<volatile int*>(smem + 560);
+    S.red_item = reinterpret_cast<volatile int*>(smem + 576);
     S.red = reinterpret_cast<float*>(smem + L.red_off);
     S.corr = reinterpret_cast<float*>(smem + L.corr_off);
     S.s_idx = reinterpret_cast<int*>(smem + L.route_off);
@@ -477,25 +480,47 @@ __device__ __forceinline__ void fail(const Ctx& x, int lane) {
     }
 }
 
-// Partials of item j -> reduction buffer.  The warp that writes the last
-// partial sums them (in warp order, so the result does not depend on which
-// warp that is) and gets 1 with the sums in v; the others get 0 and move on
-// at once (-1: timeout).
-__device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&acc)[4],
-                                           float (&v)[4]) {
+// Partials of item j -> reduction buffer j % kRedBufs (once the sum of item
+// j - kRedBufs has released it).  false: timeout.
+__device__ __forceinline__ bool post_partial(const Ctx& x, int j, int item,
+                                             const float (&acc)[4]) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rb = j % kRedBufs, ruse = j / kRedBufs;
-    if (ruse > 0 && !mbar_wait(&x.S.red_empty[rb], (ruse - 1) & 1)) return -1;
+    if (ruse > 0 && !mbar_wait(&x.S.red_empty[rb], (ruse - 1) & 1)) return false;
     // [warp][lane] float4 per buffer: one 16-byte store per lane
     const uint32_t rbuf = smem_addr(x.S.red) + (rb * (kCW * 4 * 32) + lane * 4) * 4;
     sts_f4(rbuf + warp * 512, make_float4(acc[0], acc[1], acc[2], acc[3]));
+    if (lane == 0) x.S.red_item[rb] = item;
     __threadfence_block();
     __syncwarp();
-    int arrived = 0;
-    if (lane == 0) arrived = atomicAdd(x.S.red_cnt + rb, 1);
-    arrived = __shfl_sync(0xffffffffu, arrived, 0);
-    if (arrived != kCW - 1) return 0;
+    if (lane == 0) atomicAdd(x.S.red_cnt + rb, 1);
+    return true;
+}
+
+// Sum of item m (its kCW partials in warp order, so the result does not
+// depend on timing) and its epilogue h' = w * silu(g) * u for the slot's
+// tokens, by warp m % kCW kRedLag items later: off the critical path of the
+// warp that finished item m last.  The tile is then counted in this CTA's
+// done_local (a CTA-scope release); the producer thread publishes the counts
+// GPU-wide.  false: timeout or abort.
+__device__ bool finish_item(const Ctx& x, int m) {
+    const FfnArgs& a = x.a;
+    const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+    const int rb = m % kRedBufs;
+    const volatile int* cnt = x.S.red_cnt + rb;
+    if (*cnt != kCW) {
+        const uint64_t t0 = global_timer_ns();
+        while (*cnt != kCW) {
+            if (*x.S.abort_flag) return false;
+            __nanosleep(64);
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                fail(x, lane);
+                return false;
+            }
+        }
+    }
     __threadfence_block();
+    const uint32_t rbuf = smem_addr(x.S.red) + (rb * (kCW * 4 * 32) + lane * 4) * 4;
     float4 sum = lds_f4(rbuf);
 #pragma unroll
     for (int w = 1; w < kCW; ++w) {
@@ -505,27 +530,49 @@ __device__ __forceinline__ int reduce_item(const Ctx& x, int j, const float (&ac
         sum.z += p.z;
         sum.w += p.w;
     }
-    v[0] = sum.x;
-    v[1] = sum.y;
-    v[2] = sum.z;
-    v[3] = sum.w;
+    const int item = x.S.red_item[rb];
     __syncwarp();
     if (lane == 0) {
         x.S.red_cnt[rb] = 0;
         mbar_arrive(&x.S.red_empty[rb]);
     }
-    return 1;
+    const int slot = item / x.gu_tiles, tile = item - slot * x.gu_tiles;
+    const SlotEntry* en = x.S.table + slot;
+    if (en->e < 0) return true;
+    const float v[4] = {sum.x, sum.y, sum.z, sum.w};
+    const int n = tile * kGuRows + r;
+    const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
+    const int list_begin = en->list_begin;
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+        const int t = 2 * c + e2;
+        if (t >= a.T) continue;
+        const int p = en->pos[t];
+        if (p < 0) continue;
+        const float gv = v[e2], uv = v[2 + e2];
+        float h = en->w[t] * (gv / (1.f + expf(-gv)) * uv);
+        if (fabsf(h) > 65504.f) {
+            report(a.status, COLI_ERR_RANGE);
+            h = copysignf(65504.f, h);
+        }
+        a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn(h);
+    }
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(x.S.done_local + slot, 1);
+    }
+    return true;
 }
 
 // One gate/up item, staged in stage j % kStagesD (its full barrier already
-// passed).  Returns false when the kernel must wind down.  The reducing warp
-// writes h' and counts the tile in this CTA's done_local (a CTA-scope
-// release); the producer thread publishes the counts GPU-wide, so the
-// GPU-scope fence stalls no consumer.
-__device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, int j,
+// passed): this warp's partial sums, posted for the item's reducing warp;
+// then, if this warp reduces item j - kRedLag, that item's sum and epilogue.
+// Returns false when the kernel must wind down.
+__device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
                                             const uint32_t (&breg)[kMaxGW][8],
                                             const int (&coff)[kMaxGW], int g_lo) {
-    const FfnArgs& a = x.a;
+    const int slot = item / x.gu_tiles;
     const Layout& L = x.L;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int stage = j % kStagesD;
@@ -584,36 +631,12 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int slot, int tile, in
     __syncwarp();
     if (lane == 0) mbar_arrive(&x.S.empty[stage]);
 
-    float v[4];
-    const int red = reduce_item(x, j, acc, v);
-    if (red < 0) {
+    if (!post_partial(x, j, item, acc)) {
         fail(x, lane);
         return false;
     }
-    if (red == 0 || !valid) return true;
-    // ---- epilogue (one warp): h' = w * silu(g) * u for the slot's tokens ----
-    const int n = tile * kGuRows + r;
-    const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
-    const int list_begin = en->list_begin;
-#pragma unroll
-    for (int e2 = 0; e2 < 2; ++e2) {
-        const int t = 2 * c + e2;
-        if (t >= a.T) continue;
-        const int p = en->pos[t];
-        if (p < 0) continue;
-        const float gv = v[e2], uv = v[2 + e2];
-        float h = en->w[t] * (gv / (1.f + expf(-gv)) * uv);
-        if (fabsf(h) > 65504.f) {
-            report(a.status, COLI_ERR_RANGE);
-            h = copysignf(65504.f, h);
-        }
-        a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn(h);
-    }
-    __syncwarp();
-    if (lane == 0) {
-        __threadfence_block();
-        atomicAdd(x.S.done_local + slot, 1);
-    }
+    const int m = j - kRedLag;
+    if (m >= 0 && m % kCW == (int)(threadIdx.x >> 5)) return finish_item(x, m);
     return true;
 }
 
@@ -1015,11 +1038,13 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         }
         const int item = S.stage_item[stage];
         if (item < 0) break;
-        const int slot = item / gu_tiles;
-        alive = gateup_item(ctx, slot, item - slot * gu_tiles, j, breg, coff, gg_lo);
+        alive = gateup_item(ctx, item, j, breg, coff, gg_lo);
         ++j;
         if (!alive) break;
     }
+    // the sums of the last kRedLag items
+    for (int m = j - kRedLag; alive && m < j; ++m)
+        if (m >= 0 && m % kCW == warp) alive = finish_item(ctx, m);
 
     // phase 2: down + combine over this CTA's output tiles, slot by slot;
     // h' fragments of the next slot are loaded while this one is computed
