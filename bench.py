@@ -60,7 +60,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one fused decode launch, from the ncu capture
 # summarised in profiles/decode_fused_kernel_glm_t1.md (tokens per step ->
 # bytes); a workload without a capture of the current kernel reports null.
-FUSED_DECODE_DRAM_BYTES = {1: 180_604_928 + 3_590_912}
+FUSED_DECODE_DRAM_BYTES = {1: 180_612_608 + 3_990_272}
 PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 
 
