@@ -553,65 +553,66 @@ __global__ void combine_kernel(const FfnArgs a) {
 }
 
 // The same combine, four consecutive outputs per thread and one token per
-// grid row (no per-element division; 16-byte loads of y).  Same operations in
+// grid row at a time (no per-element division; 16-byte loads of y).  Same operations in
 // the same order per element, so the result equals combine_kernel's bit for
 // bit.  Needs H % 4 == 0 and 16-byte aligned y, out and residual (8-byte for
 // bf16 out / residual).
 __global__ void __launch_bounds__(256) combine_vec_kernel(const FfnArgs a) {
     pdl_wait();
     const int H = a.H, k = a.k, P = a.T * a.k;
-    const int t = blockIdx.y;
     const int m = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (m >= H) return;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-        const int s = __ldg(a.inv + t * k + j);
-        if (s < 0 || s >= P) {
-            report(a.status, COLI_ERR_BAD_INDEX);
-            continue;
+    for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j) {
+            const int s = __ldg(a.inv + t * k + j);
+            if (s < 0 || s >= P) {
+                report(a.status, COLI_ERR_BAD_INDEX);
+                continue;
+            }
+            const float w = __ldg(a.topk_w + t * k + j);
+            const float4 v = __ldg(reinterpret_cast<const float4*>(a.y + (int64_t)s * H + m));
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
         }
-        const float w = __ldg(a.topk_w + t * k + j);
-        const float4 v = __ldg(reinterpret_cast<const float4*>(a.y + (int64_t)s * H + m));
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1]);
-        acc[2] = fmaf(w, v.z, acc[2]);
-        acc[3] = fmaf(w, v.w, acc[3]);
-    }
-    for (int sh = 0; sh < a.n_shared; ++sh) {
-        const float4 v =
-            __ldg(reinterpret_cast<const float4*>(a.y + (int64_t)(P + sh * a.T + t) * H + m));
-        acc[0] += v.x;
-        acc[1] += v.y;
-        acc[2] += v.z;
-        acc[3] += v.w;
-    }
-    const int64_t o = (int64_t)t * H + m;
-    if (a.out_bf16) {
-        if (a.residual) {
-            const uint2 r = *reinterpret_cast<const uint2*>(
-                reinterpret_cast<const __nv_bfloat16*>(a.residual) + o);
-            acc[0] += __uint_as_float(r.x << 16);
-            acc[1] += __uint_as_float(r.x & 0xFFFF0000u);
-            acc[2] += __uint_as_float(r.y << 16);
-            acc[3] += __uint_as_float(r.y & 0xFFFF0000u);
+        for (int sh = 0; sh < a.n_shared; ++sh) {
+            const float4 v =
+                __ldg(reinterpret_cast<const float4*>(a.y + (int64_t)(P + sh * a.T + t) * H + m));
+            acc[0] += v.x;
+            acc[1] += v.y;
+            acc[2] += v.z;
+            acc[3] += v.w;
         }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
-        uint2 w2;
-        w2.x = *reinterpret_cast<const uint32_t*>(&lo);
-        w2.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o) = w2;
-    } else {
-        if (a.residual) {
-            const float4 r = *reinterpret_cast<const float4*>(
-                reinterpret_cast<const float*>(a.residual) + o);
-            acc[0] += r.x;
-            acc[1] += r.y;
-            acc[2] += r.z;
-            acc[3] += r.w;
+        const int64_t o = (int64_t)t * H + m;
+        if (a.out_bf16) {
+            if (a.residual) {
+                const uint2 r = *reinterpret_cast<const uint2*>(
+                    reinterpret_cast<const __nv_bfloat16*>(a.residual) + o);
+                acc[0] += __uint_as_float(r.x << 16);
+                acc[1] += __uint_as_float(r.x & 0xFFFF0000u);
+                acc[2] += __uint_as_float(r.y << 16);
+                acc[3] += __uint_as_float(r.y & 0xFFFF0000u);
+            }
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+            uint2 w2;
+            w2.x = *reinterpret_cast<const uint32_t*>(&lo);
+            w2.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o) = w2;
+        } else {
+            if (a.residual) {
+                const float4 r = *reinterpret_cast<const float4*>(
+                    reinterpret_cast<const float*>(a.residual) + o);
+                acc[0] += r.x;
+                acc[1] += r.y;
+                acc[2] += r.z;
+                acc[3] += r.w;
+            }
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) =
+                make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) =
-            make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
 }
 
@@ -672,11 +673,11 @@ cudaError_t launch_stream(const FfnArgs& a, const Geo& g, int num_sms, cudaStrea
 cudaError_t launch_combine_impl(const FfnArgs& a, int num_sms, cudaStream_t st) {
     const size_t oa = a.out_bf16 ? 8 : 16;
     auto al = [](const void* p, size_t n) { return reinterpret_cast<uintptr_t>(p) % n == 0; };
-    if (a.H % 4 == 0 && a.T >= 1 && a.T <= 65535 && al(a.y, 16) && al(a.out, oa) &&
+    if (a.H % 4 == 0 && a.T >= 1 && al(a.y, 16) && al(a.out, oa) &&
         (!a.residual || al(a.residual, oa))) {
         cudaLaunchAttribute attr[1];
         cudaLaunchConfig_t cfg = pdl_config(1, 256, 0, st, attr);
-        cfg.gridDim = dim3((unsigned)((a.H / 4 + 255) / 256), (unsigned)a.T);
+        cfg.gridDim = dim3((unsigned)((a.H / 4 + 255) / 256), (unsigned)std::min(a.T, 65535));
         return cudaLaunchKernelEx(&cfg, combine_vec_kernel, a);
     }
     const int64_t n = (int64_t)a.T * a.H;
