@@ -420,14 +420,16 @@ def run_stack(args, rank, world, local):
                          "streams far more than L2 per step",
                    "parallelism": f"replicas x{world}"},
         "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": achieved,
+        "roofline": {"bound": "hbm",
+                     "kernel": "gateup_kernel" if T * k < E else "prefill_gemm_kernel<gate/up>",
+                     "achieved": achieved,
                      "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
                      "peak_source": P["src"], "traffic": None,
                      "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
         "cpu_baseline": None,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
-        "gpu_launches": 4 * L * args.steps,
+        "gpu_launches": (4 if T * k < E else 6) * L * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -551,9 +553,11 @@ def run_ours(args, rank, world, local):
     step_bytes = (n_uniq + n_sh) * expert_bytes(H, I)
     # dominant kernel: up to 8 tokens the fused decode kernel (routing, gate/up,
     # down and combine; it streams every active expert whole), otherwise the
-    # gate/up kernel of the streaming or tensor-core path
-    fused = T <= 8
-    tensor = kind == "uniform"  # prefill: the tensor-core grouped GEMM
+    # gate/up kernel of the streaming or tensor-core path (the library's
+    # default takes the tensor-core grouped GEMM once T*k >= E)
+    fused = T <= 8 and T * k < E
+    stream = not fused and T * k < E
+    tensor = kind == "uniform"  # prefill: tensor-bound
     k_ms = phase_ms[1] / max(n_calls, 1)
     if tensor:
         # gate/up GEMM: 2/3 of the pair FLOPs over all (token, expert) pairs + shared
@@ -566,7 +570,9 @@ def run_ours(args, rank, world, local):
     else:
         k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
         achieved = k_bytes / (k_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": "decode_fused_kernel" if fused else "gateup_kernel",
+        roof = {"bound": "hbm",
+                "kernel": "decode_fused_kernel" if fused else "gateup_kernel" if stream
+                else "prefill_gemm_kernel<gate/up>",
                 "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
                 "frac": achieved / P["hbm"], "peak_source": P["src"],
                 "traffic": FUSED_DECODE_DRAM_BYTES.get(T) if fused else None,
@@ -588,7 +594,7 @@ def run_ours(args, rank, world, local):
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 4},
-        "gpu_launches": (1 if fused else 4 if T <= 64 else 6) * args.steps,
+        "gpu_launches": (1 if fused else 4 if stream and T <= 64 else 6) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -104,7 +104,8 @@ typedef struct {
     int32_t n_shared;           /* shared experts, 0..4 */
     const coli_expert *experts; /* host array, n_routed + n_shared entries */
     int32_t prefill_min_tokens; /* T*k/E at or above which the tensor-core
-                                   grouped GEMM is used; 0 = library default */
+                                   grouped GEMM is used; 0 = library default
+                                   (1: every call with T*k >= E) */
 } coli_moe_desc;
 
 typedef struct coli_moe coli_moe; /* opaque: device copy of the expert table */

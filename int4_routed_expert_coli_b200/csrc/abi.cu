@@ -13,8 +13,12 @@
 #include "prefill.cuh"
 
 // Average routed tokens per expert (T*k/E) at or above which a call runs the
-// tensor-core grouped GEMM instead of the streaming dequant-GEMV.
-constexpr int kDefaultPrefillMin = 32;
+// tensor-core grouped GEMM instead of the streaming dequant-GEMV (calls of up
+// to 8 tokens below it take the fused decode kernel).  Measured on the
+// GLM-5.2 shape with Zipf routing: at T = 32 (T*k/E = 1) the grouped GEMM
+// takes 1.10 ms against the streaming path's 1.51 ms, at T = 64 1.54 ms
+// against 2.32 ms.
+constexpr int kDefaultPrefillMin = 1;
 
 namespace {
 

@@ -559,8 +559,13 @@ __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
             if (slot < g.n_shared) {
                 ntok = g.T;
             } else if (slot < n_slots) {
+                // an expert id or token list the union could not have produced
+                // is reported; its slot gets no tiles
                 const int e = g.active[slot - g.n_shared];
-                if (e >= 0 && e < g.E) ntok = g.offsets[e + 1] - g.offsets[e];
+                const int b = (e >= 0 && e < g.E) ? g.offsets[e] : 0;
+                const int en = (e >= 0 && e < g.E) ? g.offsets[e + 1] : -1;
+                if (e >= 0 && e < g.E && b >= 0 && en >= b && en <= P) ntok = en - b;
+                else report(g.status, COLI_ERR_BAD_INDEX);
             }
             cnt[u] = slot < n_slots ? (max(ntok, 0) + BN - 1) / BN : 0;
         }

@@ -85,12 +85,14 @@ def test_tiny_layer_f32_residual_many_tokens(tiny):
     assert_close(out.cpu().numpy(), ref, "tiny T=203")
 
 
-def test_ragged_dims_two_shared():
-    """H, I multiples of 128 but not of 256; 12 experts top-3; 2 shared."""
+@pytest.mark.parametrize("prefill_min", [0, 10 ** 6])  # default path / streaming forced
+def test_ragged_dims_two_shared(prefill_min):
+    """H, I multiples of 128 but not of 256; 12 experts top-3; 2 shared;
+    both the default (tensor-core) path and the streaming dequant-GEMV."""
     from int4_routed_expert_coli_b200 import coli_moe as c
     H, I, E, k, T = 384, 384, 12, 3, 19
     bank = synth.make_expert_bank(H, I, E + 2, seed=8, device="cuda")
-    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=2)
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=2, prefill_min_tokens=prefill_min)
     x = synth.make_activations(T, H, seed=9, device="cuda")
     lg = synth.make_logits_normal(T, E, seed=9, device="cuda")
     out, idx, w, _ = _layer(layer, x, logits=lg)
@@ -113,10 +115,15 @@ def test_glm_decode_steps(glm):
         assert_close(out.cpu().numpy(), ref, f"decode step {s}")
 
 
-@pytest.mark.parametrize("T,n_sample", [(4, 4), (32, 8)])
-def test_glm_small_batch_zipf(glm, T, n_sample):
-    """Speculative-verify / small batch: Zipf-1.1 routing, 71.6 % repeats."""
+@pytest.mark.parametrize("T,n_sample,stream", [(4, 4, False), (32, 8, False), (32, 8, True)])
+def test_glm_small_batch_zipf(glm, T, n_sample, stream):
+    """Speculative-verify / small batch: Zipf-1.1 routing, 71.6 % repeats
+    (T = 32 on the default tensor-core path and on the streaming path)."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
     bank, layer = glm
+    if stream:
+        layer = c.MoELayer(bank, n_routed=GLM["E"], top_k=GLM["k"], n_shared=1,
+                           prefill_min_tokens=10 ** 6)
     _, logits = synth.zipf_routing(T, 256, 8, steps=2, seed=T)
     for s, lg_np in enumerate(logits):
         x = synth.make_activations(T, 6144, seed=3000 + s, device="cuda")
