@@ -32,7 +32,8 @@
 // group) offset sum as the initial accumulator for gate/up, exact unpack for
 // down, m16n8k16 MMA with fp32 accumulation, gs64 scale applied to each
 // group's partial.  Eleven consumer warps split K; a gate/up item's partials
-// are summed by one rotating warp through four reduction buffers.
+// are summed through four reduction buffers, item j by warp j mod 11 two
+// items later (in warp order, so the sum does not depend on timing).
 //
 // Every wait is bounded (COLI_ERR_TIMEOUT).  The counters are zero on entry;
 // the last CTA to finish puts them back to zero.

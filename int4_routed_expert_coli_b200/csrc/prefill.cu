@@ -243,7 +243,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
     constexpr int kStage = kBBytes + NA * kPkBytes;
     constexpr int kACols = NA * BK / 2;                      // operand columns per K-block
-    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 2 gate/up, 4 down
+    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 2
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -251,9 +251,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // TMA landed
     uint64_t* dq_full = full + 16;                             // operand written to TMEM
     uint64_t* empty = full + 32;                               // MMAs done reading the stage
-    uint64_t* acc_full = full + 48;                            // [2] accumulator ready
-    uint64_t* acc_empty = full + 50;                           // [2] accumulator drained
-    uint64_t* a_empty = full + 52;                             // [8] MMAs done with an operand
+    uint64_t* acc_full = full + 48;                            // accumulator ready
+    uint64_t* acc_empty = full + 50;                           // accumulator drained
+    uint64_t* a_empty = full + 52;                             // [kAStages] MMAs done with an operand
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 512);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
     uint8_t* stage0 = smem + kHeaderP;
@@ -268,10 +268,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             mbar_init(&dq_full[s], 4);
             mbar_init(&a_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kEpiWarps);
-        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -361,15 +359,15 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
                 const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-                const int buf = 0;  // one accumulator (NA x BN = 384 columns)
-                const uint32_t ause = (uint32_t)lt;
-                if (ause > 0 && !mbar_wait(&acc_empty[buf], (ause - 1) & 1)) {
+                // one accumulator (NA x BN = 384 columns): tile lt waits for the
+                // epilogue of tile lt - 1
+                if (lt > 0 && !mbar_wait(acc_empty, (uint32_t)(lt - 1) & 1)) {
                     timeout();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t idesc = idesc_f16(ti.n_mma);
-                const uint32_t d0 = tmem_base + (uint32_t)(buf * NA * BN);
+                const uint32_t d0 = tmem_base;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     const int s = rs.i, as = ra.i;
@@ -390,7 +388,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     mma_commit(&a_empty[as]);
                 }
                 if (!ok) break;
-                mma_commit(&acc_full[buf]);
+                mma_commit(acc_full);
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -475,13 +473,12 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
             const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-            const int buf = 0;
-            if (!mbar_wait(&acc_full[buf], (uint32_t)lt & 1)) {
+            if (!mbar_wait(acc_full, (uint32_t)lt & 1)) {
                 if (lane == 0) timeout();
                 break;
             }
             tc_fence_after();
-            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BN);
+            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16);
             const int feat = ti.m_tile * kFeat + row;
             if constexpr (kGU) {
                 // gate and up of this lane's feature sit in the same lane; the
@@ -524,7 +521,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (lane == 0) mbar_arrive(acc_empty);
         }
     }
 
