@@ -156,24 +156,32 @@ class ClockSampler:
 
 
 def dist_setup(args):
+    """One process per GPU under torchrun (NCCL); without a GPU (the CPU-only
+    reference arm, or tests of this plumbing) the ranks use gloo."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=300)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time: every rank calls this with its own value."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
