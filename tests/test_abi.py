@@ -78,6 +78,8 @@ def test_host_validation_without_gpu():
     assert L.coli_moe_create(ctypes.byref(d), ctypes.byref(h)) == c.COLI_ERR_SHAPE
     d = c.CDesc(256, 128, 1, 2, 64, 1, tab, 0)       # k > E
     assert L.coli_moe_create(ctypes.byref(d), ctypes.byref(h)) == c.COLI_ERR_SHAPE
+    d = c.CDesc(256, 128, 1, 1, 64, 1, tab, -1)      # negative tensor-core threshold
+    assert L.coli_moe_create(ctypes.byref(d), ctypes.byref(h)) == c.COLI_ERR_INVALID_ARG
     d = c.CDesc(256, 128, 1, 1, 64, 1, tab, 0)       # NULL expert pointers
     assert L.coli_moe_create(ctypes.byref(d), ctypes.byref(h)) == c.COLI_ERR_INVALID_ARG
     for f in ("gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s"):
