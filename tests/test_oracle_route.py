@@ -120,3 +120,73 @@ def test_router_logits_match_numpy():
     got = oracle.router_logits(xb, wr)
     ref = bf16_bits_to_f64(xb) @ wr.astype(np.float64).T
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+# ---- router logits: closed forms ------------------------------------------
+# The router scores every routed expert for each token, logits[t][e] =
+# sum_h x[t][h] W_r[e][h] ("zhichai.net/topic/178503686", MoE-sparsity
+# section).  Shapes below are non-square, so a transposed or mis-strided read
+# of W_r or x cannot reproduce the expected values.
+
+BF16_ONE = 0x3F80
+
+
+def test_router_logits_golden_worked_example():
+    xs, ws, ls = [], [], []
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "router_logits.txt")):
+        f = line.split("#")[0].split("[")[0].split()
+        if not f:
+            continue
+        if f[0] == "x":
+            xs.append([int(v, 16) for v in f[1:]])
+        elif f[0] == "w":
+            ws.append([float(v) for v in f[1:]])
+        elif f[0] == "l":
+            ls.append([float(v) for v in f[1:]])
+    got = oracle.router_logits(np.array(xs, np.uint16), np.array(ws, np.float32))
+    assert got.shape == (2, 4)
+    assert np.array_equal(got, np.array(ls))
+
+
+def test_router_logits_one_hot_tokens_pick_router_columns():
+    """x[t] = one-hot at h_t (bf16 1.0): logits[t][e] = W_r[e][h_t] exactly."""
+    T, H, E = 3, 7, 5
+    hot = [2, 6, 0]
+    x = np.zeros((T, H), np.uint16)
+    for t, h in enumerate(hot):
+        x[t, h] = BF16_ONE
+    # distinct dyadic entries (exact in fp32): 1/8 steps per expert, 1/64 per column
+    wr = np.array([[(e + 1) / 8 + h / 64 for h in range(H)] for e in range(E)], np.float32)
+    got = oracle.router_logits(x, wr)
+    for t, h in enumerate(hot):
+        for e in range(E):
+            assert got[t, e] == (e + 1) / 8 + h / 64
+
+
+def test_router_logits_one_hot_router_rows_pick_token_elements():
+    """W_r[e] = 1/8 at column c_e, 0 elsewhere: logits[t][e] = x[t][c_e] / 8."""
+    T, H, E = 2, 6, 4
+    cols = [5, 0, 3, 3]
+    vals = [[0x4000, 0xBF80, 0x3F00, 0x4080, 0x0000, 0xC040],   # 2 -1 0.5 4 0 -3
+            [0x3E80, 0x4120, 0xC100, 0x3F80, 0x8000, 0x3FC0]]   # .25 10 -8 1 -0 1.5
+    decoded = [[2, -1, 0.5, 4, 0, -3], [0.25, 10, -8, 1, 0, 1.5]]
+    wr = np.zeros((E, H), np.float32)
+    for e, c in enumerate(cols):
+        wr[e, c] = 0.125
+    got = oracle.router_logits(np.array(vals, np.uint16), wr)
+    for t in range(T):
+        for e, c in enumerate(cols):
+            assert got[t, e] == decoded[t][c] / 8
+
+
+def test_router_logits_constant_token_signed_rows():
+    """x = 0.5 everywhere (H = 8); row e of W_r holds e + 1 entries +2^-6 and
+    the rest -2^-6, so logits[t][e] = 0.5 * 2^-6 * (2(e + 1) - 8)."""
+    H, E = 8, 4
+    x = np.full((2, H), 0x3F00, np.uint16)
+    wr = np.full((E, H), -2.0 ** -6, np.float32)
+    for e in range(E):
+        wr[e, : e + 1] = 2.0 ** -6
+    got = oracle.router_logits(x, wr)
+    expect = [-0.046875, -0.03125, -0.015625, 0.0]
+    assert np.array_equal(got, np.array([expect, expect]))
