@@ -17,6 +17,11 @@ Multi-GPU (torchrun): every rank runs its own replica on its own token
 stream (no data-path collective); the timed total is the max over ranks and
 `value` counts the tokens of all ranks ("scaling": "weak").
 
+Without --workload the run measures every workload: the decode line is the
+headline and the others (verify4, batch32, prefill, stack) are attached to it
+under "workloads", each with its own roofline, CPU baseline, end-to-end
+figure and clock record.  --workload NAME measures that one alone.
+
 Prints one JSON line on rank 0.
 """
 from __future__ import annotations
@@ -57,11 +62,14 @@ WORKLOADS = {
 STACK_LAYERS = 16
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) of one fused decode launch, from the ncu capture
-# summarised in profiles/decode_fused_kernel_glm_t1.md (tokens per step ->
-# bytes); a workload without a capture of the current kernel reports null.
-FUSED_DECODE_DRAM_BYTES = {1: 180_612_608 + 3_990_272}
 PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
+# DRAM bytes (read + write) per launch of a workload's dominant kernel, taken
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).  Each
+# entry names the kernel source file and its SHA-256 at capture time; when
+# the file has changed since, the bench reports traffic as null.  Entries:
+# workload -> (source file, sha256, bytes per launch, how the figure was
+# obtained).
+DRAM_TRAFFIC = {}
 
 
 def expert_bytes(H, I):
@@ -70,6 +78,23 @@ def expert_bytes(H, I):
 
 def gateup_bytes(H, I):
     return 2 * (H * I // 2) + 2 * (H * I // 64) * 2
+
+
+def _sha256(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def traffic_for(workload):
+    """(bytes per launch or None, source note) for the workload's dominant kernel."""
+    ent = DRAM_TRAFFIC.get(workload)
+    if ent is None:
+        return None, "no ncu capture of the current kernel for this workload"
+    src, sha, nbytes, how = ent
+    if _sha256(os.path.join(ROOT, src)) != sha:
+        return None, f"stale: {src} changed since the ncu capture"
+    return nbytes, how
 
 
 def peaks():
@@ -316,10 +341,31 @@ def stack_inputs(n, seed, device):
     return xs, lgs
 
 
-def run_stack(args, rank, world, local):
+def oracle_stack_sample(banks, x0, lgs_step, n_threads, tok=2):
+    """The oracle on `tok` tokens of one stack step through every layer (each
+    layer's bf16 output feeds the next, as on the GPU); returns the seconds
+    spent in the oracle and the tokens."""
+    import oracle
+    E, k, n_sh = GLM["E"], GLM["k"], GLM["n_shared"]
+    H, I = GLM["H"], GLM["I"]
+    x = x0[:tok].cpu()
+    sec = 0.0
+    for l, bank in enumerate(banks):
+        idx, w = oracle.route(lgs_step[l][:tok].float().cpu().numpy(), k)
+        needed = set(idx.ravel().tolist()) | set(range(E, E + n_sh))
+        ex = oracle.Experts([bank.expert_numpy(e) if e in needed else None for e in range(bank.n)])
+        xb = x.view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        y = oracle.layer(H, I, E, k, n_sh, ex, xb, idx, w, n_threads=n_threads)
+        sec += time.perf_counter() - t0
+        x = (x.double() + torch.from_numpy(np.asarray(y))).to(torch.bfloat16)
+    return sec, tok
+
+
+def run_stack(args, rank, world, local, with_cpu=True):
     """Config 5: 16 independent layers, each step runs them in sequence on
     one token batch, x_(l+1) = x_l + MoE_l(x_l) (bf16 stream, residual added
-    in fp32 by the combine)."""
+    in fp32 by the combine).  Returns the JSON line (rank 0) or None."""
     from int4_routed_expert_coli_b200 import coli_moe as c
     T, _, desc = WORKLOADS["stack"]
     H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
@@ -404,8 +450,20 @@ def run_stack(args, rank, world, local):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world)
 
+    cpu = None
+    if rank == 0 and world == 1 and with_cpu and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        sec, toks = oracle_stack_sample(banks, xs[args.warmup],
+                                        [lgs[l][args.warmup] for l in range(L)], cores)
+        cpu = {"value": toks / sec, "unit": "tokens/s", "cores": min(cores, toks * (k + n_sh)),
+               "kind": "oracle",
+               "sample": f"{toks} tokens of one step through all {L} layers (each layer's "
+                         f"output feeds the next), every routed + shared expert, double "
+                         f"precision, {sec:.1f} s"}
+    del layers, banks
+    torch.cuda.empty_cache()
     if rank != 0:
-        return
+        return None
     P = peaks()
     tokens = T * args.steps * world
     value = tokens / (total_ms / 1e3)
@@ -414,6 +472,7 @@ def run_stack(args, rank, world, local):
     k_bytes = statistics.mean(statistics.mean(us) for us in uniq) * gateup_bytes(H, I) + \
         n_sh * gateup_bytes(H, I)
     achieved = k_bytes / (k_ms / 1e3) / 1e9
+    traffic, traffic_src = traffic_for("stack")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -432,20 +491,23 @@ def run_stack(args, rank, world, local):
                      "kernel": "gateup_kernel" if T * k < E else "prefill_gemm_kernel<gate/up>",
                      "achieved": achieved,
                      "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
-                     "peak_source": P["src"], "traffic": None,
+                     "peak_source": P["src"], "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
-        "cpu_baseline": None,
+        "phase_ms_per_layer_call": {"before": phase_ms[0] / max(n_calls, 1), "main": k_ms,
+                                    "after": phase_ms[2] / max(n_calls, 1)},
+        "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
         "gpu_launches": (4 if T * k < E else 6) * L * args.steps,
         "clocks": clocks,
     }
-    print(json.dumps(line), flush=True)
+    return line
 
 
-def run_ours(args, rank, world, local):
+def run_ours(args, rank, world, local, name, with_cpu=True):
+    """One workload through coli_moe_layer; returns the JSON line (rank 0) or
+    None."""
     from int4_routed_expert_coli_b200 import coli_moe as c
-    name = args.workload
     T, kind, desc = WORKLOADS[name]
     H, I, E, k, n_sh = GLM["H"], GLM["I"], GLM["E"], GLM["k"], GLM["n_shared"]
     if E != 256:  # a smaller resident bank (profiling runs) says so in the label
@@ -539,7 +601,7 @@ def run_ours(args, rank, world, local):
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) --------
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and with_cpu and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
         tok = min(T, 8)
         # about 600 (token, expert) evaluations: ~10 s on 16 host cores
@@ -552,8 +614,10 @@ def run_ours(args, rank, world, local):
                "sample": f"{n_s} steps x {tok} token(s), every routed + shared expert of each "
                          f"token, double precision, {sec:.1f} s"}
 
+    del layer, bank
+    torch.cuda.empty_cache()
     if rank != 0:
-        return
+        return None
     P = peaks()
     tokens = T * args.steps * world
     value = tokens / (total_ms / 1e3)
@@ -567,6 +631,7 @@ def run_ours(args, rank, world, local):
     stream = not fused and T * k < E
     tensor = kind == "uniform"  # prefill: tensor-bound
     k_ms = phase_ms[1] / max(n_calls, 1)
+    traffic, traffic_src = traffic_for(name)
     if tensor:
         # gate/up GEMM: 2/3 of the pair FLOPs over all (token, expert) pairs + shared
         k_work = (T * k + T * n_sh) * PAIR_FLOP * 2 / 3
@@ -574,7 +639,8 @@ def run_ours(args, rank, world, local):
         roof = {"bound": "tensor", "kernel": "prefill_gemm_kernel<gate/up>",
                 "achieved": achieved, "peak": P["bf16"], "unit": "TFLOP/s",
                 "frac": achieved / P["bf16"], "peak_source": P["src"] + " (bf16 burst; fp16 taken equal)",
-                "traffic": None, "algorithmic_flop_per_launch": k_work, "avg_launch_ms": k_ms}
+                "traffic": traffic, "traffic_source": traffic_src,
+                "algorithmic_flop_per_launch": k_work, "avg_launch_ms": k_ms}
     else:
         k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
         achieved = k_bytes / (k_ms / 1e3) / 1e9
@@ -583,7 +649,7 @@ def run_ours(args, rank, world, local):
                 else "prefill_gemm_kernel<gate/up>",
                 "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
                 "frac": achieved / P["hbm"], "peak_source": P["src"],
-                "traffic": FUSED_DECODE_DRAM_BYTES.get(T) if fused else None,
+                "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -605,7 +671,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": (1 if fused else 4 if stream and T <= 64 else 6) * args.steps,
         "clocks": clocks,
     }
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -614,7 +680,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="measure one workload alone (default: decode as the headline line, "
+                         "the others attached under \"workloads\")")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's tokens per step (small profiler cases)")
@@ -626,16 +694,36 @@ def main():
         ap.error("--warmup must be at least 3")
     GLM["E"] = args.routed_experts
     if args.tokens > 0:
-        T0, kind, desc = WORKLOADS[args.workload]
-        WORKLOADS[args.workload] = (args.tokens, kind, desc.replace(f"T={T0}", f"T={args.tokens}"))
+        name = args.workload or "decode"
+        T0, kind, desc = WORKLOADS[name]
+        WORKLOADS[name] = (args.tokens, kind, desc.replace(f"T={T0}", f"T={args.tokens}"))
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
+            if args.workload is None:
+                args.workload = "decode"
             run_reference(args, rank, world)
-        elif args.workload == "stack":
-            run_stack(args, rank, world, local)
-        else:
-            run_ours(args, rank, world, local)
+            return
+
+        def one(name):
+            if name == "stack":
+                return run_stack(args, rank, world, local)
+            return run_ours(args, rank, world, local, name)
+
+        line = one(args.workload or "decode")
+        if args.workload is None:
+            extra = {}
+            for name in ("verify4", "batch32", "prefill", "stack"):
+                sub = one(name)
+                if sub is not None:
+                    for key in ("metric", "n_gpus", "steps", "warmup", "higher_is_better",
+                                "scaling", "vs_baseline", "data"):
+                        sub.pop(key, None)
+                    extra[name] = sub
+            if line is not None:
+                line["workloads"] = extra
+        if line is not None:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -200,13 +200,17 @@ coli_status coli_moe_layer(const coli_moe *h, int32_t T, const void *x_bf16, con
  *              before anything is launched
  *   x_bf16, logits, residual, out, out_dtype: as coli_moe_layer
  *   status_out nullable device int32: receives the call's device status word
- *              (as coli_moe_get_status would read it) at the end of the call
+ *              (as coli_moe_get_status would read it) at the end of the call;
+ *              written only when the call returns COLI_OK with T > 0 (a call
+ *              that returns an error, or T == 0, leaves it untouched)
  * The scratch is one fixed __device__ array per GPU that loads the library,
  * held until exit.  The first call on a device (with that device current)
- * looks up the array's device address; make that first call before any stream
- * capture.  Every call shares the array and clears its status word itself;
- * calls whose work overlaps on the GPU race on it, so order them on one
- * stream.  Other errors as coli_moe_create and coli_moe_layer. */
+ * looks up the array's device address.  Every call also copies the expert
+ * pointer table from pageable host memory into the array, so no call of this
+ * entry point may be made under stream capture.  Every call shares the array
+ * and clears its status word itself; calls whose work overlaps on the GPU
+ * race on it, so order them on one stream.  Other errors as coli_moe_create
+ * and coli_moe_layer. */
 coli_status coli_moe_layer_noalloc(const coli_moe_desc *desc, int32_t T, const void *x_bf16,
                                    const float *logits, const void *residual, void *out,
                                    coli_out_dtype out_dtype, int32_t *status_out, void *stream);
@@ -231,9 +235,16 @@ coli_status coli_moe_profile_read(double *ms, int32_t *n_calls);
  * gate/up kernel never fills one staged tile: its consumers' bounded wait
  * (about one second) runs out, the kernel winds down without hanging or
  * faulting, and the status word reads COLI_ERR_TIMEOUT; the output of that
- * call is undefined and the context stays usable.  0 switches it off.
+ * call is undefined and the context stays usable.  0 switches every hook
+ * off.
  * Returns COLI_ERR_INVALID_ARG for an unknown code. */
 #define COLI_INJECT_WITHHOLD_STAGE 1
+/* With COLI_INJECT_NOT_RESIDENT the next call that would run the fused
+ * decode kernel (up to 8 tokens) behaves as if its cooperative launch had
+ * been refused because the grid cannot be resident at once (a GPU with fewer
+ * usable SMs than the handle saw): nothing is launched for it and the call
+ * runs on the streaming kernels instead, with the same result. */
+#define COLI_INJECT_NOT_RESIDENT 2
 coli_status coli_moe_debug_inject(int32_t what);
 
 /* Static English text for a status code (never NULL). */

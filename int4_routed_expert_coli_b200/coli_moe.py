@@ -180,6 +180,7 @@ def coli_moe_get_status(ws, stream=None):
 
 
 COLI_INJECT_WITHHOLD_STAGE = 1
+COLI_INJECT_NOT_RESIDENT = 2
 
 
 def coli_moe_debug_inject(what: int):

@@ -146,7 +146,8 @@ cudaError_t run_fused(const coli_moe* h, const coli::FfnArgs& a, const float* lo
 
 // The FFN of a call whose union lists (and inverse map) are ready: tensor-core
 // grouped GEMM for prefill-sized batches, the fused decode kernel for up to
-// 8 tokens, streaming GEMV otherwise.
+// 8 tokens, streaming GEMV otherwise (also when the fused kernel's grid
+// cannot be resident at once).
 // `x_prepared`: the fused prep kernel already built the GEMV operand of x.
 cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* ws,
                     cudaStream_t st, bool x_prepared) {
@@ -159,7 +160,11 @@ cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* 
         coli::profile_mark(4, st);
         return err;
     }
-    if (use_fused(h, T)) return run_fused(h, a, nullptr, nullptr, nullptr, ws, st);
+    if (!x_prepared && use_fused(h, T)) {
+        err = run_fused(h, a, nullptr, nullptr, nullptr, ws, st);
+        if (err != cudaErrorCooperativeLaunchTooLarge) return err;
+        err = cudaSuccess;  // not launched: stream instead
+    }
     if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
     if (err != cudaSuccess) return err;
     return coli::launch_ffn_stream(a, h->num_sms, st);
@@ -185,10 +190,15 @@ extern "C" {
 coli_status coli_moe_debug_inject(int32_t what) {
     if (what == 0) {
         g_withhold_item = -1;
+        coli::decode_force_not_resident(false);
         return COLI_OK;
     }
     if (what == COLI_INJECT_WITHHOLD_STAGE) {
         g_withhold_item = 0;  // the first item of CTA 0: a shared-expert gate/up tile
+        return COLI_OK;
+    }
+    if (what == COLI_INJECT_NOT_RESIDENT) {
+        coli::decode_force_not_resident(true);
         return COLI_OK;
     }
     return COLI_ERR_INVALID_ARG;
@@ -282,8 +292,10 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
     if (err == cudaSuccess && coli::prefill_available())
         err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
+    // the fused decode kernel only where one CTA per SM can be resident at once
     if (err == cudaSuccess && h->d_wmaps &&
         coli::decode_supported(h->H, h->I, 1, h->E, h->k, h->n_shared, h->num_sms) &&
+        coli::decode_coresident(h->H, h->I, h->E, h->k, h->n_shared, h->num_sms) &&
         coli::build_decode_maps(host, n, h->H, h->I, &h->d_dmaps) != cudaSuccess) {
         h->d_dmaps = nullptr;  // the fused decode path is an optimisation: go without it
         cudaGetLastError();
@@ -402,8 +414,11 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
     if (err == cudaSuccess && use_fused(h, T)) {
         // one launch: every CTA routes the tokens itself
         err = run_fused(h, a, lg, topk_idx_out, topk_w_out, ws, st);
-        profile_end_call();
-        return from_cuda(err);
+        if (err != cudaErrorCooperativeLaunchTooLarge) {
+            profile_end_call();
+            return from_cuda(err);
+        }
+        err = cudaSuccess;  // the grid cannot be resident at once: the streaming path below
     }
     if (T <= coli::kSmallT && !prefill) {
         // one launch: route, union, inverse map and activation preparation

@@ -1123,6 +1123,13 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     }
 }
 
+// False once the runtime refused the cooperative launch together with
+// programmatic dependent launch; later launches are cooperative only.
+bool g_coop_with_pdl = true;
+
+// A cooperative launch: the runtime starts it only if every CTA of the grid
+// can be resident at once (cudaErrorCooperativeLaunchTooLarge otherwise),
+// which the CTAs' waits on one another need.
 template <int NV>
 cudaError_t launch_nv(const DecodeArgs& d, int blocks, int smem, cudaStream_t st) {
     cudaError_t err = cudaFuncSetAttribute(decode_fused_kernel<NV>,
@@ -1133,17 +1140,47 @@ cudaError_t launch_nv(const DecodeArgs& d, int blocks, int smem, cudaStream_t st
     cfg.blockDim = dim3(kThreadsD);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+    cfg.numAttrs = g_coop_with_pdl ? 2 : 1;
+    err = cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+    if (err != cudaSuccess && err != cudaErrorCooperativeLaunchTooLarge && g_coop_with_pdl) {
+        cudaGetLastError();  // a refused configuration launched nothing
+        g_coop_with_pdl = false;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+    }
+    return err;
+}
+
+// Resident CTAs of the kernel instance per SM at `smem` bytes of shared memory.
+template <int NV>
+int resident_per_sm(int smem) {
+    if (cudaFuncSetAttribute(decode_fused_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+        return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_fused_kernel<NV>, kThreadsD,
+                                                      smem) != cudaSuccess)
+        return 0;
+    return n;
 }
 
 int max_slots_for(int E, int k, int T, int n_shared) {
     return std::min(E, T * k) + n_shared;
 }
+
+// Template instance for E routed experts (logits per routing lane).
+int nv_for(int E) {
+    const int nv = (E + 31) / 32;
+    return nv <= 1 ? 1 : nv <= 2 ? 2 : nv <= 4 ? 4 : nv <= 8 ? 8 : nv <= 16 ? 16 : 32;
+}
+
+bool g_force_not_resident = false;  // test hook (coli_moe_debug_inject)
 
 }  // namespace
 
@@ -1194,21 +1231,49 @@ cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I
     return err;
 }
 
+bool decode_coresident(int H, int I, int E, int k, int n_shared, int num_sms) {
+    // the largest shared-memory footprint (8 tokens) of either template
+    // instance a handle can launch (routing from logits, or a given union)
+    const Layout L = make_layout(H, I, max_slots_for(E, k, 8, n_shared));
+    int per_sm = resident_per_sm<1>(L.smem);
+    switch (nv_for(E)) {
+        case 1: per_sm = std::min(per_sm, resident_per_sm<1>(L.smem)); break;
+        case 2: per_sm = std::min(per_sm, resident_per_sm<2>(L.smem)); break;
+        case 4: per_sm = std::min(per_sm, resident_per_sm<4>(L.smem)); break;
+        case 8: per_sm = std::min(per_sm, resident_per_sm<8>(L.smem)); break;
+        case 16: per_sm = std::min(per_sm, resident_per_sm<16>(L.smem)); break;
+        default: per_sm = std::min(per_sm, resident_per_sm<32>(L.smem)); break;
+    }
+    cudaGetLastError();
+    return per_sm >= 1 && num_sms >= 1;
+}
+
+void decode_force_not_resident(bool on) { g_force_not_resident = on; }
+
 cudaError_t launch_decode_fused(const DecodeArgs& d0, int num_sms, cudaStream_t st) {
     DecodeArgs d = d0;
-    d.f.withhold_item = take_withhold_item();
+    if (g_force_not_resident) {  // test hook: behave as if the launch were refused
+        g_force_not_resident = false;
+        return cudaErrorCooperativeLaunchTooLarge;
+    }
     d.max_slots = max_slots_for(d.f.E, d.f.k, d.f.T, d.f.n_shared);
     const Layout L = make_layout(d.f.H, d.f.I, d.max_slots);
     const int blocks = num_sms;  // persistent: one CTA per SM, all resident
+    d.f.withhold_item = take_withhold_item();
     profile_mark(1, st);
     cudaError_t err;
-    const int nv = d.logits ? (d.f.E + 31) / 32 : 1;
-    if (nv <= 1) err = launch_nv<1>(d, blocks, L.smem, st);
-    else if (nv <= 2) err = launch_nv<2>(d, blocks, L.smem, st);
-    else if (nv <= 4) err = launch_nv<4>(d, blocks, L.smem, st);
-    else if (nv <= 8) err = launch_nv<8>(d, blocks, L.smem, st);
-    else if (nv <= 16) err = launch_nv<16>(d, blocks, L.smem, st);
-    else err = launch_nv<32>(d, blocks, L.smem, st);
+    switch (d.logits ? nv_for(d.f.E) : 1) {
+        case 1: err = launch_nv<1>(d, blocks, L.smem, st); break;
+        case 2: err = launch_nv<2>(d, blocks, L.smem, st); break;
+        case 4: err = launch_nv<4>(d, blocks, L.smem, st); break;
+        case 8: err = launch_nv<8>(d, blocks, L.smem, st); break;
+        case 16: err = launch_nv<16>(d, blocks, L.smem, st); break;
+        default: err = launch_nv<32>(d, blocks, L.smem, st); break;
+    }
+    if (err == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();  // nothing was launched: the caller takes another path
+        return err;
+    }
     profile_mark(2, st);
     profile_mark(3, st);
     profile_mark(4, st);

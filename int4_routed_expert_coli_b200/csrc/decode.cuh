@@ -31,8 +31,18 @@ bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_s
 // scale matrices (2-D, padded rows).
 cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I,
                               CUtensorMap** d_maps);
-// Routing (or the given union), gate/up, down and combine in one launch.
+// True when at least one CTA of the kernel fits on an SM (so a grid of one
+// CTA per SM can be resident at once).
+bool decode_coresident(int H, int I, int E, int k, int n_shared, int num_sms);
+// Routing (or the given union), gate/up, down and combine in one cooperative
+// launch.  Returns cudaErrorCooperativeLaunchTooLarge, with nothing launched
+// and the error cleared, when the grid cannot be resident at once (fewer
+// usable SMs than the handle saw, e.g. a partitioned GPU): the caller then
+// runs the call on another path.
 cudaError_t launch_decode_fused(const DecodeArgs& d, int num_sms, cudaStream_t st);
+// Test hook: with `on`, the next launch_decode_fused behaves as if the launch
+// had been refused for lack of co-resident SMs; false clears it.
+void decode_force_not_resident(bool on);
 // Encode a 3-D uint8 tensor map over a [rows][row_bytes] matrix viewed as
 // [rows][row_bytes / 128][128], box {128, segs, box_rows}, 128-byte swizzle;
 // chunks past the row end read as zero.

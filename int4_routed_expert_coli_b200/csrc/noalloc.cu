@@ -14,7 +14,9 @@
 // passes the array's name to a kernel (on the host it is only a stand-in, not
 // a device address); the first call on each device, with that device
 // current, looks up the array's device address with cudaGetSymbolAddress and
-// keeps it.  That first call should come before any stream capture.
+// keeps it.  Every call copies the expert pointer table into the array from
+// pageable host memory, a copy a stream capture cannot record: no call of
+// this entry point may be made under stream capture.
 //
 // Sharing: every call (on a device) uses the same array, which keeps the last
 // call's contents; the call clears the part that must start at zero (the

@@ -67,3 +67,27 @@ def reference_layer(bank, E, k, n_shared, x, logits, residual=None, sample=None)
     out = oracle.layer(bank.hidden, bank.inter, E, k, n_shared, ex, bits(x), idx, w, residual=res,
                        sample=sample.astype(np.int32), n_threads=threads())
     return out, idx, w
+
+
+def covering_sample(idx: np.ndarray, n_total: int) -> np.ndarray:
+    """A deterministic token sample in which every expert that ``idx``
+    ([T][k]) routes to appears at least once: a greedy set cover (the token
+    that adds the most uncovered experts, lowest index on ties), then evenly
+    spaced tokens up to ``n_total``.  Sorted ascending."""
+    T = idx.shape[0]
+    E = int(idx.max()) + 1
+    hit = np.zeros((T, E), dtype=bool)
+    hit[np.arange(T)[:, None], idx] = True
+    uncovered = hit.any(axis=0)
+    chosen = []
+    while uncovered.any():
+        gain = hit[:, uncovered].sum(axis=1)
+        t = int(np.argmax(gain))   # first maximum: the lowest token index
+        chosen.append(t)
+        uncovered &= ~hit[t]
+    picked = set(chosen)
+    for t in np.linspace(0, T - 1, n_total).round().astype(np.int64):
+        if len(picked) >= n_total:
+            break
+        picked.add(int(t))
+    return np.array(sorted(picked), dtype=np.int64)

@@ -86,3 +86,45 @@ def test_withheld_stage_in_fused_decode_times_out():
     assert c.coli_moe_get_status(ws) == c.COLI_OK
     ref, _, _ = reference_layer(bank, 256, 8, 1, x, lg)
     assert_close(out.cpu().numpy(), ref, "after timeout")
+
+
+def test_fused_decode_refused_launch_takes_the_streaming_path():
+    """GLM-5.2 shape, T = 1 and T = 4: when the fused decode kernel's
+    cooperative launch is refused (its grid of one CTA per SM cannot be
+    resident at once, as on a partitioned GPU; forced here by the test hook),
+    the call runs on the streaming kernels and still matches the oracle, for
+    the layer call and for the FFN call on a prepared union."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    bank = synth.make_expert_bank(6144, 2048, 257, seed=29, device="cuda")
+    layer = c.MoELayer(bank, n_routed=256, top_k=8, n_shared=1)
+    for T in (1, 4):
+        x = synth.make_activations(T, 6144, seed=30 + T, device="cuda")
+        lg = synth.make_logits_normal(T, 256, seed=40 + T, device="cuda")
+        ws = layer.workspace(T)
+        assert c.coli_moe_debug_inject(c.COLI_INJECT_NOT_RESIDENT) == c.COLI_OK
+        try:
+            out = layer.layer(x, logits=lg, ws=ws)
+        finally:
+            c.coli_moe_debug_inject(0)
+        assert c.coli_moe_get_status(ws) == c.COLI_OK
+        ref, _, _ = reference_layer(bank, 256, 8, 1, x, lg)
+        assert_close(out.cpu().numpy(), ref, f"refused fused launch, layer T={T}")
+
+        # the FFN entry point on a prepared union takes the same fallback
+        k, E = 8, 256
+        idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+        c.coli_moe_route(T, E, k, lg, idx, w)
+        i32 = dict(dtype=torch.int32, device="cuda")
+        counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+        pairs, active, na = torch.empty(T * k, **i32), torch.empty(E, **i32), torch.empty(1, **i32)
+        c.coli_moe_union(T, E, k, idx, counts, offsets, pairs, active, na)
+        out2 = torch.empty(T, 6144, dtype=torch.float32, device="cuda")
+        assert c.coli_moe_debug_inject(c.COLI_INJECT_NOT_RESIDENT) == c.COLI_OK
+        try:
+            c.coli_moe_ffn(layer.handle, T, x, w, counts, offsets, pairs, active, na, None,
+                           out2, c.COLI_OUT_F32, ws)
+        finally:
+            c.coli_moe_debug_inject(0)
+        assert c.coli_moe_get_status(ws) == c.COLI_OK
+        assert_close(out2.cpu().numpy(), ref, f"refused fused launch, ffn T={T}")
