@@ -215,6 +215,24 @@ coli_status coli_moe_layer_noalloc(const coli_moe_desc *desc, int32_t T, const v
                                    const float *logits, const void *residual, void *out,
                                    coli_out_dtype out_dtype, int32_t *status_out, void *stream);
 
+/* Combine step of the expert-parallel layer (experts partitioned over
+ * ranks): a local-cluster worker receives one layer's routed batch-union and
+ * runs the FFN ("yunpan.plus/t/30351-1-1", capability three, local cluster
+ * paragraph); the owner of a token then sums what comes back:
+ *   out[t] = ((sum_{j<k} rows[t*k + j]) + shared[t]) + residual[t]
+ * in fp32, in exactly that order.
+ *   rows     [T*k][H] fp32: the token's routed outputs, each already
+ *            multiplied by its gate weight, in slot order (nullable if k == 0)
+ *   shared   [T][H] fp32 nullable: the shared experts' output
+ *   residual [T][H] nullable, same dtype as out
+ *   out      [T][H] fp32 or bf16 (round to nearest even)
+ * All device pointers, 16-byte aligned; H a multiple of 4.  Asynchronous on
+ * `stream`.  Errors: INVALID_ARG (NULL, negative sizes, bad enum), SHAPE
+ * (H % 4), ALIGN. */
+coli_status coli_moe_combine_rows(int32_t T, int32_t k, int32_t H, const float *rows,
+                                  const float *shared, const void *residual, void *out,
+                                  coli_out_dtype out_dtype, void *stream);
+
 /* Synchronise `stream` and return the workspace's device status word
  * (COLI_OK, COLI_ERR_BAD_INDEX or COLI_ERR_TIMEOUT), or COLI_ERR_CUDA if the
  * stream reports an error.  The word stays set until coli_moe_workspace_clear. */

@@ -35,7 +35,8 @@ COLI_OUT_BF16 = 1
 
 EXPORTS = ("coli_moe_create", "coli_moe_destroy", "coli_moe_workspace_size",
            "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union", "coli_moe_ffn",
-           "coli_moe_layer", "coli_moe_layer_noalloc", "coli_moe_get_status",
+           "coli_moe_layer", "coli_moe_layer_noalloc", "coli_moe_combine_rows",
+           "coli_moe_get_status",
            "coli_moe_debug_inject",
            "coli_moe_profile_enable",
            "coli_moe_profile_read", "coli_status_string")
@@ -84,6 +85,8 @@ def _load():
     L.coli_moe_layer.restype = ctypes.c_int
     L.coli_moe_layer_noalloc.argtypes = [ctypes.POINTER(CDesc), i32, P, P, P, P, ctypes.c_int, P, P]
     L.coli_moe_layer_noalloc.restype = ctypes.c_int
+    L.coli_moe_combine_rows.argtypes = [i32, i32, i32, P, P, P, P, ctypes.c_int, P]
+    L.coli_moe_combine_rows.restype = ctypes.c_int
     L.coli_moe_get_status.argtypes = [P, P]
     L.coli_moe_get_status.restype = ctypes.c_int
     L.coli_moe_debug_inject.argtypes = [i32]
@@ -168,6 +171,13 @@ def coli_moe_layer_noalloc(desc, T, x, logits, residual, out, out_dtype, status_
     s = lib.coli_moe_layer_noalloc(ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(residual),
                                    _ptr(out), out_dtype, _ptr(status_out), _stream(stream))
     return _check(s, "coli_moe_layer_noalloc", raise_on_error)
+
+
+def coli_moe_combine_rows(T, k, H, rows, shared, residual, out, out_dtype, stream=None,
+                          raise_on_error=True):
+    s = lib.coli_moe_combine_rows(T, k, H, _ptr(rows), _ptr(shared), _ptr(residual), _ptr(out),
+                                  out_dtype, _stream(stream))
+    return _check(s, "coli_moe_combine_rows", raise_on_error)
 
 
 def coli_moe_workspace_clear(ws, stream=None, raise_on_error=True):

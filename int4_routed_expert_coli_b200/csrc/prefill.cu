@@ -57,14 +57,36 @@
 namespace coli {
 namespace {
 
-constexpr int BM = 128, BN = 192, BK = 64;
+constexpr int BM = 128, BK = 64;
 constexpr int kBRowQuant = 32;      // activation rows are loaded in multiples of 32
 constexpr int kThreadsP = 512;
-constexpr int kEpiWarps = 8;  // warps 8-15: two per tensor-memory lane quarter
 constexpr uint32_t kTmemColsP = 512;
-constexpr uint32_t kAccCols = 2 * BN;  // accumulators; the operand ring follows
 constexpr int kHeaderP = 2048;
 constexpr int kSmemLimitP = 227 * 1024;
+
+// Two shapes of the same pipeline.  Large token tiles (prefill: ~128 tokens
+// per expert): 192-token tiles, one accumulator, a 2-deep operand ring, 4
+// dequantising warps (one weight row of both blocks per thread) and 8
+// epilogue warps.  Small token tiles (a few tokens per expert, every call
+// with T <= 64): 64-token tiles, a double-buffered accumulator, a 4-deep
+// operand ring, 8 dequantising warps (one weight row of one block per
+// thread) and 4 epilogue warps: there the dequantisation, not the MMA or the
+// epilogue, sets the rate.
+template <bool kSmall>
+struct Cfg {
+    static constexpr int BN = kSmall ? 64 : 192;            // tokens per tile (max)
+    static constexpr int kAccBufs = kSmall ? 2 : 1;
+    static constexpr uint32_t kAccCols = 2 * BN * kAccBufs;  // accumulators, then the ring
+    static constexpr int kACols = BK;                        // operand columns per K-block (2 blocks)
+    static constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;
+    static constexpr int kDqWarp0 = kSmall ? 8 : 4;
+    static constexpr int kDqWarps = kSmall ? 8 : 4;
+    static constexpr int kEpiWarp0 = kSmall ? 4 : 8;
+    static constexpr int kEpiWarps = kSmall ? 4 : 8;
+    static constexpr int kBBytes = BN * BK * 2;               // activation tile per stage
+    static constexpr int kStage = kBBytes + 2 * BM * BK / 2;  // + two blocks of packed codes
+};
+static_assert(Cfg<false>::kAStages == 2 && Cfg<true>::kAStages == 4, "operand ring depth");
 
 // Position of element k (0..7) of an 8-group in the operand order.
 __host__ __device__ __forceinline__ int perm8(int k) { return (k & 3) * 2 + (k >> 2); }
@@ -188,6 +210,7 @@ struct TileInfo {
     bool valid;
 };
 
+template <int BN>
 __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_t tile,
                                               int n_slots, int m_tiles) {
     TileInfo ti;
@@ -232,18 +255,17 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_
 // Two MMAs per K step on one activation tile: kGU gate/up (the gate rows and
 // the up rows of the same 128 features, K = H), otherwise down (two blocks of
 // 128 rows of W_d, 256 output features, K = I).
-template <bool kGU>
+template <bool kGU, bool kSmall>
 __global__ void __launch_bounds__(kThreadsP, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     const __grid_constant__ CUtensorMap bmap64,
                     const __grid_constant__ CUtensorMap bmap32, const GemmArgs a, int stages) {
+    using C = Cfg<kSmall>;
+    constexpr int BN = C::BN;
     constexpr int NA = 2;                                    // weight blocks per tile
     constexpr int kFeat = kGU ? BM : 2 * BM;                 // output features per tile
-    constexpr int kBBytes = BN * BK * 2;                     // 24 KB
-    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per matrix
-    constexpr int kStage = kBBytes + NA * kPkBytes;
-    constexpr int kACols = NA * BK / 2;                      // operand columns per K-block
-    constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;  // 2
+    constexpr int kPkBytes = BM * BK / 2;                    // 4 KB per block
+    constexpr int kAStages = C::kAStages;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -251,8 +273,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // TMA landed
     uint64_t* dq_full = full + 16;                             // operand written to TMEM
     uint64_t* empty = full + 32;                               // MMAs done reading the stage
-    uint64_t* acc_full = full + 48;                            // accumulator ready
-    uint64_t* acc_empty = full + 50;                           // accumulator drained
+    uint64_t* acc_full = full + 48;                            // [2] accumulator ready
+    uint64_t* acc_empty = full + 50;                           // [2] accumulator drained
     uint64_t* a_empty = full + 52;                             // [kAStages] MMAs done with an operand
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 512);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 520);
@@ -265,11 +287,13 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&dq_full[s], 4);
+            mbar_init(&dq_full[s], C::kDqWarps);
             mbar_init(&a_empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kEpiWarps);
+        for (int b = 0; b < C::kAccBufs; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], C::kEpiWarps);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -299,7 +323,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
     const int G = K / kGroup;
     const int64_t n_tiles = (int64_t)__ldg(a.ntile_start + n_slots) * m_tiles;
 
-    auto stage_ptr = [&](int s) { return stage0 + (size_t)s * kStage; };
+    auto stage_ptr = [&](int s) { return stage0 + (size_t)s * C::kStage; };
     auto timeout = [&]() {
         report(a.status, COLI_ERR_TIMEOUT);
         *abort_flag = 1;
@@ -311,7 +335,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             const uint64_t policy = policy_evict_first();
             Ring rs;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
-                const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+                const TileInfo ti = tile_info<BN>(a, kGU, tile, n_slots, m_tiles);
                 const CUtensorMap* wm = a.wmaps + (size_t)ti.e * 3;
                 const int f0 = ti.m_tile * kFeat;
                 // only the token rows the tile has, rounded up to 32, in at
@@ -326,7 +350,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     rs.next(stages);
                     uint8_t* st = stage_ptr(s);
                     mbar_arrive_expect_tx(&full[s], NA * kPkBytes + brows * BK * 2);
-                    uint8_t* pk = st + kBBytes;
+                    uint8_t* pk = st + C::kBBytes;
                     if constexpr (kGU) {
                         tma_load_2d_hint(pk, wm + 0, kb * (BK / 2), f0, &full[s], policy);
                         tma_load_2d_hint(pk + kPkBytes, wm + 1, kb * (BK / 2), f0, &full[s],
@@ -358,16 +382,18 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             int64_t lt = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag;
                  tile += gridDim.x, ++lt) {
-                const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-                // one accumulator (NA x BN = 384 columns): tile lt waits for the
-                // epilogue of tile lt - 1
-                if (lt > 0 && !mbar_wait(acc_empty, (uint32_t)(lt - 1) & 1)) {
+                const TileInfo ti = tile_info<BN>(a, kGU, tile, n_slots, m_tiles);
+                // accumulator buffer lt % kAccBufs: wait for the epilogue of
+                // the tile that used it before
+                const int buf = (int)(lt % C::kAccBufs);
+                const int64_t use = lt / C::kAccBufs;
+                if (use > 0 && !mbar_wait(&acc_empty[buf], (uint32_t)(use - 1) & 1)) {
                     timeout();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t idesc = idesc_f16(ti.n_mma);
-                const uint32_t d0 = tmem_base;
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * NA * BN);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     const int s = rs.i, as = ra.i;
@@ -380,7 +406,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     ra.next(kAStages);
                     tc_fence_after();
                     const uint64_t bdesc = desc_sw128(smem_addr(stage_ptr(s)));
-                    const uint32_t a0 = tmem_base + kAccCols + (uint32_t)(as * kACols);
+                    const uint32_t a0 = tmem_base + C::kAccCols + (uint32_t)(as * C::kACols);
 #pragma unroll
                     for (int m = 0; m < NA; ++m)
                         mma_kblock_ts(d0 + m * BN, a0 + m * (BK / 2), bdesc, idesc, kb != 0);
@@ -388,17 +414,22 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     mma_commit(&a_empty[as]);
                 }
                 if (!ok) break;
-                mma_commit(acc_full);
+                mma_commit(&acc_full[buf]);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= C::kDqWarp0 && warp < C::kDqWarp0 + C::kDqWarps) {
         // ------------------------------- dequant -------------------------------
-        const int row = threadIdx.x - 128;  // MMA row of the tile owned by this thread
+        // large tiles: one weight row of both blocks per thread; small tiles:
+        // two warps per lane quarter, each one block
+        const int q = warp & 3;
+        const int row = q * 32 + lane;  // MMA row of the tile owned by this thread
+        constexpr int kMyBlocks = kSmall ? 1 : NA;
+        const int blk0 = kSmall ? (warp - C::kDqWarp0) >> 2 : 0;
         // this warp's 32 lanes of the operand ring
-        const uint32_t ta = tmem_base + ((uint32_t)(warp & 3) << 21) + kAccCols;
+        const uint32_t ta = tmem_base + ((uint32_t)q << 21) + C::kAccCols;
         Ring rs, ra;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
+            const TileInfo ti = tile_info<BN>(a, kGU, tile, n_slots, m_tiles);
             const DevExpert ex = a.experts[ti.e];
             // gate/up: gate and up row of feature f0 + row; down: W_d rows
             // f0 + row and f0 + 128 + row (the latter past H in a ragged last
@@ -406,15 +437,25 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             const int f0 = ti.m_tile * kFeat;
             const int64_t srow = (int64_t)(f0 + row) * G;
             const bool has1 = kGU || f0 + BM < a.H;
-            const uint16_t* sc0 = (kGU ? ex.gate_s : ex.down_s) + srow;
-            const uint16_t* sc1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * G;
-            uint16_t nxt0 = __ldg(sc0), nxt1 = has1 ? __ldg(sc1) : 0;
+            const uint16_t* sc_b0 = (kGU ? ex.gate_s : ex.down_s) + srow;
+            const uint16_t* sc_b1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * G;
+            const uint16_t* scp[kMyBlocks];
+            bool live[kMyBlocks];
+            uint16_t nxt[kMyBlocks];
+#pragma unroll
+            for (int m = 0; m < kMyBlocks; ++m) {
+                const int blk = blk0 + m;
+                scp[m] = blk == 0 ? sc_b0 : sc_b1;
+                live[m] = blk == 0 || has1;
+                nxt[m] = live[m] ? __ldg(scp[m]) : 0;
+            }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
-                const uint16_t cur[2] = {nxt0, nxt1};
-                if (kb + 1 < KB) {
-                    nxt0 = __ldg(sc0 + kb + 1);
-                    if (has1) nxt1 = __ldg(sc1 + kb + 1);
+                uint16_t cur[kMyBlocks];
+#pragma unroll
+                for (int m = 0; m < kMyBlocks; ++m) {
+                    cur[m] = nxt[m];
+                    if (kb + 1 < KB && live[m]) nxt[m] = __ldg(scp[m] + kb + 1);
                 }
                 const int s = rs.i, as = ra.i;
                 if (!mbar_wait(&full[s], (uint32_t)rs.pass & 1) ||
@@ -427,35 +468,40 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                 ra.next(kAStages);
                 tc_fence_after();
 #pragma unroll
-                for (int m = 0; m < NA; ++m) {
-                    const uint4* pk = reinterpret_cast<const uint4*>(stage_ptr(s) + kBBytes +
-                                                                     m * kPkBytes + row * 32);
+                for (int m = 0; m < kMyBlocks; ++m) {
+                    const int blk = blk0 + m;
+                    const uint4* pk = reinterpret_cast<const uint4*>(stage_ptr(s) + C::kBBytes +
+                                                                     blk * kPkBytes + row * 32);
                     const uint4 p0 = pk[0], p1 = pk[1];
                     const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    // bf16 scale -> fp16 (exact for scales in fp16's normal range)
-                    const __half sh = __float2half_rn(__uint_as_float((uint32_t)cur[m] << 16));
-                    const __half2 s2 = __halves2half2(sh, sh);
+                    // bf16 scale s -> fp16 s, s / 16 and -72 s (all exact: the
+                    // scale's 8 significant bits, 72 = 64 + 8 adds 3 more)
+                    const float sf = __uint_as_float((uint32_t)cur[m] << 16);
+                    const __half2 s2 = __float2half2_rn(sf);
+                    const __half2 s16 = __float2half2_rn(sf * 0.0625f);
+                    const __half2 c72 = __float2half2_rn(-72.f * sf);
+                    const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
                     uint32_t cols[32];  // column 4c + i: elements i, i + 4 of 8-group c
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const uint32_t w = words[c], w8 = w >> 8;
+                        // even codes: (1032 + q) - 1032, times s; odd codes
+                        // (1152 + 16 q): one fused multiply-add with s / 16 and
+                        // -72 s, whose exact result q s is an fp16 value
                         uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
                         uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
                         uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
                         uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
-                        const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
-                        const __half2 sx = __floats2half2_rn(0.0625f, 0.0625f);
-                        const __half2 hi = __floats2half2_rn(-72.f, -72.f);
                         __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
-                        __half2 v1 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t1), sx, hi), s2);
+                        __half2 v1 = __hfma2(*reinterpret_cast<__half2*>(&t1), s16, c72);
                         __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
-                        __half2 v3 = __hmul2(__hfma2(*reinterpret_cast<__half2*>(&t3), sx, hi), s2);
+                        __half2 v3 = __hfma2(*reinterpret_cast<__half2*>(&t3), s16, c72);
                         cols[4 * c + 0] = *reinterpret_cast<uint32_t*>(&v0);
                         cols[4 * c + 1] = *reinterpret_cast<uint32_t*>(&v1);
                         cols[4 * c + 2] = *reinterpret_cast<uint32_t*>(&v2);
                         cols[4 * c + 3] = *reinterpret_cast<uint32_t*>(&v3);
                     }
-                    tmem_st32(ta + (uint32_t)(as * kACols + m * (BK / 2)), cols);
+                    tmem_st32(ta + (uint32_t)(as * C::kACols + blk * (BK / 2)), cols);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -464,29 +510,31 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             }
             if (!ok) break;
         }
-    } else if (warp >= 8) {
+    } else if (warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + C::kEpiWarps) {
         // ------------------------------- epilogue ------------------------------
         const int q = warp & 3;
-        const int c_first = ((warp - 8) >> 2) * 32;  // the two warps of a quarter take
-                                                     // alternate 32-token chunks
+        // large tiles: the two warps of a quarter take alternate 32-token chunks
+        const int c_first = ((warp - C::kEpiWarp0) >> 2) * 32;
+        constexpr int c_step = 32 * (C::kEpiWarps / 4);
         const int row = q * 32 + lane;  // accumulator lane = MMA row of the tile
         int64_t lt = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
-            const TileInfo ti = tile_info(a, kGU, tile, n_slots, m_tiles);
-            if (!mbar_wait(acc_full, (uint32_t)lt & 1)) {
+            const TileInfo ti = tile_info<BN>(a, kGU, tile, n_slots, m_tiles);
+            const int buf = (int)(lt % C::kAccBufs);
+            if (!mbar_wait(&acc_full[buf], (uint32_t)(lt / C::kAccBufs) & 1)) {
                 if (lane == 0) timeout();
                 break;
             }
             tc_fence_after();
-            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16);
+            const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NA * BN);
             const int feat = ti.m_tile * kFeat + row;
             if constexpr (kGU) {
-                // gate and up of this lane's feature sit in the same lane; the
-                // next tile's MMAs wait for this (single accumulator buffer),
+                // gate and up of this lane's feature sit in the same lane; with
+                // one accumulator buffer the next tile's MMAs wait for this,
                 // so SiLU uses the fast exponential and division
                 const int col = perm_col(feat);
                 __half* hcol = a.hbuf + (int64_t)ti.out_row0 * a.I + col;
-                for (int c0 = c_first; c0 < ti.ntok; c0 += 64) {
+                for (int c0 = c_first; c0 < ti.ntok; c0 += c_step) {
                     uint32_t vg[32], vu[32];
                     tmem_ld32(tq + c0, vg);
                     tmem_ld32(tq + BN + c0, vu);
@@ -506,7 +554,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             } else {
                 const bool has1 = feat + BM < a.H;
                 float* yrow = a.y + (int64_t)ti.out_row0 * a.H + feat;
-                for (int c0 = c_first; c0 < ti.ntok; c0 += 64) {
+                for (int c0 = c_first; c0 < ti.ntok; c0 += c_step) {
                     uint32_t v0[32], v1[32];
                     tmem_ld32(tq + c0, v0);
                     tmem_ld32(tq + BN + c0, v1);
@@ -521,7 +569,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
@@ -539,7 +587,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
 // xg[s] = fp16(x[pairs[s] / k]) for s < P (the union's order), xg[P + t] =
 // fp16(x[t]) (the shared experts' rows), columns in operand order.  Block 0
 // also lays out the tile list: ntile_start[slot] = sum over earlier slots of
-// ceil(tokens / BN).
+// ceil(tokens / bn), bn the GEMM's token-tile width.
 __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
     pdl_wait();
     pdl_launch_dependents();
@@ -564,7 +612,7 @@ __global__ void __launch_bounds__(1024) gather_kernel(GatherArgs g) {
                 if (e >= 0 && e < g.E && b >= 0 && en >= b && en <= P) ntok = en - b;
                 else report(g.status, COLI_ERR_BAD_INDEX);
             }
-            cnt[u] = slot < n_slots ? (max(ntok, 0) + BN - 1) / BN : 0;
+            cnt[u] = slot < n_slots ? (max(ntok, 0) + g.bn - 1) / g.bn : 0;
         }
         int total;
         const int base = block_exclusive_scan(cnt[0] + cnt[1], scan_tmp, &total);
@@ -641,19 +689,17 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kGU>
+template <bool kSmall>
 int gemm_stages() {
-    constexpr int kStage = BN * BK * 2 + 2 * BM * BK / 2;
-    return std::min(16, (kSmemLimitP - kHeaderP - 1024) / kStage);
+    return std::min(16, (kSmemLimitP - kHeaderP - 1024) / Cfg<kSmall>::kStage);
 }
 
-template <bool kGU>
+template <bool kGU, bool kSmall>
 cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num_sms,
                         cudaStream_t st) {
-    constexpr int kStage = BN * BK * 2 + 2 * BM * BK / 2;
-    const int stages = gemm_stages<kGU>();
-    const int smem = kHeaderP + 1024 + stages * kStage;
-    cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU>,
+    const int stages = gemm_stages<kSmall>();
+    const int smem = kHeaderP + 1024 + stages * Cfg<kSmall>::kStage;
+    cudaError_t err = cudaFuncSetAttribute(prefill_gemm_kernel<kGU, kSmall>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -666,8 +712,8 @@ cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<kGU>, bmap[0], bmap[1], bmap[2], a,
-                              stages);
+    return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel<kGU, kSmall>, bmap[0], bmap[1], bmap[2],
+                              a, stages);
 }
 
 }  // namespace
@@ -706,7 +752,11 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
                            int num_sms, cudaStream_t st) {
     const int P = f.T * f.k;
     const int S = P + f.T * f.n_shared;
+    // small token tiles when every list fits one (T <= 64) or the routed
+    // experts average at most 8 tokens
+    const bool small = f.T <= Cfg<true>::BN || (int64_t)P <= 8 * (int64_t)f.E;
     GatherArgs g;
+    g.bn = small ? Cfg<true>::BN : Cfg<false>::BN;
     g.T = f.T;
     g.k = f.k;
     g.E = f.E;
@@ -762,10 +812,12 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
             return cudaErrorInvalidValue;
     }
     profile_mark(1, st);
-    cudaError_t err = launch_gemm<true>(xmap, a, num_sms, st);
+    cudaError_t err = small ? launch_gemm<true, true>(xmap, a, num_sms, st)
+                            : launch_gemm<true, false>(xmap, a, num_sms, st);
     if (err != cudaSuccess) return err;
     profile_mark(2, st);
-    err = launch_gemm<false>(hmap, a, num_sms, st);
+    err = small ? launch_gemm<false, true>(hmap, a, num_sms, st)
+                : launch_gemm<false, false>(hmap, a, num_sms, st);
     profile_mark(3, st);
     return err;
 }

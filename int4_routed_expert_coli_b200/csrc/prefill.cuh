@@ -22,6 +22,7 @@ struct GemmArgs {
 
 struct GatherArgs {
     int T, k, E, H, n_shared;
+    int bn;                  // token-tile width of the GEMM that follows
     const __nv_bfloat16* x;  // [T][H]
     const int* pairs;        // [T*k]
     const int* offsets;
