@@ -439,23 +439,46 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             const bool has1 = kGU || f0 + BM < a.H;
             const uint16_t* sc_b0 = (kGU ? ex.gate_s : ex.down_s) + srow;
             const uint16_t* sc_b1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * G;
+            // Scales: a row's scales are contiguous, so where a row of them
+            // is a whole number of 16-byte chunks (G % 8 == 0) a thread
+            // loads 8 at a time, one chunk (8 K-blocks) ahead, and the load
+            // latency hides behind 8 K-blocks of work; otherwise one scale
+            // per K-block, one ahead.
+            const bool vec = (G & 7) == 0;
             const uint16_t* scp[kMyBlocks];
             bool live[kMyBlocks];
+            uint4 chunk[kMyBlocks], chunk_nxt[kMyBlocks];
             uint16_t nxt[kMyBlocks];
 #pragma unroll
             for (int m = 0; m < kMyBlocks; ++m) {
                 const int blk = blk0 + m;
                 scp[m] = blk == 0 ? sc_b0 : sc_b1;
                 live[m] = blk == 0 || has1;
-                nxt[m] = live[m] ? __ldg(scp[m]) : 0;
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                chunk[m] = z;
+                chunk_nxt[m] = (vec && live[m]) ? __ldg(reinterpret_cast<const uint4*>(scp[m])) : z;
+                nxt[m] = (!vec && live[m]) ? __ldg(scp[m]) : 0;
             }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb) {
                 uint16_t cur[kMyBlocks];
+                const int sub = kb & 7;
 #pragma unroll
                 for (int m = 0; m < kMyBlocks; ++m) {
-                    cur[m] = nxt[m];
-                    if (kb + 1 < KB && live[m]) nxt[m] = __ldg(scp[m] + kb + 1);
+                    if (vec) {
+                        if (sub == 0) {
+                            chunk[m] = chunk_nxt[m];
+                            if (kb + 8 < KB && live[m])
+                                chunk_nxt[m] =
+                                    __ldg(reinterpret_cast<const uint4*>(scp[m] + kb + 8));
+                        }
+                        const uint32_t w2 = sub < 4 ? (sub < 2 ? chunk[m].x : chunk[m].y)
+                                                    : (sub < 6 ? chunk[m].z : chunk[m].w);
+                        cur[m] = (uint16_t)((sub & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
+                    } else {
+                        cur[m] = nxt[m];
+                        if (kb + 1 < KB && live[m]) nxt[m] = __ldg(scp[m] + kb + 1);
+                    }
                 }
                 const int s = rs.i, as = ra.i;
                 if (!mbar_wait(&full[s], (uint32_t)rs.pass & 1) ||
@@ -474,28 +497,31 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                                                                      blk * kPkBytes + row * 32);
                     const uint4 p0 = pk[0], p1 = pk[1];
                     const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    // bf16 scale s -> fp16 s, s / 16 and -72 s (all exact: the
-                    // scale's 8 significant bits, 72 = 64 + 8 adds 3 more)
+                    // bf16 scale s -> fp16 s and s / 16 (exact for scales in
+                    // fp16's normal range: 8 significant bits)
                     const float sf = __uint_as_float((uint32_t)cur[m] << 16);
                     const __half2 s2 = __float2half2_rn(sf);
                     const __half2 s16 = __float2half2_rn(sf * 0.0625f);
-                    const __half2 c72 = __float2half2_rn(-72.f * sf);
                     const __half2 lo = __floats2half2_rn(1032.f, 1032.f);
+                    const __half2 hi = __floats2half2_rn(1152.f, 1152.f);
                     uint32_t cols[32];  // column 4c + i: elements i, i + 4 of 8-group c
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const uint32_t w = words[c], w8 = w >> 8;
-                        // even codes: (1032 + q) - 1032, times s; odd codes
-                        // (1152 + 16 q): one fused multiply-add with s / 16 and
-                        // -72 s, whose exact result q s is an fp16 value
+                        // even codes (1032 + q) - 1032 = q, odd codes
+                        // (1152 + 16 q) - 1152 = 16 q, both exact; times s and
+                        // s / 16, exact (q s has at most 11 significant bits).
+                        // A single fused multiply-add with a -72 s or -1032 s
+                        // addend would not be exact: those products need up to
+                        // 12 and 15 significant bits.
                         uint32_t t0 = (w & 0x000F000Fu) ^ 0x64086408u;
                         uint32_t t1 = (w & 0x00F000F0u) ^ 0x64806480u;
                         uint32_t t2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
                         uint32_t t3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
                         __half2 v0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t0), lo), s2);
-                        __half2 v1 = __hfma2(*reinterpret_cast<__half2*>(&t1), s16, c72);
+                        __half2 v1 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t1), hi), s16);
                         __half2 v2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t2), lo), s2);
-                        __half2 v3 = __hfma2(*reinterpret_cast<__half2*>(&t3), s16, c72);
+                        __half2 v3 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&t3), hi), s16);
                         cols[4 * c + 0] = *reinterpret_cast<uint32_t*>(&v0);
                         cols[4 * c + 1] = *reinterpret_cast<uint32_t*>(&v1);
                         cols[4 * c + 2] = *reinterpret_cast<uint32_t*>(&v2);
