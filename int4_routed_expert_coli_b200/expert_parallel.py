@@ -196,4 +196,4 @@ def _sub_bank(bank, lo, hi):
     from .synth import ExpertBank
     return ExpertBank(bank.hidden, bank.inter, hi - lo, bank.gate_q[lo:hi], bank.up_q[lo:hi],
                       bank.down_q[lo:hi], bank.gate_s[lo:hi], bank.up_s[lo:hi],
-                      bank.down_s[lo:hi])
+                      bank.down_s[lo:hi], bank.per_row)

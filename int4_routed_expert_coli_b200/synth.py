@@ -11,7 +11,9 @@ Formats (the layer's inputs, as the C-ABI header documents them):
   are uint8, two signed int4 codes per byte along the reduction dimension;
   a uniformly random byte gives two independent codes uniform over [-8, 7].
 * scales ``gate_s``/``up_s`` ``[I][H/64]`` and ``down_s`` ``[H][I/64]`` are
-  bf16, drawn from U(0.005, 0.02) in fp32 and rounded to bf16 (RNE).
+  bf16, drawn from U(0.005, 0.02) in fp32 and rounded to bf16 (RNE); in the
+  per-row format (``per_row=True``) one scale per row, ``[I][1]`` and
+  ``[H][1]``, drawn the same way.
 * activations ``x`` ``[T][H]`` are bf16 drawn from N(0, 1).
 * router logits ``[T][E]`` are fp32; the router weight ``[E][H]`` is fp32
   N(0, 0.02).
@@ -54,18 +56,23 @@ class ExpertBank:
     gate_s: torch.Tensor  # [n][I][H/64] bf16
     up_s: torch.Tensor    # [n][I][H/64] bf16
     down_s: torch.Tensor  # [n][H][I/64] bf16
+    per_row: bool = False  # scales [rows][1]: one per row instead of one per 64 codes
 
     def expert_numpy(self, e: int) -> dict:
-        """Copy expert ``e`` to host numpy arrays (scales as raw bf16 bits)."""
+        """Copy expert ``e`` to host numpy arrays (scales as raw bf16 bits;
+        "group" 64 for gs64, 0 for one scale per row)."""
         out = {}
         for name in ("gate_q", "up_q", "down_q"):
             out[name] = getattr(self, name)[e].cpu().numpy()
         for name in ("gate_s", "up_s", "down_s"):
             out[name] = getattr(self, name)[e].cpu().view(torch.int16).numpy().view(np.uint16)
+        out["group"] = 0 if self.per_row else GROUP
         return out
 
     def nbytes_per_expert(self) -> int:
         h, i = self.hidden, self.inter
+        if self.per_row:
+            return 3 * h * i // 2 + (2 * i + h) * 2
         return 3 * h * i // 2 + 3 * (h * i // GROUP) * 2
 
 
@@ -88,10 +95,11 @@ STACK_CODE_RANGE = (-7, 7)
 
 def make_expert_bank(hidden: int, inter: int, n_experts: int, seed: int,
                      device="cpu", scale_range=(0.005, 0.02),
-                     code_range=(-8, 7)) -> ExpertBank:
-    """Random int4 gs64 experts: codes uniform over code_range (default
-    [-8, 7]: every nibble value), scales U(scale_range) rounded to bf16
-    (default U(.005, .02))."""
+                     code_range=(-8, 7), per_row: bool = False) -> ExpertBank:
+    """Random int4 experts: codes uniform over code_range (default [-8, 7]:
+    every nibble value), scales U(scale_range) rounded to bf16 (default
+    U(.005, .02)), one per 64 codes of a row (gs64) or, with per_row, one per
+    row."""
     if hidden % (2 * GROUP) or inter % (2 * GROUP):
         raise ValueError("hidden and inter must be multiples of 128")
     g = _gen(seed, device)
@@ -114,10 +122,11 @@ def make_expert_bank(hidden: int, inter: int, n_experts: int, seed: int,
         s.uniform_(scale_range[0], scale_range[1], generator=g)
         return s.to(torch.bfloat16)
 
-    gate_s = scales(inter, hidden // GROUP)
-    up_s = scales(inter, hidden // GROUP)
-    down_s = scales(hidden, inter // GROUP)
-    return ExpertBank(hidden, inter, n_experts, gate_q, up_q, down_q, gate_s, up_s, down_s)
+    gate_s = scales(inter, 1 if per_row else hidden // GROUP)
+    up_s = scales(inter, 1 if per_row else hidden // GROUP)
+    down_s = scales(hidden, 1 if per_row else inter // GROUP)
+    return ExpertBank(hidden, inter, n_experts, gate_q, up_q, down_q, gate_s, up_s, down_s,
+                      per_row)
 
 
 def make_activations(tokens: int, hidden: int, seed: int, device="cpu") -> torch.Tensor:

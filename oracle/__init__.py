@@ -36,7 +36,8 @@ def build(force: bool = False) -> str:
 class Expert(ctypes.Structure):
     _fields_ = [("gate_q", ctypes.c_void_p), ("up_q", ctypes.c_void_p),
                 ("down_q", ctypes.c_void_p), ("gate_s", ctypes.c_void_p),
-                ("up_s", ctypes.c_void_p), ("down_s", ctypes.c_void_p)]
+                ("up_s", ctypes.c_void_p), ("down_s", ctypes.c_void_p),
+                ("group", ctypes.c_int32)]
 
 
 def lib():
@@ -53,6 +54,8 @@ def lib():
         L.oracle_int4_pack.restype = None
         L.oracle_weight.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
         L.oracle_weight.restype = ctypes.c_double
+        L.oracle_weight_per_row.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_weight_per_row.restype = ctypes.c_double
         L.oracle_route.argtypes = [i32, i32, i32, P, P, P]
         L.oracle_route.restype = i32
         L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P]
@@ -103,6 +106,13 @@ def weight(q: np.ndarray, s_bits: np.ndarray, K: int, n: int, k: int) -> float:
     return lib().oracle_weight(_p(q), _p(s_bits), K, n, k)
 
 
+def weight_per_row(q: np.ndarray, s_bits: np.ndarray, K: int, n: int, k: int) -> float:
+    """W[n][k] of a per-row int4 matrix (one bf16 scale per row)."""
+    q = _c(q, np.uint8)
+    s_bits = _c(s_bits, np.uint16)
+    return lib().oracle_weight_per_row(_p(q), _p(s_bits), K, n, k)
+
+
 # ---- routing and union ------------------------------------------------------
 
 def route(logits: np.ndarray, k: int):
@@ -151,8 +161,9 @@ def union(idx: np.ndarray, E: int):
 
 class Experts:
     """Host expert table for the oracle: ``experts[e]`` is a dict of numpy
-    arrays (gate_q, up_q, down_q uint8; gate_s, up_s, down_s uint16 bf16 bits)
-    or None for an expert the caller knows is never selected."""
+    arrays (gate_q, up_q, down_q uint8; gate_s, up_s, down_s uint16 bf16 bits,
+    and optionally "group": 64 for gs64, the default, or 0 for one scale per
+    row) or None for an expert the caller knows is never selected."""
 
     def __init__(self, experts: list):
         self.keep = []
@@ -168,6 +179,7 @@ class Experts:
             self.keep.append(arrs)
             for name, a in arrs.items():
                 setattr(self.table[e], name, a.ctypes.data)
+            self.table[e].group = int(ex.get("group", 64))
         self.present = [ex is not None for ex in experts]
 
 

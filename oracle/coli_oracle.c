@@ -44,7 +44,9 @@
 
 typedef struct {
     const uint8_t *gate_q, *up_q, *down_q;   /* [I][H/2], [I][H/2], [H][I/2] */
-    const uint16_t *gate_s, *up_s, *down_s;  /* bf16 bits [I][H/64], [I][H/64], [H][I/64] */
+    const uint16_t *gate_s, *up_s, *down_s;  /* bf16 bits [I][H/64], [I][H/64], [H][I/64];
+                                                per-row: [I][1], [I][1], [H][1] */
+    int32_t group;                           /* 64: gs64; 0: one scale per row */
 } oracle_expert;
 
 /* ---- scalar formats --------------------------------------------------- */
@@ -74,11 +76,32 @@ void oracle_int4_pack(const int8_t *codes, int64_t n, uint8_t *row) {
     }
 }
 
+/* Dequantised weight W[n][k] of a [rows][K] matrix in the legacy per-row
+ * int4 format: the same codes, one bf16 scale per row, W[n][k] = q[n][k] *
+ * s[n] ("ssnai.com/JustVugg_colibri.html", decision guide: the older per-row
+ * int4 GLM-5.2 mirror; "yunpan.plus/t/30351-1-1", capability four: gs64
+ * against per-row int4).  The pages do not print the layout; this reading
+ * keeps everything of gs64 but the scale index. */
+double oracle_weight_per_row(const uint8_t *q, const uint16_t *s, int64_t K, int64_t n,
+                             int64_t k) {
+    const uint8_t *row = q + n * (K / 2);
+    return (double)oracle_int4_code(row, k) * oracle_bf16_to_double(s[n]);
+}
+
+/* W[n][k] of an expert matrix in the expert's format (gs64 or per-row). */
+static double weight_of(const uint8_t *q, const uint16_t *s, int64_t K, int32_t group, int64_t n,
+                        int64_t k);
+
 /* Dequantised weight W[n][k] of a [rows][K] gs64 matrix. */
 double oracle_weight(const uint8_t *q, const uint16_t *s, int64_t K, int64_t n, int64_t k) {
     const uint8_t *row = q + n * (K / 2);
     double scale = oracle_bf16_to_double(s[n * (K / 64) + k / 64]);
     return (double)oracle_int4_code(row, k) * scale;
+}
+
+static double weight_of(const uint8_t *q, const uint16_t *s, int64_t K, int32_t group, int64_t n,
+                        int64_t k) {
+    return group == 0 ? oracle_weight_per_row(q, s, K, n, k) : oracle_weight(q, s, K, n, k);
 }
 
 /* ---- routing ----------------------------------------------------------- */
@@ -192,14 +215,15 @@ static void expert_ffn(int H, int I, const oracle_expert *ex, const double *x, d
     for (int n = 0; n < I; ++n) {
         double g = 0.0, u = 0.0;
         for (int k = 0; k < H; ++k) {
-            g += oracle_weight(ex->gate_q, ex->gate_s, H, n, k) * x[k];
-            u += oracle_weight(ex->up_q, ex->up_s, H, n, k) * x[k];
+            g += weight_of(ex->gate_q, ex->gate_s, H, ex->group, n, k) * x[k];
+            u += weight_of(ex->up_q, ex->up_s, H, ex->group, n, k) * x[k];
         }
         tmp[n] = silu(g) * u;
     }
     for (int m = 0; m < H; ++m) {
         double acc = 0.0;
-        for (int n = 0; n < I; ++n) acc += oracle_weight(ex->down_q, ex->down_s, I, m, n) * tmp[n];
+        for (int n = 0; n < I; ++n)
+            acc += weight_of(ex->down_q, ex->down_s, I, ex->group, m, n) * tmp[n];
         y[m] = acc;
     }
 }

@@ -36,3 +36,27 @@ def swiglu_mlp(ex, x):
     u = x @ wu.T
     h = g / (1.0 + np.exp(-g)) * u
     return h @ wd.T
+
+
+def dequant_rows(q, s_bits):
+    """Per-row int4: [rows][K/2] uint8 + [rows][1] bf16 bits -> [rows][K]."""
+    q = np.asarray(q, dtype=np.uint8)
+    lo = (q & 0x0F).astype(np.int64)
+    hi = (q >> 4).astype(np.int64)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    codes = np.empty((q.shape[0], q.shape[1] * 2), dtype=np.float64)
+    codes[:, 0::2] = lo
+    codes[:, 1::2] = hi
+    return codes * bf16_bits_to_f64(np.asarray(s_bits).reshape(-1, 1))
+
+
+def swiglu_mlp_rows(ex, x):
+    """Dense SwiGLU MLP of a per-row int4 expert, numpy matmuls."""
+    wg = dequant_rows(ex["gate_q"], ex["gate_s"])
+    wu = dequant_rows(ex["up_q"], ex["up_s"])
+    wd = dequant_rows(ex["down_q"], ex["down_s"])
+    g = x @ wg.T
+    u = x @ wu.T
+    h = g / (1.0 + np.exp(-g)) * u
+    return h @ wd.T
