@@ -60,6 +60,7 @@ WORKLOADS = {
                           "T=64, per-layer Zipf-1.1 routing, x_(l+1) = x_l + MoE_l(x_l) in bf16"),
 }
 STACK_LAYERS = 16
+PREFETCH_BYTES = 96 << 20  # L2 budget of the stack's lookahead prefetch (--prefetch-mb)
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
@@ -387,45 +388,83 @@ def run_stack(args, rank, world, local, with_cpu=True):
         flush_buf.sum()
         fence_buf.zero_()
 
-    def step(i, x0, out_last=None):
+    # Router-lookahead L2 prefetch: while layer l runs, a side stream
+    # prefetches the experts layer l + 1 used in the previous step (the
+    # prediction), whole experts in the order layer l + 1 streams them, up to
+    # PREFETCH_BYTES.  Routings are double-buffered by step parity; the main
+    # stream joins the side stream at the end of every step.
+    side = torch.cuda.Stream(dev)
+    idx_bufs = [[torch.zeros(T, k, dtype=torch.int32, device=dev) for _ in range(L)]
+                for _ in range(2)]
+    starts = [torch.cuda.Event() for _ in range(L)]
+    side_done = torch.cuda.Event()
+
+    def step(i, x0, out_last=None, prefetch=False):
         x = x0
+        cur, prev = idx_bufs[i % 2], idx_bufs[(i - 1) % 2]
         for l in range(L):
+            if prefetch and i > 0 and l + 1 < L:
+                starts[l].record(stream)
+                side.wait_event(starts[l])
+                c.coli_moe_prefetch(layers[l + 1].handle, T, k, prev[l + 1], PREFETCH_BYTES,
+                                    None, side)
             out = acts[l] if (l < L - 1 or out_last is None) else out_last
             c.coli_moe_layer(layers[l].handle, T, x, lgs[l][i], None, x, out, c.COLI_OUT_BF16,
-                             None, None, ws, stream)
+                             cur[l], None, ws, stream)
             x = out
+        if prefetch:
+            side_done.record(side)
+            stream.wait_event(side_done)
         return x
 
     for i in range(args.warmup):
-        step(i, xs[i])
+        step(i, xs[i], prefetch=(i % 2 == 1))
         flush_l2()
     torch.cuda.synchronize(dev)
     if c.coli_moe_get_status(ws) != c.COLI_OK:
         raise RuntimeError("device status after warm-up: " + c.status_string(c.coli_moe_get_status(ws)))
-    uniq = [[len(set(torch.topk(lgs[l][i], k, dim=1).indices.flatten().tolist()))
-             for l in range(L)] for i in range(args.warmup, n)]
+    sets = [[set(torch.topk(lgs[l][i], k, dim=1).indices.flatten().tolist()) for l in range(L)]
+            for i in range(n)]
+    uniq = [[len(sets[i][l]) for l in range(L)] for i in range(args.warmup, n)]
+
+    def timed(prefetch):
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for j in range(args.steps):
+            ev[j][0].record(stream)
+            step(args.warmup + j, xs[args.warmup + j], prefetch=prefetch)
+            ev[j][1].record(stream)
+            flush_l2()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
 
     sampler = ClockSampler(dev.index) if rank == 0 else None
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for j in range(args.steps):
-        ev[j][0].record(stream)
-        step(args.warmup + j, xs[args.warmup + j])
-        ev[j][1].record(stream)
-        flush_l2()
-    torch.cuda.synchronize(dev)
-    barrier(world)
+    total_ms = timed(True)
     clocks = sampler.stop() if sampler else None
-    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    off_ms = timed(False)
     if c.coli_moe_get_status(ws) != c.COLI_OK:
         raise RuntimeError("device status: " + c.status_string(c.coli_moe_get_status(ws)))
+    # realised prediction: the share of layer l+1's experts (l + 1 >= 1) that
+    # the previous step had used, and of the experts actually prefetched
+    # (whole experts within the budget, ascending) the share that was used
+    per_expert = expert_bytes(H, I)
+    n_pf = max(0, PREFETCH_BYTES // per_expert - n_sh)
+    hit_all, hit_pf = [], []
+    for i in range(args.warmup, n):
+        for l in range(1, L):
+            act, pred = sets[i][l], sets[i - 1][l]
+            hit_all.append(len(act & pred) / len(act))
+            pf = sorted(pred)[:n_pf]
+            if pf:
+                hit_pf.append(len(act & set(pf)) / len(pf))
 
     torch.cuda.synchronize(dev)
     c.coli_moe_profile_enable(True)
     for j in range(args.steps):
-        step(args.warmup + j, xs[args.warmup + j])
+        step(args.warmup + j, xs[args.warmup + j], prefetch=True)
         flush_l2()
     torch.cuda.synchronize(dev)
     c.coli_moe_profile_enable(False)
@@ -443,7 +482,7 @@ def run_stack(args, rank, world, local, with_cpu=True):
     for j in range(args.steps):
         ev2[j][0].record(stream)
         x_dev.copy_(x_host[j], non_blocking=True)
-        step(args.warmup + j, x_dev, out_last=out_dev)
+        step(args.warmup + j, x_dev, out_last=out_dev, prefetch=True)
         out_host[j].copy_(out_dev, non_blocking=True)
         ev2[j][1].record(stream)
         flush_l2()
@@ -495,10 +534,16 @@ def run_stack(args, rank, world, local, with_cpu=True):
                      "algorithmic_bytes_per_launch": k_bytes, "avg_launch_ms": k_ms},
         "phase_ms_per_layer_call": {"before": phase_ms[0] / max(n_calls, 1), "main": k_ms,
                                     "after": phase_ms[2] / max(n_calls, 1)},
+        "l2_prefetch": {"budget_bytes": PREFETCH_BYTES, "experts_per_layer": n_pf + n_sh,
+                        "ms_per_step_on": total_ms / args.steps,
+                        "ms_per_step_off": off_ms / args.steps,
+                        "predicted_share_of_next_layer_experts": statistics.mean(hit_all),
+                        "prefetched_experts_used_share": statistics.mean(hit_pf) if hit_pf
+                        else None},
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
-        "gpu_launches": (4 if T * k < E else 6) * L * args.steps,
+        "gpu_launches": ((4 if T * k < E else 6) * L + (L - 1)) * args.steps,
         "clocks": clocks,
     }
     return line
@@ -684,6 +729,8 @@ def main():
                     help="measure one workload alone (default: decode as the headline line, "
                          "the others attached under \"workloads\")")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefetch-mb", type=int, default=None,
+                    help="L2 budget (MiB) of the stack's router-lookahead prefetch")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's tokens per step (small profiler cases)")
     ap.add_argument("--routed-experts", type=int, default=GLM["E"],
@@ -693,6 +740,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     GLM["E"] = args.routed_experts
+    if args.prefetch_mb is not None:
+        global PREFETCH_BYTES
+        PREFETCH_BYTES = args.prefetch_mb << 20
     if args.tokens > 0:
         name = args.workload or "decode"
         T0, kind, desc = WORKLOADS[name]

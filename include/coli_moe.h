@@ -40,6 +40,11 @@
  *   down_s       : bf16  [H][I/64]
  *   A code is a two's-complement nibble q in [-8, 7]; the LOW nibble of byte b
  *   is element 2b, the HIGH nibble element 2b+1; W[n][k] = q[n][k] * s[n][k/64].
+ * Per-row int4 (group_size COLI_GROUP_PER_ROW), the format of the older
+ * GLM-5.2 mirror ("ssnai.com/JustVugg_colibri.html", decision guide;
+ * "yunpan.plus/t/30351-1-1", capability four: gs64 against per-row int4):
+ * the same codes, one scale per row, W[n][k] = q[n][k] * s[n]:
+ *   gate_s, up_s : bf16  [I][1]     down_s : bf16  [H][1]
  *
  * Conventions for every call:
  *   - all tensor arguments are DEVICE pointers owned by the caller, row-major
@@ -100,13 +105,15 @@ typedef struct {
     int32_t inter;              /* I, multiple of 128, at most 12288 */
     int32_t n_routed;           /* E, 1..1024 */
     int32_t top_k;              /* k, 1..min(E, 32) */
-    int32_t group_size;         /* must be 64 */
+    int32_t group_size;         /* 64 (gs64) or COLI_GROUP_PER_ROW */
     int32_t n_shared;           /* shared experts, 0..4 */
     const coli_expert *experts; /* host array, n_routed + n_shared entries */
     int32_t prefill_min_tokens; /* T*k/E at or above which the tensor-core
                                    grouped GEMM is used; 0 = library default
                                    (1: every call with T*k >= E) */
 } coli_moe_desc;
+
+#define COLI_GROUP_PER_ROW 0 /* group_size of the per-row int4 format */
 
 typedef struct coli_moe coli_moe; /* opaque: device copy of the expert table */
 
@@ -232,6 +239,23 @@ coli_status coli_moe_layer_noalloc(const coli_moe_desc *desc, int32_t T, const v
 coli_status coli_moe_combine_rows(int32_t T, int32_t k, int32_t H, const float *rows,
                                   const float *shared, const void *residual, void *out,
                                   coli_out_dtype out_dtype, void *stream);
+
+/* Router-lookahead prefetch into L2 (the pages' one-layer-ahead prefetch,
+ * "yunpan.plus/t/30351-1-1", capabilities one and two, PILOT=1, with HBM ->
+ * L2 in place of disk -> RAM): issue L2 prefetches of the weights of the
+ * experts a routing names, in the order a layer call of handle `h` streams
+ * them (shared experts first, then routed experts by ascending index), whole
+ * experts only, until `max_bytes` would be exceeded.  Meant to run on a
+ * second stream while the previous layer computes, with the previous step's
+ * routing of `h`'s layer as the prediction.  Nothing is written; the layer
+ * call's results do not depend on it.
+ *   topk_idx [T][k] int32 device: the predicted routing
+ *   ws       nullable; if given (at least COLI_WS_HEADER_BYTES, 256-byte
+ *            aligned), an index outside [0, E) is recorded in its status word
+ * Errors: INVALID_ARG (NULL handle, T < 0, k outside [1, E]), SHAPE, ALIGN,
+ * WORKSPACE. */
+coli_status coli_moe_prefetch(const coli_moe *h, int32_t T, int32_t k, const int32_t *topk_idx,
+                              size_t max_bytes, void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronise `stream` and return the workspace's device status word
  * (COLI_OK, COLI_ERR_BAD_INDEX or COLI_ERR_TIMEOUT), or COLI_ERR_CUDA if the

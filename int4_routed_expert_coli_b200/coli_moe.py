@@ -32,10 +32,12 @@ COLI_OUT_F32 = 0
 COLI_WS_LOGITS_OFFSET = 16384  # router logits left in the workspace by coli_moe_layer
 COLI_WS_HEADER_BYTES = 16384
 COLI_OUT_BF16 = 1
+COLI_GROUP_PER_ROW = 0  # coli_moe_desc.group_size of the per-row int4 format
 
 EXPORTS = ("coli_moe_create", "coli_moe_destroy", "coli_moe_workspace_size",
            "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union", "coli_moe_ffn",
            "coli_moe_layer", "coli_moe_layer_noalloc", "coli_moe_combine_rows",
+           "coli_moe_prefetch",
            "coli_moe_get_status",
            "coli_moe_debug_inject",
            "coli_moe_profile_enable",
@@ -87,6 +89,8 @@ def _load():
     L.coli_moe_layer_noalloc.restype = ctypes.c_int
     L.coli_moe_combine_rows.argtypes = [i32, i32, i32, P, P, P, P, ctypes.c_int, P]
     L.coli_moe_combine_rows.restype = ctypes.c_int
+    L.coli_moe_prefetch.argtypes = [P, i32, i32, P, sz, P, sz, P]
+    L.coli_moe_prefetch.restype = ctypes.c_int
     L.coli_moe_get_status.argtypes = [P, P]
     L.coli_moe_get_status.restype = ctypes.c_int
     L.coli_moe_debug_inject.argtypes = [i32]
@@ -180,6 +184,14 @@ def coli_moe_combine_rows(T, k, H, rows, shared, residual, out, out_dtype, strea
     return _check(s, "coli_moe_combine_rows", raise_on_error)
 
 
+def coli_moe_prefetch(handle, T, k, topk_idx, max_bytes, ws=None, stream=None,
+                      raise_on_error=True):
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    s = lib.coli_moe_prefetch(handle, T, k, _ptr(topk_idx), int(max_bytes), _ptr(ws), ws_bytes,
+                              _stream(stream))
+    return _check(s, "coli_moe_prefetch", raise_on_error)
+
+
 def coli_moe_workspace_clear(ws, stream=None, raise_on_error=True):
     s = lib.coli_moe_workspace_clear(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     return _check(s, "coli_moe_workspace_clear", raise_on_error)
@@ -219,6 +231,8 @@ class MoELayer:
 
     def __init__(self, bank, n_routed: int, top_k: int, n_shared: int = 1,
                  prefill_min_tokens: int = 0):
+        """`bank.per_row` selects the per-row int4 format (group_size
+        COLI_GROUP_PER_ROW) instead of gs64."""
         if bank.n != n_routed + n_shared:
             raise ValueError("bank holds a different number of experts")
         self.bank = bank
@@ -228,7 +242,9 @@ class MoELayer:
             for name in ("gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s"):
                 t = getattr(bank, name)[e]
                 setattr(tab[e], name, t.data_ptr())
-        desc = CDesc(bank.hidden, bank.inter, n_routed, top_k, 64, n_shared, tab, prefill_min_tokens)
+        group = COLI_GROUP_PER_ROW if getattr(bank, "per_row", False) else 64
+        desc = CDesc(bank.hidden, bank.inter, n_routed, top_k, group, n_shared, tab,
+                     prefill_min_tokens)
         self._table = tab
         self.desc = desc
         h = ctypes.c_void_p()

@@ -87,6 +87,7 @@ coli::FfnArgs make_args(const coli_moe* h, int32_t T, const void* x, const float
     a.residual = residual;
     a.out = out;
     a.out_bf16 = od == COLI_OUT_BF16;
+    a.per_row = h->per_row;
     a.status = at<int>(ws, 0);
     a.withhold_item = -1;
     return a;
@@ -235,7 +236,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (!out) return COLI_ERR_INVALID_ARG;
     *out = nullptr;
     if (!d || !d->experts) return COLI_ERR_INVALID_ARG;
-    if (d->group_size != kGroup) return COLI_ERR_SHAPE;
+    if (d->group_size != kGroup && d->group_size != COLI_GROUP_PER_ROW) return COLI_ERR_SHAPE;
     if (d->hidden <= 0 || d->inter <= 0 || d->hidden % 128 || d->inter % 128) return COLI_ERR_SHAPE;
     if (d->n_routed < 1 || d->n_routed > coli::kMaxExperts) return COLI_ERR_SHAPE;
     if (d->top_k < 1 || d->top_k > d->n_routed || d->top_k > coli::kMaxTopK) return COLI_ERR_SHAPE;
@@ -269,6 +270,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     h->k = d->top_k;
     h->n_shared = d->n_shared;
     h->prefill_min = d->prefill_min_tokens;
+    h->per_row = d->group_size == COLI_GROUP_PER_ROW;
     h->num_sms = sms;
     h->d_experts = nullptr;
     h->d_wmaps = nullptr;
@@ -296,7 +298,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (err == cudaSuccess && h->d_wmaps &&
         coli::decode_supported(h->H, h->I, 1, h->E, h->k, h->n_shared, h->num_sms) &&
         coli::decode_coresident(h->H, h->I, h->E, h->k, h->n_shared, h->num_sms) &&
-        coli::build_decode_maps(host, n, h->H, h->I, &h->d_dmaps) != cudaSuccess) {
+        coli::build_decode_maps(host, n, h->H, h->I, h->per_row, &h->d_dmaps) != cudaSuccess) {
         h->d_dmaps = nullptr;  // the fused decode path is an optimisation: go without it
         cudaGetLastError();
     }

@@ -31,10 +31,13 @@ struct DevExpert {
     const uint8_t* gate_q;   // [I][H/2]
     const uint8_t* up_q;     // [I][H/2]
     const uint8_t* down_q;   // [H][I/2]
-    const uint16_t* gate_s;  // [I][H/64] bf16
-    const uint16_t* up_s;    // [I][H/64] bf16
-    const uint16_t* down_s;  // [H][I/64] bf16
+    const uint16_t* gate_s;  // [I][H/64] bf16 (per-row format: [I][1])
+    const uint16_t* up_s;    // [I][H/64] bf16 (per-row format: [I][1])
+    const uint16_t* down_s;  // [H][I/64] bf16 (per-row format: [H][1])
 };
+
+// Scale columns of a row of K codes: K / 64 (gs64) or 1 (per-row).
+__host__ __device__ inline int scale_cols(int K, int per_row) { return per_row ? 1 : K / kGroup; }
 
 // Byte offsets of the workspace regions for a call with T tokens.
 struct WsLayout {
@@ -104,6 +107,7 @@ struct FfnArgs {
     const void* residual;      // [T][H] nullable
     void* out;                 // [T][H]
     int out_bf16;
+    int per_row;               // scales: one per row instead of one per 64 codes
     int* status;
     int withhold_item;         // test hook: producer never fills this item (-1 = off)
 };

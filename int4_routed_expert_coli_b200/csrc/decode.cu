@@ -98,25 +98,33 @@ __host__ __device__ inline int dn_segs_for(int row_bytes) {
 struct Layout {
     int gu_segs, dn_segs;       // 128-byte chunks per staged code row
     int gGp, dGp;               // padded scale row lengths (bf16 elements)
+    int gsr, gsg, dsr, dsg;     // staged scale (row, group) strides in bytes, gate/up and down
     int gu_op, gu_sc, gu_tx;    // gate/up item: code copy, scale copy, bytes per stage
     int dn_op, dn_sc;           // down tile: code copy, scale copy
     int stage_bytes;
     int red_off, corr_off, route_off, table_off, cnt_off, stage_off, smem;
 };
 
-__host__ __device__ inline Layout make_layout(int H, int I, int max_slots) {
+// per_row: one scale per row (staged as the item's rows' scales, 2 bytes
+// each, every group reading its row's one scale).
+__host__ __device__ inline Layout make_layout(int H, int I, int max_slots, int per_row) {
     Layout L;
     L.gu_segs = gu_segs_for(H / 2);
     L.dn_segs = dn_segs_for(I / 2);
     // every consumer warp owns kMaxGW (kMaxDW) consecutive groups; the groups
-    // past the end read zero scales from the padding columns
+    // past the end read zero scales from the padding columns (gs64), or the
+    // row's scale times a zero activation fragment (per-row)
     L.gGp = padded_groups(kCW * kMaxGW > H / kGroup ? kCW * kMaxGW : H / kGroup);
     L.dGp = padded_groups(kCW * kMaxDW > I / kGroup ? kCW * kMaxDW : I / kGroup);
+    L.gsr = per_row ? 2 : L.gGp * 2;
+    L.gsg = per_row ? 0 : 2;
+    L.dsr = per_row ? 2 : L.dGp * 2;
+    L.dsg = per_row ? 0 : 2;
     L.gu_op = kGuRows * L.gu_segs * 128;
-    L.gu_sc = kGuRows * L.gGp * 2;
+    L.gu_sc = kGuRows * L.gsr;
     L.gu_tx = 2 * L.gu_op + 2 * L.gu_sc;
     L.dn_op = kDnRows * L.dn_segs * 128;
-    L.dn_sc = kDnRows * L.dGp * 2;
+    L.dn_sc = kDnRows * L.dsr;
     const int dn_stage = kMaxMT * (L.dn_op + L.dn_sc);
     L.stage_bytes = ((L.gu_tx > dn_stage ? L.gu_tx : dn_stage) + 1023) / 1024 * 1024;
     L.red_off = 1024;
@@ -583,7 +591,7 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t st = smem_addr(x.S.stage0) + stage * L.stage_bytes;
     if (valid) {
-        const uint32_t scA = st + 2 * L.gu_op + r * L.gGp * 2;
+        const uint32_t scA = st + 2 * L.gu_op + r * L.gsr;
         const uint32_t scB = scA + L.gu_sc;
         const uint32_t cor = smem_addr(x.S.corr) + c * 16;
         const Magic mg = magic();
@@ -604,8 +612,8 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
                 part[u][1] = cr.y;
                 part[u][2] = cr.z;
                 part[u][3] = cr.w;
-                fa[u] = __uint_as_float(lds_u16(scA + grp * 2) << 16);
-                fb[u] = __uint_as_float(lds_u16(scB + grp * 2) << 16);
+                fa[u] = __uint_as_float(lds_u16(scA + grp * L.gsg) << 16);
+                fb[u] = __uint_as_float(lds_u16(scB + grp * L.gsg) << 16);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the group
@@ -713,7 +721,7 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
         // accumulator that is never read.  Row r + 8 of a tile sits 8 staged
         // rows after row r.
         const int row8 = 8 * L.dn_segs * 128;
-        const uint32_t sc0 = st + kMaxMT * L.dn_op + r * L.dGp * 2;
+        const uint32_t sc0 = st + kMaxMT * L.dn_op + r * L.dsr;
 #pragma unroll
         for (int i = 0; i < kMaxDW; ++i) {
             const int gs = g_lo + i;
@@ -742,9 +750,9 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
             }
 #pragma unroll
             for (int m = 0; m < kMaxMT; ++m) {
-                const uint32_t sc = sc0 + m * L.dn_sc + gs * 2;
+                const uint32_t sc = sc0 + m * L.dn_sc + gs * L.dsg;
                 const float fa = __uint_as_float(lds_u16(sc) << 16);
-                const float fb = __uint_as_float(lds_u16(sc + 16 * L.dGp) << 16);
+                const float fb = __uint_as_float(lds_u16(sc + 8 * L.dsr) << 16);
                 acc[m][0] = fmaf(fa, part[m][0], acc[m][0]);
                 acc[m][1] = fmaf(fa, part[m][1], acc[m][1]);
                 acc[m][2] = fmaf(fb, part[m][2], acc[m][2]);
@@ -760,7 +768,7 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
 template <int NV>
 __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const DecodeArgs d) {
     const FfnArgs& a = d.f;
-    const Layout L = make_layout(a.H, a.I, d.max_slots);
+    const Layout L = make_layout(a.H, a.I, d.max_slots, a.per_row);
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned start, by pointer arithmetic on the shared array (so
     // the compiler keeps it a shared-memory pointer)
@@ -908,8 +916,15 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                 mbar_arrive_expect_tx(bar, L.gu_tx);
                 tma_load_3d(st, maps + 0, 0, 0, n0, bar, policy);
                 tma_load_3d(st + L.gu_op, maps + 1, 0, 0, n0, bar, policy);
-                tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
-                tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
+                if (a.per_row) {  // 8 rows' scales: 16 contiguous bytes per matrix
+                    const DevExpert& ex = a.experts[e];
+                    bulk_g2s_evict_first(st + 2 * L.gu_op, ex.gate_s + n0, L.gu_sc, bar, policy);
+                    bulk_g2s_evict_first(st + 2 * L.gu_op + L.gu_sc, ex.up_s + n0, L.gu_sc, bar,
+                                         policy);
+                } else {
+                    tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
+                    tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
+                }
             }
             // down stages carry item -1, which tells the consumers that gate/up
             // is over; without down work a single empty stage does
@@ -936,8 +951,12 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                     for (int m = 0; m < my_mt; ++m) {
                         const int m0 = (bm + m * G) * kDnRows;
                         tma_load_3d(st + m * L.dn_op, maps + 2, 0, 0, m0, bar, policy);
-                        tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0, bar,
-                                    policy);
+                        if (a.per_row)  // 16 rows' scales: 32 contiguous bytes
+                            bulk_g2s_evict_first(st + kMaxMT * L.dn_op + m * L.dn_sc,
+                                                 a.experts[e].down_s + m0, L.dn_sc, bar, policy);
+                        else
+                            tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0, bar,
+                                        policy);
                     }
                 }
             }
@@ -1189,7 +1208,7 @@ bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_s
     // the slot counters live between the two counter offsets of the header
     const int counters = (int)((kTileCntOffset - kSlotCntOffset) / 4);
     if (kSyncSlots + max_slots_for(E, k, T, n_shared) > counters) return false;
-    const Layout L = make_layout(H, I, max_slots_for(E, k, T, n_shared));
+    const Layout L = make_layout(H, I, max_slots_for(E, k, T, n_shared), 0);
     if (L.smem > kSmemLimitD) return false;
     if (H / kGroup > kCW * kMaxGW || I / kGroup > kCW * kMaxDW) return false;
     if (T * E > kRedFloats) return false;  // logits staged in the reduction buffers
@@ -1197,10 +1216,10 @@ bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_s
     return L.gu_segs <= 256 && L.dn_segs <= 256 && L.gGp <= 256 && L.dGp <= 256;
 }
 
-cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I,
+cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I, int per_row,
                               CUtensorMap** d_maps) {
     *d_maps = nullptr;
-    const Layout L = make_layout(H, I, 0);
+    const Layout L = make_layout(H, I, 0, 0);
     CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * kMaps];
     if (!maps) return cudaErrorMemoryAllocation;
     bool ok = true;
@@ -1208,12 +1227,14 @@ cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I
     for (int e = 0; e < n && ok; ++e) {
         const DevExpert& x = host_experts[e];
         CUtensorMap* m = maps + (size_t)e * kMaps;
+        // per-row scales are copied with 1-D bulk copies (their rows are 2
+        // bytes, below a tensor map's 16-byte stride): no scale maps
         ok = encode_tma(&m[0], x.gate_q, 3, I, H / 2, L.gu_segs, kGuRows) &&
              encode_tma(&m[1], x.up_q, 3, I, H / 2, L.gu_segs, kGuRows) &&
              encode_tma(&m[2], x.down_q, 3, H, I / 2, L.dn_segs, kDnRows) &&
-             encode_tma_rows_u16(&m[3], x.gate_s, I, gG, L.gGp, kGuRows) &&
-             encode_tma_rows_u16(&m[4], x.up_s, I, gG, L.gGp, kGuRows) &&
-             encode_tma_rows_u16(&m[5], x.down_s, H, dG, L.dGp, kDnRows);
+             (per_row || (encode_tma_rows_u16(&m[3], x.gate_s, I, gG, L.gGp, kGuRows) &&
+                          encode_tma_rows_u16(&m[4], x.up_s, I, gG, L.gGp, kGuRows) &&
+                          encode_tma_rows_u16(&m[5], x.down_s, H, dG, L.dGp, kDnRows)));
     }
     if (!ok) {
         delete[] maps;
@@ -1234,7 +1255,7 @@ cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I
 bool decode_coresident(int H, int I, int E, int k, int n_shared, int num_sms) {
     // the largest shared-memory footprint (8 tokens) of either template
     // instance a handle can launch (routing from logits, or a given union)
-    const Layout L = make_layout(H, I, max_slots_for(E, k, 8, n_shared));
+    const Layout L = make_layout(H, I, max_slots_for(E, k, 8, n_shared), 0);
     int per_sm = resident_per_sm<1>(L.smem);
     switch (nv_for(E)) {
         case 1: per_sm = std::min(per_sm, resident_per_sm<1>(L.smem)); break;
@@ -1257,7 +1278,7 @@ cudaError_t launch_decode_fused(const DecodeArgs& d0, int num_sms, cudaStream_t 
         return cudaErrorCooperativeLaunchTooLarge;
     }
     d.max_slots = max_slots_for(d.f.E, d.f.k, d.f.T, d.f.n_shared);
-    const Layout L = make_layout(d.f.H, d.f.I, d.max_slots);
+    const Layout L = make_layout(d.f.H, d.f.I, d.max_slots, d.f.per_row);
     const int blocks = num_sms;  // persistent: one CTA per SM, all resident
     d.f.withhold_item = take_withhold_item();
     profile_mark(1, st);

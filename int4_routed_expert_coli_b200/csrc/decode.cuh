@@ -27,9 +27,9 @@ struct DecodeArgs {
 // True when a call with T tokens can run the fused decode kernel on a GPU
 // with num_sms SMs.
 bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_sms);
-// Tensor maps of every expert's packed code matrices (3-D, swizzled) and
-// scale matrices (2-D, padded rows).
-cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I,
+// Tensor maps of every expert's packed code matrices (3-D, swizzled) and,
+// for gs64 (per_row == 0), scale matrices (2-D, padded rows).
+cudaError_t build_decode_maps(const DevExpert* host_experts, int n, int H, int I, int per_row,
                               CUtensorMap** d_maps);
 // True when at least one CTA of the kernel fits on an SM (so a grid of one
 // CTA per SM can be resident at once).

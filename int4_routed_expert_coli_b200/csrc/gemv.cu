@@ -132,22 +132,26 @@ __device__ __forceinline__ void load_b(uint32_t bw[8], const __half* p) {
 // Geometry of one kernel kind.
 struct Geo {
     int K;           // reduction length (H for gate/up, I for down)
-    int G;           // scale groups per row, K / 64
+    int G;           // 64-groups per row, K / 64 (offset sums are per group)
+    int SG;          // scale columns per row: G (gs64) or 1 (per-row format)
+    int gs;          // scale column step per group: 1 (gs64) or 0 (per-row)
     int rows;        // staged rows per item: 16 * MT
     int row_stride;  // bytes per staged row: K/2 + 32
-    int scale_off;   // offset of the scale block ([rows][G] bf16) in a stage
+    int scale_off;   // offset of the scale block ([rows][SG] bf16) in a stage
     int stage_bytes;
     int tiles;       // items per expert
 };
 
-inline Geo make_geo(int K, int rows, int tiles) {
+inline Geo make_geo(int K, int rows, int tiles, int per_row) {
     Geo g;
     g.K = K;
     g.G = K / kGroup;
+    g.SG = scale_cols(K, per_row);
+    g.gs = per_row ? 0 : 1;
     g.rows = rows;
     g.row_stride = K / 2 + 32;
     g.scale_off = rows * g.row_stride;
-    g.stage_bytes = g.scale_off + (int)align_up((size_t)rows * g.G * 2, 16);
+    g.stage_bytes = g.scale_off + (int)align_up((size_t)rows * g.SG * 2, 16);
     g.tiles = tiles;
     return g;
 }
@@ -274,7 +278,7 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
             const DevExpert ex = a.experts[sl.e];
             const int tile = (int)(item % g.tiles);
             if (lane == 0)
-                mbar_arrive_expect_tx(&full[stage], g.rows * row_bytes + g.rows * g.G * 2);
+                mbar_arrive_expect_tx(&full[stage], g.rows * row_bytes + g.rows * g.SG * 2);
             __syncwarp();
             if constexpr (kGU) {
                 // rows 0..7: gate rows n0.., rows 8..15: up rows n0..; scales likewise
@@ -285,9 +289,9 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
                     bulk_g2s_evict_first(st + lane * g.row_stride, src, row_bytes, &full[stage],
                                          policy);
                 } else if (lane < 18) {
-                    const uint16_t* src = (lane == 16 ? ex.gate_s : ex.up_s) + (int64_t)n0 * g.G;
-                    bulk_g2s_evict_first(st + g.scale_off + (lane - 16) * 8 * g.G * 2, src,
-                                         8 * g.G * 2, &full[stage], policy);
+                    const uint16_t* src = (lane == 16 ? ex.gate_s : ex.up_s) + (int64_t)n0 * g.SG;
+                    bulk_g2s_evict_first(st + g.scale_off + (lane - 16) * 8 * g.SG * 2, src,
+                                         8 * g.SG * 2, &full[stage], policy);
                 }
             } else {
                 const int m0 = tile * g.rows;
@@ -296,8 +300,8 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
                                          ex.down_q + (int64_t)(m0 + i) * row_bytes, row_bytes,
                                          &full[stage], policy);
                 if (lane == 0)
-                    bulk_g2s_evict_first(st + g.scale_off, ex.down_s + (int64_t)m0 * g.G,
-                                         g.rows * g.G * 2, &full[stage], policy);
+                    bulk_g2s_evict_first(st + g.scale_off, ex.down_s + (int64_t)m0 * g.SG,
+                                         g.rows * g.SG * 2, &full[stage], policy);
             }
         }
         if (aborted) {
@@ -378,16 +382,16 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
                 if (ok) {
                     const uint8_t* rowA = st + r * g.row_stride + c * 8;
                     const uint8_t* rowB = st + (8 + r) * g.row_stride + c * 8;
-                    const uint16_t* scA = scales + r * g.G;
-                    const uint16_t* scB = scales + (8 + r) * g.G;
+                    const uint16_t* scA = scales + r * g.SG;
+                    const uint16_t* scB = scales + (8 + r) * g.SG;
 #pragma unroll
                     for (int i = 0; i < KW; ++i) {
                         const int grp = g_lo + i;
                         if (grp >= g_hi) break;
                         const uint2 wa = *reinterpret_cast<const uint2*>(rowA + grp * 32);
                         const uint2 wb = *reinterpret_cast<const uint2*>(rowB + grp * 32);
-                        const float fa = bf16_bits_to_float(scA[grp]);
-                        const float fb = bf16_bits_to_float(scB[grp]);
+                        const float fa = bf16_bits_to_float(scA[grp * g.gs]);
+                        const float fb = bf16_bits_to_float(scB[grp * g.gs]);
                         const float cr0 = corr_s[(2 * c) * g.G + grp];
                         const float cr1 = corr_s[(2 * c + 1) * g.G + grp];
                         float part[4];
@@ -446,8 +450,10 @@ stream_ffn_kernel(const FfnArgs a, const Geo g, int stages) {
                                 const uint8_t* rowB = st + (mt * 16 + 8 + r) * g.row_stride + c * 8;
                                 const uint2 wa = *reinterpret_cast<const uint2*>(rowA + grp * 32);
                                 const uint2 wb = *reinterpret_cast<const uint2*>(rowB + grp * 32);
-                                const float fa = bf16_bits_to_float(scales[(mt * 16 + r) * g.G + grp]);
-                                const float fb = bf16_bits_to_float(scales[(mt * 16 + 8 + r) * g.G + grp]);
+                                const float fa = bf16_bits_to_float(
+                                    scales[(mt * 16 + r) * g.SG + grp * g.gs]);
+                                const float fb = bf16_bits_to_float(
+                                    scales[(mt * 16 + 8 + r) * g.SG + grp * g.gs]);
                                 float part[4];
                                 group_partial<!kGU>(part, wa, wb, bw);
                                 acc[mt][nt][0] = fmaf(fa, part[0] - c0, acc[mt][nt][0]);
@@ -691,7 +697,7 @@ cudaError_t launch_combine_impl(const FfnArgs& a, int num_sms, cudaStream_t st) 
 // gate/up launch: T <= 8 uses the register-resident activation path when a
 // warp's share of the groups fits KW.
 cudaError_t launch_gateup(const FfnArgs& a, int num_sms, cudaStream_t st) {
-    const Geo g = make_geo(a.H, 16, a.I / 8);
+    const Geo g = make_geo(a.H, 16, a.I / 8, a.per_row);
     const int per_warp = (g.G + kConsumerWarps - 1) / kConsumerWarps;
     if (a.T <= 8) {
         if (per_warp <= 2) return launch_stream<true, 1, 1, true, 2>(a, g, num_sms, st);
@@ -704,8 +710,11 @@ cudaError_t launch_gateup(const FfnArgs& a, int num_sms, cudaStream_t st) {
 }
 
 cudaError_t launch_down(const FfnArgs& a, int num_sms, cudaStream_t st) {
-    if (a.T <= 8) return launch_stream<false, 2, 1, false, 1>(a, make_geo(a.I, 32, a.H / 32), num_sms, st);
-    return launch_stream<false, 1, 2, false, 1>(a, make_geo(a.I, 16, a.H / 16), num_sms, st);
+    if (a.T <= 8)
+        return launch_stream<false, 2, 1, false, 1>(a, make_geo(a.I, 32, a.H / 32, a.per_row),
+                                                   num_sms, st);
+    return launch_stream<false, 1, 2, false, 1>(a, make_geo(a.I, 16, a.H / 16, a.per_row),
+                                               num_sms, st);
 }
 
 }  // namespace
@@ -715,7 +724,7 @@ cudaError_t launch_combine(const FfnArgs& a, int num_sms, cudaStream_t st) {
 }
 
 bool stream_shapes_fit(int H, int I) {
-    const Geo g1 = make_geo(H, 16, I / 8), g2 = make_geo(I, 32, H / 32);
+    const Geo g1 = make_geo(H, 16, I / 8, 0), g2 = make_geo(I, 32, H / 32, 0);
     return fixed_smem_bytes(1, 2, true, g1.G) + 2 * g1.stage_bytes <= kSmemLimit &&
            fixed_smem_bytes(2, 2, false, g2.G) + 2 * g2.stage_bytes <= kSmemLimit;
 }

@@ -8,6 +8,7 @@
 struct coli_moe {
     int device;
     int H, I, E, k, n_shared, prefill_min;
+    int per_row;                 // one scale per row (COLI_GROUP_PER_ROW) instead of gs64
     int num_sms;
     coli::DevExpert* d_experts;  // device table, E + n_shared entries
     CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)

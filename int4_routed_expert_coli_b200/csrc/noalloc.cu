@@ -79,7 +79,7 @@ extern "C" coli_status coli_moe_layer_noalloc(const coli_moe_desc* d, int32_t T,
                                               int32_t* status_out, void* stream) {
     // the descriptor checks coli_moe_create makes, without its allocations
     if (!d || !d->experts || T < 0) return COLI_ERR_INVALID_ARG;
-    if (d->group_size != coli::kGroup) return COLI_ERR_SHAPE;
+    if (d->group_size != coli::kGroup && d->group_size != COLI_GROUP_PER_ROW) return COLI_ERR_SHAPE;
     if (d->hidden <= 0 || d->inter <= 0 || d->hidden % 128 || d->inter % 128) return COLI_ERR_SHAPE;
     if (d->hidden > 12288 || d->inter > 12288 || !coli::stream_shapes_fit(d->hidden, d->inter))
         return COLI_ERR_SHAPE;
@@ -141,6 +141,7 @@ extern "C" coli_status coli_moe_layer_noalloc(const coli_moe_desc* d, int32_t T,
     h.k = d->top_k;
     h.n_shared = d->n_shared;
     h.prefill_min = d->prefill_min_tokens;
+    h.per_row = d->group_size == COLI_GROUP_PER_ROW;
     h.num_sms = s->num_sms;
     h.d_experts = reinterpret_cast<coli::DevExpert*>(base);
     h.d_wmaps = nullptr;

@@ -435,16 +435,19 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
             // f0 + row and f0 + 128 + row (the latter past H in a ragged last
             // tile: scale 0, and its codes are zero-filled)
             const int f0 = ti.m_tile * kFeat;
-            const int64_t srow = (int64_t)(f0 + row) * G;
+            const int SG = scale_cols(K, a.per_row);  // scale columns per row
+            const int gstep = a.per_row ? 0 : 1;      // scale column step per K-block
+            const int64_t srow = (int64_t)(f0 + row) * SG;
             const bool has1 = kGU || f0 + BM < a.H;
             const uint16_t* sc_b0 = (kGU ? ex.gate_s : ex.down_s) + srow;
-            const uint16_t* sc_b1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * G;
+            const uint16_t* sc_b1 = kGU ? ex.up_s + srow : ex.down_s + srow + (int64_t)BM * SG;
             // Scales: a row's scales are contiguous, so where a row of them
             // is a whole number of 16-byte chunks (G % 8 == 0) a thread
             // loads 8 at a time, one chunk (8 K-blocks) ahead, and the load
             // latency hides behind 8 K-blocks of work; otherwise one scale
-            // per K-block, one ahead.
-            const bool vec = (G & 7) == 0;
+            // per K-block, one ahead; in the per-row format the row's one
+            // scale, loaded once.
+            const bool vec = !a.per_row && (G & 7) == 0;
             const uint16_t* scp[kMyBlocks];
             bool live[kMyBlocks];
             uint4 chunk[kMyBlocks], chunk_nxt[kMyBlocks];
@@ -477,7 +480,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                         cur[m] = (uint16_t)((sub & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
                     } else {
                         cur[m] = nxt[m];
-                        if (kb + 1 < KB && live[m]) nxt[m] = __ldg(scp[m] + kb + 1);
+                        if (kb + 1 < KB && live[m] && gstep) nxt[m] = __ldg(scp[m] + kb + 1);
                     }
                 }
                 const int s = rs.i, as = ra.i;
@@ -826,6 +829,7 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
     a.wmaps = wmaps;
     a.hbuf = f.hp;
     a.y = f.y;
+    a.per_row = f.per_row;
     a.status = f.status;
     // activation / h tiles as 128-, 64- and 32-row boxes
     CUtensorMap xmap[3], hmap[3];

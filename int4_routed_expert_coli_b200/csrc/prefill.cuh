@@ -17,6 +17,7 @@ struct GemmArgs {
     const CUtensorMap* wmaps;  // [experts][3] packed gate / up / down codes
     __half* hbuf;            // [S][I] SwiGLU output, operand order
     float* y;                // [S][H]
+    int per_row;             // scales: one per row instead of one per 64 codes
     int* status;
 };
 

@@ -39,7 +39,7 @@ def test_header_constants_match_binding():
     from int4_routed_expert_coli_b200 import coli_moe as c
     src = open(HEADER).read()
     for name in ("COLI_WS_LOGITS_OFFSET", "COLI_WS_HEADER_BYTES", "COLI_INJECT_WITHHOLD_STAGE",
-                 "COLI_INJECT_NOT_RESIDENT"):
+                 "COLI_INJECT_NOT_RESIDENT", "COLI_GROUP_PER_ROW"):
         m = re.search(r"#define\s+" + name + r"\s+(\d+)", src)
         assert m and int(m.group(1)) == getattr(c, name), name
     for name, val in re.findall(r"\b(COLI_(?:OK|ERR_\w+|OUT_\w+))\s*=\s*(\d+)", src):
