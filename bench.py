@@ -60,7 +60,11 @@ WORKLOADS = {
                           "T=64, per-layer Zipf-1.1 routing, x_(l+1) = x_l + MoE_l(x_l) in bf16"),
 }
 STACK_LAYERS = 16
-PREFETCH_BYTES = 96 << 20  # L2 budget of the stack's lookahead prefetch (--prefetch-mb)
+# L2 budget of the stack's lookahead prefetch (--prefetch-mb): the shared
+# expert (always used).  Measured with 0, 20 and 40 MiB: no budget made a step
+# faster (larger budgets slow it down), so the stack line's value is the step
+# with the prefetch off and the "on" time is reported beside it.
+PREFETCH_BYTES = 20 << 20
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
@@ -442,9 +446,9 @@ def run_stack(args, rank, world, local, with_cpu=True):
         return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
 
     sampler = ClockSampler(dev.index) if rank == 0 else None
-    total_ms = timed(True)
+    total_ms = timed(False)
     clocks = sampler.stop() if sampler else None
-    off_ms = timed(False)
+    on_ms = timed(True)
     if c.coli_moe_get_status(ws) != c.COLI_OK:
         raise RuntimeError("device status: " + c.status_string(c.coli_moe_get_status(ws)))
     # realised prediction: the share of layer l+1's experts (l + 1 >= 1) that
@@ -464,7 +468,7 @@ def run_stack(args, rank, world, local, with_cpu=True):
     torch.cuda.synchronize(dev)
     c.coli_moe_profile_enable(True)
     for j in range(args.steps):
-        step(args.warmup + j, xs[args.warmup + j], prefetch=True)
+        step(args.warmup + j, xs[args.warmup + j])
         flush_l2()
     torch.cuda.synchronize(dev)
     c.coli_moe_profile_enable(False)
@@ -482,7 +486,7 @@ def run_stack(args, rank, world, local, with_cpu=True):
     for j in range(args.steps):
         ev2[j][0].record(stream)
         x_dev.copy_(x_host[j], non_blocking=True)
-        step(args.warmup + j, x_dev, out_last=out_dev, prefetch=True)
+        step(args.warmup + j, x_dev, out_last=out_dev)
         out_host[j].copy_(out_dev, non_blocking=True)
         ev2[j][1].record(stream)
         flush_l2()
@@ -535,15 +539,15 @@ def run_stack(args, rank, world, local, with_cpu=True):
         "phase_ms_per_layer_call": {"before": phase_ms[0] / max(n_calls, 1), "main": k_ms,
                                     "after": phase_ms[2] / max(n_calls, 1)},
         "l2_prefetch": {"budget_bytes": PREFETCH_BYTES, "experts_per_layer": n_pf + n_sh,
-                        "ms_per_step_on": total_ms / args.steps,
-                        "ms_per_step_off": off_ms / args.steps,
+                        "ms_per_step_on": on_ms / args.steps,
+                        "ms_per_step_off": total_ms / args.steps,
                         "predicted_share_of_next_layer_experts": statistics.mean(hit_all),
                         "prefetched_experts_used_share": statistics.mean(hit_pf) if hit_pf
                         else None},
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
-        "gpu_launches": ((4 if T * k < E else 6) * L + (L - 1)) * args.steps,
+        "gpu_launches": (4 if T * k < E else 6) * L * args.steps,
         "clocks": clocks,
     }
     return line

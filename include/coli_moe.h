@@ -109,8 +109,13 @@ typedef struct {
     int32_t n_shared;           /* shared experts, 0..4 */
     const coli_expert *experts; /* host array, n_routed + n_shared entries */
     int32_t prefill_min_tokens; /* T*k/E at or above which the tensor-core
-                                   grouped GEMM is used; 0 = library default
-                                   (1: every call with T*k >= E) */
+                                   grouped GEMM is used; 0 = library default:
+                                   the grouped GEMM for every call the fused
+                                   decode kernel does not take (more than 8
+                                   tokens, T*k >= E, or a shape it does not
+                                   support); a positive value: calls with
+                                   T*k >= value * E, the streaming kernels for
+                                   the rest the fused kernel does not take */
 } coli_moe_desc;
 
 #define COLI_GROUP_PER_ROW 0 /* group_size of the per-row int4 format */
@@ -273,8 +278,9 @@ coli_status coli_moe_profile_enable(int32_t enable);
 coli_status coli_moe_profile_read(double *ms, int32_t *n_calls);
 
 /* Fault injection for tests (host-global, one thread).  With
- * COLI_INJECT_WITHHOLD_STAGE the next coli_moe_layer / coli_moe_ffn call's
- * gate/up kernel never fills one staged tile: its consumers' bounded wait
+ * COLI_INJECT_WITHHOLD_STAGE the next coli_moe_layer / coli_moe_ffn call that
+ * runs the fused decode kernel or the streaming kernels (not the grouped
+ * GEMM) never fills one staged gate/up tile: its consumers' bounded wait
  * (about one second) runs out, the kernel winds down without hanging or
  * faulting, and the status word reads COLI_ERR_TIMEOUT; the output of that
  * call is undefined and the context stays usable.  0 switches every hook

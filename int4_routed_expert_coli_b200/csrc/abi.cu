@@ -12,13 +12,13 @@
 #include "handle.cuh"
 #include "prefill.cuh"
 
-// Average routed tokens per expert (T*k/E) at or above which a call runs the
-// tensor-core grouped GEMM instead of the streaming dequant-GEMV (calls of up
-// to 8 tokens below it take the fused decode kernel).  Measured on the
-// GLM-5.2 shape with Zipf routing: at T = 32 (T*k/E = 1) the grouped GEMM
-// takes 1.10 ms against the streaming path's 1.51 ms, at T = 64 1.54 ms
-// against 2.32 ms.
-constexpr int kDefaultPrefillMin = 1;
+// Which kernels a call runs.  Up to 8 tokens with fewer routed pairs than
+// experts (T*k < E), the fused decode kernel; by default every other call the
+// tensor-core grouped GEMM.  Measured on the GLM-5.2 shape (Zipf routing):
+// at T = 16 the streaming dequant-GEMV takes 1.35 ms per call, at T = 32
+// 1.51 ms against the grouped GEMM's 1.10 ms, at T = 64 2.32 ms against
+// 1.54 ms.  A positive prefill_min_tokens keeps the older rule (grouped GEMM
+// from T*k >= prefill_min * E, streaming below it).
 
 namespace {
 
@@ -119,16 +119,21 @@ void profile_begin_call(cudaStream_t st) {
 
 void profile_end_call() { g_prof.open_call = -1; }
 
+// True when the fused decode kernel can take a call with T tokens.
+bool fused_ok(const coli_moe* h, int64_t T) {
+    return h->d_dmaps != nullptr && T * h->k < h->E &&
+           coli::decode_supported(h->H, h->I, (int)T, h->E, h->k, h->n_shared, h->num_sms);
+}
+
 // True when a call with T tokens runs the tensor-core grouped GEMM.
 bool use_prefill(const coli_moe* h, int64_t T) {
-    return h->d_wmaps != nullptr && T * h->k >= (int64_t)h->prefill_min * h->E;
+    if (h->d_wmaps == nullptr) return false;
+    if (h->prefill_min > 0) return T * h->k >= (int64_t)h->prefill_min * h->E;
+    return !fused_ok(h, T);
 }
 
 // True when a call with T tokens runs the fused decode kernel.
-bool use_fused(const coli_moe* h, int64_t T) {
-    return h->d_dmaps != nullptr && !use_prefill(h, T) &&
-           coli::decode_supported(h->H, h->I, (int)T, h->E, h->k, h->n_shared, h->num_sms);
-}
+bool use_fused(const coli_moe* h, int64_t T) { return fused_ok(h, T) && !use_prefill(h, T); }
 
 // The fused decode kernel: routing from `logits` (or the union in `a` when
 // logits is null), gate/up, down and combine in one launch.
@@ -275,7 +280,6 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     h->d_experts = nullptr;
     h->d_wmaps = nullptr;
     h->d_dmaps = nullptr;
-    if (h->prefill_min == 0) h->prefill_min = kDefaultPrefillMin;
     coli::DevExpert* host = static_cast<coli::DevExpert*>(std::malloc(sizeof(coli::DevExpert) * n));
     if (!host) {
         delete h;

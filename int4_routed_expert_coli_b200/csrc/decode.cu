@@ -765,8 +765,18 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
     return true;
 }
 
-template <int NV>
-__global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const DecodeArgs d) {
+// NV: logits per routing lane.  HC, IC, PR > 0 (PR >= 0): the layer's H, I
+// and scale format fixed at compile time (the GLM-5.2 shape), so every stride
+// of the shared-memory layout is a constant and the address arithmetic of the
+// inner loops folds into immediates; 0 (and PR = -1): taken from the call.
+template <int NV, int HC, int IC, int PR>
+__global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const DecodeArgs d0) {
+    DecodeArgs d = d0;
+    if constexpr (HC > 0) {
+        d.f.H = HC;
+        d.f.I = IC;
+    }
+    if constexpr (PR >= 0) d.f.per_row = PR;
     const FfnArgs& a = d.f;
     const Layout L = make_layout(a.H, a.I, d.max_slots, a.per_row);
     extern __shared__ uint8_t smem_raw[];
@@ -1149,10 +1159,10 @@ bool g_coop_with_pdl = true;
 // A cooperative launch: the runtime starts it only if every CTA of the grid
 // can be resident at once (cudaErrorCooperativeLaunchTooLarge otherwise),
 // which the CTAs' waits on one another need.
-template <int NV>
+template <int NV, int HC = 0, int IC = 0, int PR = -1>
 cudaError_t launch_nv(const DecodeArgs& d, int blocks, int smem, cudaStream_t st) {
-    cudaError_t err = cudaFuncSetAttribute(decode_fused_kernel<NV>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = decode_fused_kernel<NV, HC, IC, PR>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(blocks);
@@ -1166,28 +1176,31 @@ cudaError_t launch_nv(const DecodeArgs& d, int blocks, int smem, cudaStream_t st
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = g_coop_with_pdl ? 2 : 1;
-    err = cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+    err = cudaLaunchKernelEx(&cfg, kern, d);
     if (err != cudaSuccess && err != cudaErrorCooperativeLaunchTooLarge && g_coop_with_pdl) {
         cudaGetLastError();  // a refused configuration launched nothing
         g_coop_with_pdl = false;
         cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, decode_fused_kernel<NV>, d);
+        err = cudaLaunchKernelEx(&cfg, kern, d);
     }
     return err;
 }
 
 // Resident CTAs of the kernel instance per SM at `smem` bytes of shared memory.
-template <int NV>
+template <int NV, int HC = 0, int IC = 0, int PR = -1>
 int resident_per_sm(int smem) {
-    if (cudaFuncSetAttribute(decode_fused_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    auto kern = decode_fused_kernel<NV, HC, IC, PR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 0;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_fused_kernel<NV>, kThreadsD,
-                                                      smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreadsD, smem) != cudaSuccess)
         return 0;
     return n;
 }
+
+// The shape with a compile-time instance: GLM-5.2 (H 6144, I 2048), gs64.
+constexpr int kFixH = 6144, kFixI = 2048;
+bool fixed_shape(int H, int I, int per_row) { return H == kFixH && I == kFixI && !per_row; }
 
 int max_slots_for(int E, int k, int T, int n_shared) {
     return std::min(E, T * k) + n_shared;
@@ -1257,6 +1270,9 @@ bool decode_coresident(int H, int I, int E, int k, int n_shared, int num_sms) {
     // instance a handle can launch (routing from logits, or a given union)
     const Layout L = make_layout(H, I, max_slots_for(E, k, 8, n_shared), 0);
     int per_sm = resident_per_sm<1>(L.smem);
+    if (fixed_shape(H, I, 0))
+        per_sm = std::min(per_sm, std::min(resident_per_sm<1, kFixH, kFixI, 0>(L.smem),
+                                           resident_per_sm<8, kFixH, kFixI, 0>(L.smem)));
     switch (nv_for(E)) {
         case 1: per_sm = std::min(per_sm, resident_per_sm<1>(L.smem)); break;
         case 2: per_sm = std::min(per_sm, resident_per_sm<2>(L.smem)); break;
@@ -1283,11 +1299,18 @@ cudaError_t launch_decode_fused(const DecodeArgs& d0, int num_sms, cudaStream_t 
     d.f.withhold_item = take_withhold_item();
     profile_mark(1, st);
     cudaError_t err;
+    const bool fixed = fixed_shape(d.f.H, d.f.I, d.f.per_row);
     switch (d.logits ? nv_for(d.f.E) : 1) {
-        case 1: err = launch_nv<1>(d, blocks, L.smem, st); break;
+        case 1:
+            err = fixed ? launch_nv<1, kFixH, kFixI, 0>(d, blocks, L.smem, st)
+                        : launch_nv<1>(d, blocks, L.smem, st);
+            break;
         case 2: err = launch_nv<2>(d, blocks, L.smem, st); break;
         case 4: err = launch_nv<4>(d, blocks, L.smem, st); break;
-        case 8: err = launch_nv<8>(d, blocks, L.smem, st); break;
+        case 8:
+            err = fixed ? launch_nv<8, kFixH, kFixI, 0>(d, blocks, L.smem, st)
+                        : launch_nv<8>(d, blocks, L.smem, st);
+            break;
         case 16: err = launch_nv<16>(d, blocks, L.smem, st); break;
         default: err = launch_nv<32>(d, blocks, L.smem, st); break;
     }

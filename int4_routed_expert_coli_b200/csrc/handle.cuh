@@ -7,7 +7,8 @@
 
 struct coli_moe {
     int device;
-    int H, I, E, k, n_shared, prefill_min;
+    int H, I, E, k, n_shared;
+    int prefill_min;             // 0: grouped GEMM unless the fused decode kernel takes the call
     int per_row;                 // one scale per row (COLI_GROUP_PER_ROW) instead of gs64
     int num_sms;
     coli::DevExpert* d_experts;  // device table, E + n_shared entries

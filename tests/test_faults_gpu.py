@@ -13,10 +13,12 @@ pytestmark = [pytest.mark.gpu, requires_gpu]
 
 
 def test_withheld_stage_times_out_and_context_survives():
+    """The streaming kernels (forced: the tiny shape would take the grouped
+    GEMM by default)."""
     from int4_routed_expert_coli_b200 import coli_moe as c
     H, I, E, k, T = 256, 128, 16, 2, 4
     bank = synth.make_expert_bank(H, I, E + 1, seed=21, device="cuda")
-    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=1)
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=1, prefill_min_tokens=10 ** 6)
     x = synth.make_activations(T, H, seed=22, device="cuda")
     lg = synth.make_logits_normal(T, E, seed=23, device="cuda")
     ws = layer.workspace(T)
