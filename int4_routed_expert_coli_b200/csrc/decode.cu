@@ -28,10 +28,13 @@
 // chunks, 128-byte swizzle, so the consumers' fragment reads spread over the
 // banks) and 2-D copies of the scale rows (padded to 8 x odd columns).
 //
-// Arithmetic as in the streaming GEMV: raw fp16 unpack with the per-(token,
-// group) offset sum as the initial accumulator for gate/up, exact unpack for
-// down, m16n8k16 MMA with fp32 accumulation, gs64 scale applied to each
-// group's partial.  Eleven consumer warps split K; a gate/up item's partials
+// Arithmetic: raw fp16 unpack of the codes (1032 + q for even K, 1152 + 16 q
+// for odd K, whose activations enter divided by 16) with the per-(token,
+// group) offset sum of the activation operand as the MMA chain's initial
+// value: for gate/up the sums of x, for down the sums of the slot's h'
+// (stored with its odd elements divided by 16), computed from the h'
+// fragments with four MMAs per group; m16n8k16 MMA with fp32 accumulation,
+// the group's scale applied to each group's partial.  Eleven consumer warps split K; a gate/up item's partials
 // are summed through four reduction buffers, item j by warp j mod 11 two
 // items later (in warp order, so the sum does not depend on timing).
 //
@@ -159,16 +162,6 @@ __device__ __forceinline__ void unpack_raw_step(uint32_t w, int step, uint32_t& 
     const uint32_t v = step ? (w >> 8) : w;
     e = and_xor(v, mg.lo_mask, mg.lo_bias);
     o = and_xor(v, mg.hi_mask, mg.hi_bias);
-}
-
-// The same, exact: e = q_even, o = q_odd as fp16.
-__device__ __forceinline__ void unpack_exact_step(uint32_t w, int step, uint32_t& e, uint32_t& o,
-                                                  const Magic& mg) {
-    uint32_t re, ro;
-    unpack_raw_step(w, step, re, ro, mg);
-    // fp16 pairs (1032, 1032), (1/16, 1/16), (-72, -72) as bit patterns
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(e) : "r"(re), "r"(0x64086408u));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(o) : "r"(ro), "r"(0x2C002C00u), "r"(0xD480D480u));
 }
 
 __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t a0, uint32_t a1,
@@ -564,7 +557,9 @@ __device__ bool finish_item(const Ctx& x, int m) {
             report(a.status, COLI_ERR_RANGE);
             h = copysignf(65504.f, h);
         }
-        a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn(h);
+        // odd features are the down projection's odd-K elements: stored / 16
+        // for its raw unpack (odd codes as 1152 + 16 q)
+        a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn((n & 1) ? h * 0.0625f : h);
     }
     __syncwarp();
     if (lane == 0) {
@@ -699,8 +694,12 @@ __device__ __forceinline__ bool advance_frontier(const Ctx& x, int& frontier, in
 }
 
 // One down stage: this CTA's tiles of slot s's W_d, accumulated into acc.
+// The codes are unpacked raw (1032 + q even, 1152 + 16 q odd, against h'
+// whose odd elements are stored / 16); each group's MMA chain starts from
+// dcorr, the negated offset sums of the slot's h' for this lane's columns.
 __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt,
                                            const uint32_t (&bcur)[kMaxDW][8],
+                                           const float (&dcorr)[kMaxDW][2],
                                            const int (&dcoff)[kMaxDW], int g_lo,
                                            float (&acc)[kMaxMT][4]) {
     const Layout& L = x.L;
@@ -732,16 +731,18 @@ __device__ __forceinline__ bool down_stage(const Ctx& x, int s, int j, int my_mt
                 const uint32_t codes = st + m * L.dn_op + dcoff[i];
                 wa[m] = lds_u2(codes);
                 wb[m] = lds_u2(codes + row8);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) part[m][q] = 0.f;
+                part[m][0] = dcorr[i][0];
+                part[m][1] = dcorr[i][1];
+                part[m][2] = dcorr[i][0];
+                part[m][3] = dcorr[i][1];
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 uint32_t ae[kMaxMT], ao[kMaxMT], be[kMaxMT], bo[kMaxMT];
 #pragma unroll
                 for (int m = 0; m < kMaxMT; ++m) {
-                    unpack_exact_step((ks >> 1) ? wa[m].y : wa[m].x, ks & 1, ae[m], ao[m], mg);
-                    unpack_exact_step((ks >> 1) ? wb[m].y : wb[m].x, ks & 1, be[m], bo[m], mg);
+                    unpack_raw_step((ks >> 1) ? wa[m].y : wa[m].x, ks & 1, ae[m], ao[m], mg);
+                    unpack_raw_step((ks >> 1) ? wb[m].y : wb[m].x, ks & 1, be[m], bo[m], mg);
                 }
 #pragma unroll
                 for (int m = 0; m < kMaxMT; ++m)
@@ -1095,16 +1096,22 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         int frontier = 0;
         alive = advance_frontier(ctx, frontier, 0);
         if (alive) load_down_b(a, S.table + 0, dg_lo, b1);
+        float dcorr[kMaxDW][2];
         for (int s = 0; s < n_slots && alive; ++s, ++j) {
 #pragma unroll
-            for (int i = 0; i < kMaxDW; ++i)
+            for (int i = 0; i < kMaxDW; ++i) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) b0[i][q] = b1[i][q];
+                float cs[4];
+                offset_sums(b0[i], cs);  // zero fragments (absent tokens, groups past I) give 0
+                dcorr[i][0] = -cs[0];
+                dcorr[i][1] = -cs[1];
+            }
             if (s + 1 < n_slots) {
                 if (frontier <= s + 1) alive = advance_frontier(ctx, frontier, s + 1);
                 if (alive) load_down_b(a, S.table + s + 1, dg_lo, b1);
             }
-            if (alive) alive = down_stage(ctx, s, j, my_mt, b0, dcoff, dg_lo, acc);
+            if (alive) alive = down_stage(ctx, s, j, my_mt, b0, dcorr, dcoff, dg_lo, acc);
         }
     }
 
