@@ -59,19 +59,17 @@ namespace {
 
 constexpr int BM = 128, BK = 64;
 constexpr int kBRowQuant = 32;      // activation rows are loaded in multiples of 32
-constexpr int kThreadsP = 512;
 constexpr uint32_t kTmemColsP = 512;
 constexpr int kHeaderP = 2048;
 constexpr int kSmemLimitP = 227 * 1024;
 
-// Two shapes of the same pipeline.  Large token tiles (prefill: ~128 tokens
-// per expert): 192-token tiles, one accumulator, a 2-deep operand ring, 4
-// dequantising warps (one weight row of both blocks per thread) and 8
-// epilogue warps.  Small token tiles (a few tokens per expert, every call
-// with T <= 64): 64-token tiles, a double-buffered accumulator, a 4-deep
-// operand ring, 8 dequantising warps (one weight row of one block per
-// thread) and 4 epilogue warps: there the dequantisation, not the MMA or the
-// epilogue, sets the rate.
+// Two shapes of the same pipeline, both with 8 dequantising warps (two per
+// lane quarter, one weight row of one block per thread).  Large token tiles
+// (prefill: ~128 tokens per expert): 192-token tiles, one accumulator, a
+// 2-deep operand ring and 8 epilogue warps (20 warps in all).  Small token
+// tiles (a few tokens per expert, every call with T <= 64): 64-token tiles,
+// a double-buffered accumulator, a 4-deep operand ring and 4 epilogue warps
+// (16 warps).
 template <bool kSmall>
 struct Cfg {
     static constexpr int BN = kSmall ? 64 : 192;            // tokens per tile (max)
@@ -79,10 +77,11 @@ struct Cfg {
     static constexpr uint32_t kAccCols = 2 * BN * kAccBufs;  // accumulators, then the ring
     static constexpr int kACols = BK;                        // operand columns per K-block (2 blocks)
     static constexpr int kAStages = (int)(kTmemColsP - kAccCols) / kACols;
-    static constexpr int kDqWarp0 = kSmall ? 8 : 4;
-    static constexpr int kDqWarps = kSmall ? 8 : 4;
-    static constexpr int kEpiWarp0 = kSmall ? 4 : 8;
+    static constexpr int kDqWarp0 = 4;                       // warps 4-11: two per lane
+    static constexpr int kDqWarps = 8;                       // quarter, one block each
+    static constexpr int kEpiWarp0 = 12;
     static constexpr int kEpiWarps = kSmall ? 4 : 8;
+    static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;  // 512 or 640
     static constexpr int kBBytes = BN * BK * 2;               // activation tile per stage
     static constexpr int kStage = kBBytes + 2 * BM * BK / 2;  // + two blocks of packed codes
 };
@@ -256,7 +255,7 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, bool gu, int64_
 // the up rows of the same 128 features, K = H), otherwise down (two blocks of
 // 128 rows of W_d, 256 output features, K = I).
 template <bool kGU, bool kSmall>
-__global__ void __launch_bounds__(kThreadsP, 1)
+__global__ void __launch_bounds__(Cfg<kSmall>::kThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
                     const __grid_constant__ CUtensorMap bmap64,
                     const __grid_constant__ CUtensorMap bmap32, const GemmArgs a, int stages) {
@@ -423,8 +422,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap128,
         // two warps per lane quarter, each one block
         const int q = warp & 3;
         const int row = q * 32 + lane;  // MMA row of the tile owned by this thread
-        constexpr int kMyBlocks = kSmall ? 1 : NA;
-        const int blk0 = kSmall ? (warp - C::kDqWarp0) >> 2 : 0;
+        constexpr int kMyBlocks = 1;
+        const int blk0 = (warp - C::kDqWarp0) >> 2;
         // this warp's 32 lanes of the operand ring
         const uint32_t ta = tmem_base + ((uint32_t)q << 21) + C::kAccCols;
         Ring rs, ra;
@@ -733,7 +732,7 @@ cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms);
-    cfg.blockDim = dim3(kThreadsP);
+    cfg.blockDim = dim3(Cfg<kSmall>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
