@@ -68,13 +68,30 @@ PREFETCH_BYTES = 20 << 20
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (or TC util) vs B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
-# DRAM bytes (read + write) per launch of a workload's dominant kernel, taken
-# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).  Each
-# entry names the kernel source file and its SHA-256 at capture time; when
-# the file has changed since, the bench reports traffic as null.  Entries:
-# workload -> (source file, sha256, bytes per launch, how the figure was
-# obtained).
-DRAM_TRAFFIC = {}
+# DRAM bytes (read + write) of a workload's dominant kernel, from one ncu
+# launch-list capture (dram__bytes_read.sum + dram__bytes_write.sum), as bytes
+# per unit of work: a launch, or an expert the launch streams (the kernels'
+# traffic grows with the experts they stream, so a capture on a smaller bank
+# scales to the workload's own streamed experts).  Each entry names the
+# kernel's source file and its SHA-256 at capture time; when the file has
+# changed since, the bench reports traffic as null.
+# workload -> (source file, sha256, bytes per unit, unit, how it was measured)
+_DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
+               "1506f68fc46b9ee9ab38cc75100ddf4998dfcd10e145e90b979412589559afd1")
+_GEMM_SRC = ("int4_routed_expert_coli_b200/csrc/prefill.cu",
+             "896bf7fc35acc8db8115674e96ccda327433d88f3880fd31f647173a8a1185f3")
+_GEMM_SMALL = (*_GEMM_SRC, 13_692_332, "streamed expert",
+               "ncu launch list, 12 launches of the small-tile gate/up GEMM on a 64-expert "
+               "bank at T=32: bytes per streamed expert (unique routed + shared)")
+DRAM_TRAFFIC = {
+    "decode": (*_DECODE_SRC, 180_914_503, "launch",
+               "ncu launch list, 18 launches of the fused decode kernel on a 64-expert bank "
+               "(a T=1 step streams 8 + 1 experts on any bank)"),
+    "verify4": (*_DECODE_SRC, 180_914_503 // 9, "streamed expert",
+                "the T=1 fused-kernel capture, bytes per streamed expert"),
+    "batch32": _GEMM_SMALL,
+    "stack": _GEMM_SMALL,
+}
 
 
 def expert_bytes(H, I):
@@ -91,15 +108,16 @@ def _sha256(path):
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def traffic_for(workload):
-    """(bytes per launch or None, source note) for the workload's dominant kernel."""
+def traffic_for(workload, units):
+    """(DRAM bytes per launch of the workload's dominant kernel, or None, and
+    a note on the source); `units`: the launch's streamed experts."""
     ent = DRAM_TRAFFIC.get(workload)
     if ent is None:
-        return None, "no ncu capture of the current kernel for this workload"
-    src, sha, nbytes, how = ent
+        return None, "no ncu capture whose bytes scale to this workload"
+    src, sha, per_unit, unit, how = ent
     if _sha256(os.path.join(ROOT, src)) != sha:
         return None, f"stale: {src} changed since the ncu capture"
-    return nbytes, how
+    return (per_unit if unit == "launch" else per_unit * units), how
 
 
 def peaks():
@@ -515,7 +533,8 @@ def run_stack(args, rank, world, local, with_cpu=True):
     k_bytes = statistics.mean(statistics.mean(us) for us in uniq) * gateup_bytes(H, I) + \
         n_sh * gateup_bytes(H, I)
     achieved = k_bytes / (k_ms / 1e3) / 1e9
-    traffic, traffic_src = traffic_for("stack")
+    traffic, traffic_src = traffic_for(
+        "stack", statistics.mean(statistics.mean(us) for us in uniq) + n_sh)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -685,7 +704,7 @@ def run_ours(args, rank, world, local, name, with_cpu=True):
     stream = not fused and T * k < E
     tensor = kind == "uniform"  # prefill: tensor-bound
     k_ms = phase_ms[1] / max(n_calls, 1)
-    traffic, traffic_src = traffic_for(name)
+    traffic, traffic_src = traffic_for(name, n_uniq + n_sh)
     if tensor:
         # gate/up GEMM: 2/3 of the pair FLOPs over all (token, expert) pairs + shared
         k_work = (T * k + T * n_sh) * PAIR_FLOP * 2 / 3
