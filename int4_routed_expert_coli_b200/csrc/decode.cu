@@ -3,12 +3,14 @@
 // every active expert's int4 gs64 weights from HBM exactly once per call
 // ("batch-union", "yunpan.plus/t/30351-1-1", capability two).
 //
-// Routing.  Every CTA routes the T tokens itself from the logits (one warp
-// per token, the exact rule of the routing step) and builds the same slot
-// table in shared memory: shared experts first, then the active routed
-// experts in ascending order, each with the positions and gate weights of
-// its tokens.  Given a precomputed union instead (the FFN entry point), the
-// table is read from it.
+// Routing.  In every CTA, consumer warp t routes token t from the logits
+// (the exact rule of the routing step, with a butterfly top-k) while the
+// activations load, and the producer warp builds the slot table in shared
+// memory: shared experts first, then the active routed experts in ascending
+// order, each with the positions and gate weights of its tokens.  Given a
+// precomputed union instead (the FFN entry point), the table is read from
+// it.  The shared experts' entries need no routing, so their gate/up tiles
+// are staged and computed before the table is known.
 //
 // Gate/up.  An item is 8 gate rows + the same 8 up rows of one slot over the
 // whole hidden dimension; items are dealt round-robin to the CTAs (one per
@@ -20,8 +22,9 @@
 // streams, slot after slot, those rows of W_d.  The MMA columns are the
 // tokens, so y = sum over slots of W_d h' accumulates in registers: the
 // combine is the accumulation itself, in a fixed order (slot order, then a
-// fixed sum over the warps).  A slot's h' rows are read once its counter says
-// all its gate/up tiles are done.
+// fixed sum over the warps).  A slot's h' rows are read once it is below the
+// frontier of complete slots, which the producer warp follows by polling the
+// slots' counters and publishes in shared memory.
 //
 // Data movement.  A producer warp loads each stage with 3-D TMA tensor copies
 // of the packed code rows (viewed as 128-byte chunks plus zero-filled padding
@@ -34,9 +37,9 @@
 // value: for gate/up the sums of x, for down the sums of the slot's h'
 // (stored with its odd elements divided by 16), computed from the h'
 // fragments with four MMAs per group; m16n8k16 MMA with fp32 accumulation,
-// the group's scale applied to each group's partial.  Eleven consumer warps split K; a gate/up item's partials
-// are summed through four reduction buffers, item j by warp j mod 11 two
-// items later (in warp order, so the sum does not depend on timing).
+// the group's scale applied to each group's partial.  Sixteen consumer warps split K; a gate/up item's
+// partials are summed through four reduction buffers, item j by warp j mod 16
+// two items later (in warp order, so the sum does not depend on timing).
 //
 // Every wait is bounded (COLI_ERR_TIMEOUT).  The counters are zero on entry;
 // the last CTA to finish puts them back to zero.
@@ -51,7 +54,7 @@
 namespace coli {
 namespace {
 
-constexpr int kCW = 11;                      // consumer warps (12 warps in all)
+constexpr int kCW = 16;                      // consumer warps (17 warps in all)
 constexpr int kThreadsD = (kCW + 1) * 32;    // + producer warp
 constexpr int kStagesD = 3;
 constexpr int kRedBufs = 4;
@@ -105,7 +108,7 @@ struct Layout {
     int gu_op, gu_sc, gu_tx;    // gate/up item: code copy, scale copy, bytes per stage
     int dn_op, dn_sc;           // down tile: code copy, scale copy
     int stage_bytes;
-    int red_off, corr_off, route_off, table_off, cnt_off, stage_off, smem;
+    int red_off, corr_off, route_off, table_off, stage_off, smem;
 };
 
 // per_row: one scale per row (staged as the item's rows' scales, 2 bytes
@@ -134,8 +137,7 @@ __host__ __device__ inline Layout make_layout(int H, int I, int max_slots, int p
     L.corr_off = L.red_off + kRedFloats * 4;
     L.route_off = L.corr_off + kCW * kMaxGW * 16 * 4;
     L.table_off = L.route_off + 3 * kMaxPairs * 4;
-    L.cnt_off = L.table_off + max_slots * (int)sizeof(SlotEntry);
-    L.stage_off = (L.cnt_off + 3 * max_slots * 4 + 1023) / 1024 * 1024;
+    L.stage_off = (L.table_off + max_slots * (int)sizeof(SlotEntry) + 1023) / 1024 * 1024;
     L.smem = L.stage_off + kStagesD * L.stage_bytes + 1024;  // + alignment slack
     return L;
 }
@@ -225,9 +227,9 @@ __device__ __forceinline__ void offset_sums(const uint32_t bw[8], float c[4]) {
     mma16816(c, c, ev, ev, od, od, bw[6], bw[7]);
 }
 
-__device__ __forceinline__ int ld_relaxed(const int* p) {
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     int v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -259,8 +261,10 @@ struct Smem {
     uint64_t* empty;
     uint64_t* red_empty;
     uint64_t* tbl_ready;
+    uint64_t* routed;          // one arrival per routing warp
     volatile int* abort_flag;
     volatile int* n_slots;
+    volatile int* frontier;    // slots [0, frontier) complete GPU-wide (producer-written)
     volatile int* stage_item;  // [kStagesD] gate/up item in the stage; -1: a down stage
     int* red_cnt;      // [kRedBufs] partials written into each reduction buffer
     volatile int* red_item;  // [kRedBufs] the item whose partials a buffer holds
@@ -270,9 +274,6 @@ struct Smem {
     float* s_w;
     int* s_aux;
     SlotEntry* table;
-    int* done_local;     // [slots] gate/up tiles finished in this CTA (consumers count)
-    int* pub_local;      // [slots] of those, published to the slot counters (producer)
-    int* issued_local;   // [slots] gate/up tiles of a valid slot this CTA was given
     uint8_t* stage0;
 };
 
@@ -282,20 +283,19 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const Layout& L, int max_sl
     S.empty = S.full + kStagesD;
     S.red_empty = S.empty + kStagesD;
     S.tbl_ready = S.red_empty + kRedBufs;
+    S.routed = S.tbl_ready + 1;
     S.abort_flag = reinterpret_cast<volatile int*>(smem + 512);
     S.n_slots = S.abort_flag + 1;
     S.red_cnt = reinterpret_cast<int*>(smem + 528);
     S.stage_item = reinterpret_cast<volatile int*>(smem + 560);
     S.red_item = reinterpret_cast<volatile int*>(smem + 576);
+    S.frontier = reinterpret_cast<volatile int*>(smem + 600);
     S.red = reinterpret_cast<float*>(smem + L.red_off);
     S.corr = reinterpret_cast<float*>(smem + L.corr_off);
     S.s_idx = reinterpret_cast<int*>(smem + L.route_off);
     S.s_w = reinterpret_cast<float*>(S.s_idx + kMaxPairs);
     S.s_aux = S.s_idx + 2 * kMaxPairs;
     S.table = reinterpret_cast<SlotEntry*>(smem + L.table_off);
-    S.done_local = reinterpret_cast<int*>(smem + L.cnt_off);
-    S.pub_local = S.done_local + max_slots;
-    S.issued_local = S.pub_local + max_slots;
     S.stage0 = smem + L.stage_off;
     return S;
 }
@@ -304,42 +304,47 @@ constexpr int kConsumerThreads = kCW * 32;
 
 __device__ __forceinline__ void consumers_sync() { named_barrier(1, kConsumerThreads); }
 
-__device__ void table_init(const FfnArgs& a, const Smem& S, int max_slots) {
-    for (int i = threadIdx.x; i < max_slots; i += kConsumerThreads) {
-        SlotEntry& en = S.table[i];
-        en.e = -1;
-        en.list_begin = 0;
+__device__ __forceinline__ void clear_entry(SlotEntry& en) {
+    en.e = -1;
+    en.list_begin = 0;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            en.pos[t] = -1;
-            en.w[t] = 0.f;
-        }
+    for (int t = 0; t < 8; ++t) {
+        en.pos[t] = -1;
+        en.w[t] = 0.f;
     }
-    consumers_sync();
-    for (int i = threadIdx.x; i < a.n_shared; i += kConsumerThreads) {
+}
+
+// Slot i < n_shared: shared expert i, every token, weight 1 -- known without
+// routing.  Lanes of one warp, each its own entries.
+__device__ void table_shared(const FfnArgs& a, const Smem& S, int lane) {
+    for (int i = lane; i < a.n_shared; i += 32) {
         SlotEntry& en = S.table[i];
         en.e = a.E + i;
         en.list_begin = a.T * a.k + i * a.T;
-        for (int t = 0; t < a.T; ++t) {
-            en.pos[t] = (int8_t)t;
-            en.w[t] = 1.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            en.pos[t] = (int8_t)(t < a.T ? t : -1);
+            en.w[t] = t < a.T ? 1.f : 0.f;
         }
     }
 }
 
-// The slot table from the routing (s_idx / s_w, written by the routing
-// warps before this): the union of the pairs p = t * k + j, experts
-// ascending, tokens ascending inside an expert (the lists the batch-union
-// step defines).
-__device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
+// The routed slots of the table from the routing (s_idx / s_w): the union of
+// the pairs p = t * k + j, experts ascending, tokens ascending inside an
+// expert (the lists the batch-union step defines).  One warp.
+__device__ void table_from_logits(const DecodeArgs& d, const Smem& S, int lane) {
     const FfnArgs& a = d.f;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int P = a.T * a.k;
+    if (blockIdx.x == 0) {
+        for (int p = lane; p < P; p += 32) {
+            if (d.idx_out) d.idx_out[p] = S.s_idx[p];
+            if (d.w_out) d.w_out[p] = S.s_w[p];
+        }
+    }
+    for (int i = a.n_shared + lane; i < d.max_slots; i += 32) clear_entry(S.table[i]);
+    __syncwarp();
     if (P <= 32) {
-        // one warp, one pair per lane: leaders by match_any, ranks by shuffles
-        if (a.T > 1) consumers_sync();  // the other routing warps' pairs
-        if (warp != 0) return;
-        __syncwarp();
+        // one pair per lane: leaders by match_any, ranks by shuffles
         const bool on = lane < P;
         const int e = on ? S.s_idx[lane] : INT_MAX;
         const float w = on ? S.s_w[lane] : 0.f;
@@ -353,19 +358,6 @@ __device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
             before += eq < e;
             rank += (eq < e) & (int)((leads >> q) & 1u);
         }
-        const int n_slots = a.n_shared + __popc(leads);
-        for (int i = lane; i < n_slots; i += 32) {
-            SlotEntry& en = S.table[i];
-            const bool sh = i < a.n_shared;
-            en.e = sh ? a.E + i : -1;
-            en.list_begin = sh ? P + i * a.T : 0;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                en.pos[t] = (int8_t)((sh && t < a.T) ? t : -1);
-                en.w[t] = (sh && t < a.T) ? 1.f : 0.f;
-            }
-        }
-        __syncwarp();
         if (on) {
             SlotEntry& en = S.table[a.n_shared + rank];
             if (lead) {
@@ -375,31 +367,21 @@ __device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
             const int t = lane / a.k;
             en.pos[t] = (int8_t)__popc(peers & below);
             en.w[t] = w;
-            if (blockIdx.x == 0) {
-                if (d.idx_out) d.idx_out[lane] = e;
-                if (d.w_out) d.w_out[lane] = w;
-            }
         }
-        if (lane == 0) *S.n_slots = n_slots;
+        if (lane == 0) *S.n_slots = a.n_shared + __popc(leads);
+        __syncwarp();
         return;
     }
-    table_init(a, S, d.max_slots);
-    consumers_sync();
-    if (blockIdx.x == 0) {
-        for (int p = tid; p < P; p += kConsumerThreads) {
-            if (d.idx_out) d.idx_out[p] = S.s_idx[p];
-            if (d.w_out) d.w_out[p] = S.s_w[p];
-        }
-    }
     // a pair is its expert's leader if no earlier pair has the same expert
-    for (int p = tid; p < P; p += kConsumerThreads) {
+    for (int p = lane; p < P; p += 32) {
         const int e = S.s_idx[p];
         int lead = 1;
         for (int q = 0; q < p; ++q) lead &= S.s_idx[q] != e;
         S.s_aux[p] = lead;
     }
-    consumers_sync();
-    for (int p = tid; p < P; p += kConsumerThreads) {
+    __syncwarp();
+    int n = 0;
+    for (int p = lane; p < P; p += 32) {
         const int e = S.s_idx[p];
         int before = 0, rank = 0, pos = 0;
         for (int q = 0; q < P; ++q) {
@@ -416,32 +398,29 @@ __device__ void table_from_logits(const DecodeArgs& d, const Smem& S) {
         const int t = p / a.k;
         en.pos[t] = (int8_t)pos;
         en.w[t] = S.s_w[p];
+        n += S.s_aux[p];
     }
-    if (warp == 0) {
-        int n = 0;
-        for (int p = lane; p < P; p += 32) n += S.s_aux[p];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-        if (lane == 0) *S.n_slots = a.n_shared + n;
-    }
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if (lane == 0) *S.n_slots = a.n_shared + n;
+    __syncwarp();
 }
 
-// Slot table from a given union (counts / offsets / pairs / active /
+// The routed slots from a given union (counts / offsets / pairs / active /
 // n_active and the gate weights); an inconsistent entry is reported as
-// COLI_ERR_BAD_INDEX and its slot skipped.
-__device__ void table_from_union(const DecodeArgs& d, const Smem& S) {
+// COLI_ERR_BAD_INDEX and its slot skipped.  One warp.
+__device__ void table_from_union(const DecodeArgs& d, const Smem& S, int lane) {
     const FfnArgs& a = d.f;
-    const int tid = threadIdx.x;
     const int P = a.T * a.k;
-    table_init(a, S, d.max_slots);
-    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
+    for (int i = a.n_shared + lane; i < d.max_slots; i += 32) clear_entry(S.table[i]);
+    __syncwarp();
+    int n_act = __shfl_sync(0xffffffffu, *reinterpret_cast<const volatile int*>(a.n_active), 0);
     const int cap = d.max_slots - a.n_shared;
     if (n_act < 0 || n_act > cap) {
-        if (tid == 0) report(a.status, COLI_ERR_BAD_INDEX);
+        if (lane == 0) report(a.status, COLI_ERR_BAD_INDEX);
         n_act = n_act < 0 ? 0 : cap;
     }
-    consumers_sync();
-    for (int i = tid; i < n_act; i += kConsumerThreads) {
+    for (int i = lane; i < n_act; i += 32) {
         SlotEntry& en = S.table[a.n_shared + i];
         const int e = a.active[i];
         bool ok = e >= 0 && e < a.E;
@@ -464,7 +443,23 @@ __device__ void table_from_union(const DecodeArgs& d, const Smem& S) {
             report(a.status, COLI_ERR_BAD_INDEX);
         }
     }
-    if (tid == 0) *S.n_slots = a.n_shared + n_act;
+    if (lane == 0) *S.n_slots = a.n_shared + n_act;
+    __syncwarp();
+}
+
+// Frontier of complete slots in shared memory: the producer warp publishes
+// it with a release store after it has observed (and acquired) the slots'
+// counters; a consumer that reads it with an acquire load may then read the
+// h' rows of every slot below it.
+__device__ __forceinline__ int ld_acquire_cta(const volatile int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr((const void*)p))
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta(volatile int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr((const void*)p)), "r"(v)
+                 : "memory");
 }
 
 struct Ctx {
@@ -472,7 +467,7 @@ struct Ctx {
     const Layout& L;
     const Smem& S;
     int* sync;
-    int n_slots, gu_tiles;
+    int gu_tiles;
 };
 
 __device__ __forceinline__ void fail(const Ctx& x, int lane) {
@@ -499,13 +494,26 @@ __device__ __forceinline__ bool post_partial(const Ctx& x, int j, int item,
     return true;
 }
 
+// Publishes a gate/up tile this warp finished earlier (slot `pending`, -1:
+// none): one GPU-scope fence, which makes the tile's h' stores (by this
+// warp's lanes, ordered by the __syncwarp) visible first, then the slot's
+// counter.  Called before the warp issues new h' stores, so the fence does
+// not wait for them: the tile's own stores went out a round of items ago.
+__device__ __forceinline__ void publish_tile(const Ctx& x, int pending) {
+    if (pending < 0) return;
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        fence_acq_rel_gpu();
+        atomicAdd(x.sync + kSyncSlots + pending, 1);
+    }
+}
+
 // Sum of item m (its kCW partials in warp order, so the result does not
 // depend on timing) and its epilogue h' = w * silu(g) * u for the slot's
 // tokens, by warp m % kCW kRedLag items later: off the critical path of the
-// warp that finished item m last.  The tile is then counted in this CTA's
-// done_local (a CTA-scope release); the producer thread publishes the counts
-// GPU-wide.  false: timeout or abort.
-__device__ bool finish_item(const Ctx& x, int m) {
+// warp that finished item m last.  The tile this warp finished before is
+// published first; this one becomes `pending`.  false: timeout or abort.
+__device__ bool finish_item(const Ctx& x, int m, int& pending) {
     const FfnArgs& a = x.a;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int rb = m % kRedBufs;
@@ -541,6 +549,8 @@ __device__ bool finish_item(const Ctx& x, int m) {
     const int slot = item / x.gu_tiles, tile = item - slot * x.gu_tiles;
     const SlotEntry* en = x.S.table + slot;
     if (en->e < 0) return true;
+    publish_tile(x, pending);
+    pending = slot;
     const float v[4] = {sum.x, sum.y, sum.z, sum.w};
     const int n = tile * kGuRows + r;
     const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
@@ -561,11 +571,6 @@ __device__ bool finish_item(const Ctx& x, int m) {
         // for its raw unpack (odd codes as 1152 + 16 q)
         a.hp[(int64_t)(list_begin + p) * a.I + hcol] = __float2half_rn((n & 1) ? h * 0.0625f : h);
     }
-    __syncwarp();
-    if (lane == 0) {
-        __threadfence_block();
-        atomicAdd(x.S.done_local + slot, 1);
-    }
     return true;
 }
 
@@ -575,7 +580,7 @@ __device__ bool finish_item(const Ctx& x, int m) {
 // Returns false when the kernel must wind down.
 __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
                                             const uint32_t (&breg)[kMaxGW][8],
-                                            const int (&coff)[kMaxGW], int g_lo) {
+                                            const int (&coff)[kMaxGW], int g_lo, int& pending) {
     const int slot = item / x.gu_tiles;
     const Layout& L = x.L;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
@@ -590,15 +595,17 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
         const uint32_t scB = scA + L.gu_sc;
         const uint32_t cor = smem_addr(x.S.corr) + c * 16;
         const Magic mg = magic();
-        // three independent MMA chains at a time.  A group past the end of
+        // kChains independent MMA chains at a time.  A group past the end of
         // H (the last warp's) has a zero B fragment, a zero offset sum and a
         // zero scale, and reads real staged codes.
+        constexpr int kChains = 2;
+        static_assert(kMaxGW % kChains == 0, "whole chain sets");
 #pragma unroll
-        for (int i0 = 0; i0 < kMaxGW; i0 += 3) {
-            uint2 wa[3], wb[3];
-            float part[3][4], fa[3], fb[3];
+        for (int i0 = 0; i0 < kMaxGW; i0 += kChains) {
+            uint2 wa[kChains], wb[kChains];
+            float part[kChains][4], fa[kChains], fb[kChains];
 #pragma unroll
-            for (int u = 0; u < 3; ++u) {
+            for (int u = 0; u < kChains; ++u) {
                 const int i = i0 + u, grp = g_lo + i;
                 wa[u] = lds_u2(st + coff[i]);
                 wb[u] = lds_u2(st + L.gu_op + coff[i]);
@@ -612,19 +619,19 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the group
-                uint32_t ae[3], ao[3], be[3], bo[3];
+                uint32_t ae[kChains], ao[kChains], be[kChains], bo[kChains];
 #pragma unroll
-                for (int u = 0; u < 3; ++u) {
+                for (int u = 0; u < kChains; ++u) {
                     unpack_raw_step((ks >> 1) ? wa[u].y : wa[u].x, ks & 1, ae[u], ao[u], mg);
                     unpack_raw_step((ks >> 1) ? wb[u].y : wb[u].x, ks & 1, be[u], bo[u], mg);
                 }
 #pragma unroll
-                for (int u = 0; u < 3; ++u)
+                for (int u = 0; u < kChains; ++u)
                     mma16816(part[u], part[u], ae[u], be[u], ao[u], bo[u],
                              breg[i0 + u][2 * ks], breg[i0 + u][2 * ks + 1]);
             }
 #pragma unroll
-            for (int u = 0; u < 3; ++u) {
+            for (int u = 0; u < kChains; ++u) {
                 acc[0] = fmaf(fa[u], part[u][0], acc[0]);
                 acc[1] = fmaf(fa[u], part[u][1], acc[1]);
                 acc[2] = fmaf(fb[u], part[u][2], acc[2]);
@@ -640,7 +647,7 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
         return false;
     }
     const int m = j - kRedLag;
-    if (m >= 0 && m % kCW == (int)(threadIdx.x >> 5)) return finish_item(x, m);
+    if (m >= 0 && m % kCW == (int)(threadIdx.x >> 5)) return finish_item(x, m, pending);
     return true;
 }
 
@@ -664,33 +671,22 @@ __device__ __forceinline__ void load_down_b(const FfnArgs& a, const SlotEntry* e
     }
 }
 
-// True once all gate/up tiles of slot s are published (an invalid slot has
-// nothing to wait for).  Relaxed read.
-__device__ __forceinline__ bool slot_ready(const Ctx& x, int s) {
-    return x.S.table[s].e < 0 || ld_relaxed(x.sync + kSyncSlots + s) >= x.gu_tiles;
-}
-
-// Move `frontier` (slots [0, frontier) are complete and their h' visible to
-// this warp) past slot `need`: the lanes poll 32 slots at once, the frontier
-// jumps over the leading complete ones, and one fence orders every later h'
-// read after those observations.  Bounded wait; false on timeout or abort.
-__device__ __forceinline__ bool advance_frontier(const Ctx& x, int& frontier, int need) {
+// Wait until slot `need` is below the frontier the producer warp publishes
+// (every lane acquires it, so its later h' reads of those slots see the
+// writers' stores).  Warp-uniform; bounded; false on timeout or abort.
+__device__ __forceinline__ bool wait_frontier(const Ctx& x, int need) {
+    if (__all_sync(0xffffffffu, ld_acquire_cta(x.S.frontier) > need)) return true;
     const int lane = threadIdx.x & 31;
     const uint64_t t0 = global_timer_ns();
-    while (frontier <= need) {
-        const int s = frontier + lane;
-        const unsigned done = __ballot_sync(0xffffffffu, s >= x.n_slots || slot_ready(x, s));
-        frontier += done == 0xffffffffu ? 32 : __ffs(~done) - 1;
-        if (frontier > need) break;
-        if (*x.S.abort_flag) return false;
-        __nanosleep(256);
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            fail(x, lane);
-            return false;
-        }
+    for (;;) {
+        __nanosleep(64);
+        if (__all_sync(0xffffffffu, ld_acquire_cta(x.S.frontier) > need)) return true;
+        int stop = 0;
+        if (lane == 0) stop = *x.S.abort_flag ? 1 : global_timer_ns() - t0 > kWaitLimitNs ? 2 : 0;
+        stop = __shfl_sync(0xffffffffu, stop, 0);
+        if (stop == 2) fail(x, lane);
+        if (stop) return false;
     }
-    fence_acq_rel_gpu();
-    return true;
 }
 
 // One down stage: this CTA's tiles of slot s's W_d, accumulated into acc.
@@ -797,9 +793,11 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             S.red_cnt[b] = 0;
         }
         mbar_init(S.tbl_ready, 1);
+        mbar_init(S.routed, a.T > 0 ? a.T : 1);
+
         *S.abort_flag = 0;
+        *S.frontier = 0;
     }
-    for (int i = threadIdx.x; i < 3 * d.max_slots; i += kThreadsD) S.done_local[i] = 0;
     if (threadIdx.x == 0) {
         fence_barrier_init();
     }
@@ -808,189 +806,237 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
 
     const int G = gridDim.x, b = blockIdx.x;
     const int gu_tiles = a.I / kGuRows;
+    const int n_gu_shared = a.n_shared * gu_tiles;
     const int n_mt = a.H / kDnRows;
     const int bm = G - 1 - b;  // this CTA's down tiles: bm, bm + G, ...
     const int my_mt = bm < n_mt ? (n_mt - 1 - bm) / G + 1 : 0;
+    constexpr unsigned kAll = 0xffffffffu;
 
     if (warp == kCW) {
-        // ------------------------------ producer ------------------------------
-        if (lane == 0) {
-            const uint64_t policy = policy_evict_first();
-            const int n_gu_shared = a.n_shared * gu_tiles;
-            int n_slots = -1;
-            int j = 0;
-            bool stop = false;
-            auto table_known = [&]() -> bool {
-                if (n_slots >= 0) return true;
-                if (!mbar_wait(S.tbl_ready, 0)) {
-                    report(a.status, COLI_ERR_TIMEOUT);
-                    *S.abort_flag = 1;
-                    return false;
-                }
-                n_slots = *S.n_slots;
-                return true;
-            };
-            // Publishing: the tiles the consumers finished (done_local, a
-            // CTA-scope release by the reducing warp) go to the GPU-wide slot
-            // counters after one GPU-scope fence, which makes their h' stores
-            // visible first.  Runs whenever the producer would otherwise wait.
-            int pub_lo = 0, pub_hi = -1;  // slots this CTA has tiles of, not all published
-            auto pump = [&]() {
-                bool fenced = false;
-                for (int sl = pub_lo; sl <= pub_hi; ++sl) {
-                    const int dn = *reinterpret_cast<volatile int*>(S.done_local + sl);
-                    const int pb = S.pub_local[sl];
-                    if (dn > pb) {
-                        if (!fenced) {
-                            fence_acq_rel_gpu();
-                            fenced = true;
-                        }
-                        atomicAdd(d.sync + kSyncSlots + sl, dn - pb);
-                        S.pub_local[sl] = dn;
-                    }
-                }
-                // a slot below the newest is complete here once all its tiles are out
-                while (pub_lo < pub_hi && S.pub_local[pub_lo] == S.issued_local[pub_lo]) ++pub_lo;
-            };
-            auto all_published = [&]() -> bool {
-                return pub_hi < 0 || (pub_lo == pub_hi && S.pub_local[pub_hi] == S.issued_local[pub_hi]);
-            };
-            auto next_stage = [&](uint8_t*& st) -> bool {
-                const int stage = j % kStagesD, use = j / kStagesD;
-                if (use > 0 && !mbar_test_wait(&S.empty[stage], (use - 1) & 1)) {
+        // ---------------------------- producer warp ----------------------------
+        // Control flow is warp-uniform; lane 0 arms the barriers and issues
+        // the copies, the whole warp routes and polls the slot counters.
+        const uint64_t policy = policy_evict_first();
+        // the shared experts' slots need no routing: written before the
+        // first stage is armed, so a consumer that sees a staged item of
+        // theirs also sees their entries
+        table_shared(a, S, lane);
+        __syncwarp();
+        int n_slots = -1;
+        int j = 0;
+        bool stop = false;
+        bool pdl_done = false;
+        int frontier = 0;       // slots [0, frontier) complete GPU-wide
+        bool poll = false;  // the frontier matters once this CTA's gate/up items are out
+        auto abort_set = [&]() -> bool { return __shfl_sync(kAll, (int)*S.abort_flag, 0) != 0; };
+        auto give_up = [&]() {
+            if (lane == 0) {
+                report(a.status, COLI_ERR_TIMEOUT);
+                *S.abort_flag = 1;
+            }
+            __syncwarp();
+        };
+        // For this CTA's down phase, the frontier of complete slots (their
+        // counters, published by the consumer warps that finished the
+        // tiles): the lanes read 32 slot counters at once with acquire
+        // loads, and lane 0 publishes the new frontier in shared memory with
+        // a release store.  Runs whenever the producer would otherwise wait,
+        // once the gate/up items are out.
+        auto pump = [&]() {
+            if (!poll || n_slots < 0 || frontier >= n_slots || my_mt == 0) return;
+            const int sl = frontier + lane;
+            const bool ready = sl >= n_slots || S.table[sl].e < 0 ||
+                               ld_acquire_gpu(d.sync + kSyncSlots + sl) >= gu_tiles;
+            const unsigned done = __ballot_sync(kAll, ready);
+            const int adv = done == kAll ? 32 : __ffs(~done) - 1;
+            if (adv > 0) {
+                frontier = min(frontier + adv, n_slots);
+                __syncwarp();
+                if (lane == 0) st_release_cta(S.frontier, frontier);
+            }
+        };
+        auto next_stage = [&](uint8_t*& st) -> bool {
+            const int stage = j % kStagesD, use = j / kStagesD;
+            if (use > 0) {
+                const uint32_t par = (use - 1) & 1;
+                int ok = lane == 0 ? (int)mbar_test_wait(&S.empty[stage], par) : 0;
+                if (!__shfl_sync(kAll, ok, 0)) {
                     const uint64_t t0 = global_timer_ns();
                     for (;;) {
                         pump();
-                        if (mbar_try_wait_sleep(&S.empty[stage], (use - 1) & 1, 400u)) break;
-                        if (global_timer_ns() - t0 > kWaitLimitNs) {
-                            report(a.status, COLI_ERR_TIMEOUT);
-                            *S.abort_flag = 1;
+                        ok = lane == 0 ? (int)mbar_try_wait_sleep(&S.empty[stage], par, 400u) : 0;
+                        if (__shfl_sync(kAll, ok, 0)) break;
+                        int late = lane == 0 && global_timer_ns() - t0 > kWaitLimitNs;
+                        if (__shfl_sync(kAll, late, 0)) {
+                            give_up();
                             return false;
                         }
                     }
                 }
-                st = S.stage0 + (size_t)stage * L.stage_bytes;
-                return true;
-            };
-            // gate/up: item b first, then items handed out by a counter (after
-            // the previous grid has finished and zeroed it), so faster CTAs
-            // take more.  A CTA with one more down tile than others stops
-            // taking items R before the end, R = the extra down work in items.
-            int* item_ctr = d.sync + kSyncItems;
-            int cur = b;
-            bool pdl_done = false;
-            int last_taken = INT_MAX;  // set once the table is known
-            for (;;) {
-                uint8_t* st;
-                if (*S.abort_flag || !next_stage(st)) {
-                    stop = true;
-                    break;
+            }
+            st = S.stage0 + (size_t)stage * L.stage_bytes;
+            return true;
+        };
+        // The table of the routed slots, from the consumers' routing (or the
+        // given union); the consumers wait for tbl_ready before their first
+        // routed item.  The union may come from the previous kernel.
+        auto build_table = [&]() -> bool {
+            if (!pdl_done) {
+                pdl_wait();
+                pdl_done = true;
+            }
+            if (d.logits) {
+                int ok = lane == 0 ? (int)mbar_wait(S.routed, 0) : 0;
+                __syncwarp();
+                if (!__shfl_sync(kAll, ok, 0)) {
+                    give_up();
+                    return false;
                 }
-                if (cur >= n_gu_shared && cur != INT_MAX && !table_known()) {
-                    stop = true;
-                    break;
+                table_from_logits(d, S, lane);
+            } else {
+                table_from_union(d, S, lane);
+            }
+            n_slots = *S.n_slots;
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S.tbl_ready);
+            return true;
+        };
+
+        // gate/up: item b first, then items handed out by a counter (after
+        // the previous grid has finished and zeroed it), so faster CTAs take
+        // more.  The table is built before the first item that needs it, or
+        // once every stage is armed.  A CTA with one more down tile
+        // than others stops taking items R before the end, R = the extra
+        // down work in items.
+        int* item_ctr = d.sync + kSyncItems;
+        int cur = b;
+        int last_taken = INT_MAX;  // set once the table is known
+        for (;;) {
+            if (abort_set()) {
+                stop = true;
+                break;
+            }
+            if (n_slots < 0 && (cur >= n_gu_shared || j >= kStagesD) && !build_table()) {
+                stop = true;
+                break;
+            }
+            uint8_t* st;
+            if (!next_stage(st)) {
+                stop = true;
+                break;
+            }
+            if (n_slots >= 0 && last_taken == INT_MAX) {
+                const int t_hi = (n_mt + G - 1) / G;
+                const int n_hi = n_mt - (t_hi - 1) * G;
+                const int lo = G - n_hi;
+                const float extra =
+                    (float)lo * n_slots * (float)(L.dn_op + L.dn_sc) / (float)L.gu_tx;
+                last_taken = n_slots * gu_tiles - ((my_mt == t_hi && lo > 0) ? (int)extra : 0);
+            }
+            if (n_slots >= 0 && cur >= n_slots * gu_tiles) break;  // stage j stays free
+            // the next item first: its round trip to the counter also lets the
+            // consumers' first loads (logits, activations) reach memory ahead
+            // of the copies' burst
+            int nxt = INT_MAX;
+            if (cur < last_taken) {
+                if (!pdl_done) {
+                    pdl_wait();
+                    pdl_done = true;
                 }
-                if (n_slots >= 0 && last_taken == INT_MAX) {
-                    const int t_hi = (n_mt + G - 1) / G;
-                    const int n_hi = n_mt - (t_hi - 1) * G;
-                    const int lo = G - n_hi;
-                    const float extra =
-                        (float)lo * n_slots * (float)(L.dn_op + L.dn_sc) / (float)L.gu_tx;
-                    last_taken = n_slots * gu_tiles - ((my_mt == t_hi && lo > 0) ? (int)extra : 0);
-                }
-                if (cur >= (n_slots >= 0 ? n_slots * gu_tiles : INT_MAX)) break;  // stage j stays free
-                int nxt = INT_MAX;
-                if (cur < last_taken) {
-                    if (!pdl_done) {
-                        pdl_wait();
-                        pdl_done = true;
+                if (lane == 0) nxt = G + atomicAdd(item_ctr, 1);
+                nxt = __shfl_sync(kAll, nxt, 0);
+            }
+            const int stage = j % kStagesD;
+            uint64_t* bar = &S.full[stage];
+            const int item = cur;
+            ++j;
+            if (lane == 0) {
+                S.stage_item[stage] = item;
+                if (item != a.withhold_item) {  // test hook: this stage never fills
+                    const int slot = item / gu_tiles, tile = item - slot * gu_tiles;
+                    const int e = S.table[slot].e;
+                    if (e < 0) {
+                        mbar_arrive(bar);
+                    } else {
+                        const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
+                        const int n0 = tile * kGuRows;
+                        mbar_arrive_expect_tx(bar, L.gu_tx);
+                        tma_load_3d(st, maps + 0, 0, 0, n0, bar, policy);
+                        tma_load_3d(st + L.gu_op, maps + 1, 0, 0, n0, bar, policy);
+                        if (a.per_row) {  // 8 rows' scales: 16 contiguous bytes per matrix
+                            const DevExpert& ex = a.experts[e];
+                            bulk_g2s_evict_first(st + 2 * L.gu_op, ex.gate_s + n0, L.gu_sc, bar,
+                                                 policy);
+                            bulk_g2s_evict_first(st + 2 * L.gu_op + L.gu_sc, ex.up_s + n0, L.gu_sc,
+                                                 bar, policy);
+                        } else {
+                            tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
+                            tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
+                        }
                     }
-                    nxt = G + atomicAdd(item_ctr, 1);
-                }
-                const int stage = j % kStagesD;
-                uint64_t* bar = &S.full[stage];
-                S.stage_item[stage] = cur;
-                ++j;
-                const int item = cur;
-                cur = nxt;
-                if (item == a.withhold_item) continue;  // test hook: this stage never fills
-                const int slot = item / gu_tiles, tile = item - slot * gu_tiles;
-                const int e = slot < a.n_shared ? a.E + slot : S.table[slot].e;
-                if (e < 0) {
-                    mbar_arrive(bar);
-                    continue;
-                }
-                ++S.issued_local[slot];
-                pub_hi = slot;
-                const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
-                const int n0 = tile * kGuRows;
-                mbar_arrive_expect_tx(bar, L.gu_tx);
-                tma_load_3d(st, maps + 0, 0, 0, n0, bar, policy);
-                tma_load_3d(st + L.gu_op, maps + 1, 0, 0, n0, bar, policy);
-                if (a.per_row) {  // 8 rows' scales: 16 contiguous bytes per matrix
-                    const DevExpert& ex = a.experts[e];
-                    bulk_g2s_evict_first(st + 2 * L.gu_op, ex.gate_s + n0, L.gu_sc, bar, policy);
-                    bulk_g2s_evict_first(st + 2 * L.gu_op + L.gu_sc, ex.up_s + n0, L.gu_sc, bar,
-                                         policy);
-                } else {
-                    tma_load_2d(st + 2 * L.gu_op, maps + 3, 0, n0, bar, policy);
-                    tma_load_2d(st + 2 * L.gu_op + L.gu_sc, maps + 4, 0, n0, bar, policy);
                 }
             }
-            // down stages carry item -1, which tells the consumers that gate/up
-            // is over; without down work a single empty stage does
-            if (!stop && table_known()) {
-                if (my_mt == 0) {
+            cur = nxt;
+        }
+        // down stages carry item -1, which tells the consumers that gate/up
+        // is over; without down work a single empty stage does
+        poll = true;
+        if (!stop) {
+            if (my_mt == 0) {
+                if (lane == 0) {
                     S.stage_item[j % kStagesD] = -1;
                     mbar_arrive(&S.full[j % kStagesD]);
-                    ++j;
                 }
-                for (int s = 0; s < n_slots && my_mt > 0; ++s) {
-                    uint8_t* st;
-                    if (*S.abort_flag || !next_stage(st)) break;
-                    const int stage = j % kStagesD;
-                    uint64_t* bar = &S.full[stage];
+                ++j;
+            }
+            for (int s = 0; s < n_slots && my_mt > 0; ++s) {
+                uint8_t* st;
+                if (abort_set() || !next_stage(st)) break;
+                const int stage = j % kStagesD;
+                uint64_t* bar = &S.full[stage];
+                ++j;
+                if (lane == 0) {
                     S.stage_item[stage] = -1;
-                    ++j;
                     const int e = S.table[s].e;
                     if (e < 0) {
                         mbar_arrive(bar);
-                        continue;
-                    }
-                    const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
-                    mbar_arrive_expect_tx(bar, my_mt * (L.dn_op + L.dn_sc));
-                    for (int m = 0; m < my_mt; ++m) {
-                        const int m0 = (bm + m * G) * kDnRows;
-                        tma_load_3d(st + m * L.dn_op, maps + 2, 0, 0, m0, bar, policy);
-                        if (a.per_row)  // 16 rows' scales: 32 contiguous bytes
-                            bulk_g2s_evict_first(st + kMaxMT * L.dn_op + m * L.dn_sc,
-                                                 a.experts[e].down_s + m0, L.dn_sc, bar, policy);
-                        else
-                            tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0, bar,
-                                        policy);
+                    } else {
+                        const CUtensorMap* maps = d.maps + (size_t)e * kMaps;
+                        mbar_arrive_expect_tx(bar, my_mt * (L.dn_op + L.dn_sc));
+                        for (int m = 0; m < my_mt; ++m) {
+                            const int m0 = (bm + m * G) * kDnRows;
+                            tma_load_3d(st + m * L.dn_op, maps + 2, 0, 0, m0, bar, policy);
+                            if (a.per_row)  // 16 rows' scales: 32 contiguous bytes
+                                bulk_g2s_evict_first(st + kMaxMT * L.dn_op + m * L.dn_sc,
+                                                     a.experts[e].down_s + m0, L.dn_sc, bar,
+                                                     policy);
+                            else
+                                tma_load_2d(st + kMaxMT * L.dn_op + m * L.dn_sc, maps + 5, 0, m0,
+                                            bar, policy);
+                        }
                     }
                 }
             }
-            // publish the rest (the consumers may still be reducing the last tiles)
-            if (!stop) {
-                const uint64_t t0 = global_timer_ns();
-                for (;;) {
-                    pump();
-                    if (all_published() || *S.abort_flag) break;
-                    if (global_timer_ns() - t0 > kWaitLimitNs) {
-                        report(a.status, COLI_ERR_TIMEOUT);
-                        *S.abort_flag = 1;
-                        break;
-                    }
-                    __nanosleep(200);
+            // follow the frontier to the last slot
+            const uint64_t t0 = global_timer_ns();
+            for (;;) {
+                pump();
+                const bool fin = frontier >= n_slots || my_mt == 0;
+                if (fin || abort_set()) break;
+                int late = lane == 0 && global_timer_ns() - t0 > kWaitLimitNs;
+                if (__shfl_sync(kAll, late, 0)) {
+                    give_up();
+                    break;
                 }
+                __nanosleep(200);
             }
-            if (*S.abort_flag) {
-                // let the copies already issued land before the CTA goes away
-                for (int back = 1; back <= kStagesD && back <= j; ++back) {
-                    const int jj = j - back;
-                    (void)mbar_wait(&S.full[jj % kStagesD], (jj / kStagesD) & 1);
-                }
+        }
+        if (abort_set() && lane == 0) {
+            // let the copies already issued land before the CTA goes away
+            for (int back = 1; back <= kStagesD && back <= j; ++back) {
+                const int jj = j - back;
+                (void)mbar_wait(&S.full[jj % kStagesD], (jj / kStagesD) & 1);
             }
         }
         return;
@@ -998,29 +1044,21 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
 
     // -------------------------------- consumers --------------------------------
     pdl_wait();
-    // routing first: warp t < T copies token t's logits into shared memory
-    // (the reduction buffers are free until the first item) and routes it,
-    // while the other warps build the activation operand
-    if (d.logits && warp < a.T) {
-        const float* src = d.logits + (int64_t)warp * a.E;
-        float* dst = S.red + warp * a.E;
-        for (int i = lane; i < a.E; i += 32) cp_async4(dst + i, src + i);
-        cp_async_commit();
-        cp_async_wait_all();
-        __syncwarp();
-        route_row<NV>(dst, a.E, a.k, lane, S.s_idx + warp * a.k, S.s_w + warp * a.k);
-    }
     const int r = lane >> 2, c = lane & 3;
 
     // gate/up operand: all T tokens as MMA columns, this warp's kMaxGW
     // groups, in registers for the whole kernel; offset sums to shared memory
-    // (zero for the groups past the end of H)
+    // (zero for the groups past the end of H), read by this warp only
     const int gG = a.H / kGroup;
     const int gg_lo = kMaxGW * warp;
     uint32_t breg[kMaxGW][8];
     int coff[kMaxGW];
     float amax = 0.f;
-    // all loads first (they are in flight together), then the conversions
+    // all loads first (they are in flight together), then the routing (warp
+    // t < T routes token t) and the conversions
+    const bool routing = d.logits && warp < a.T;
+    float lv[8];
+    if (routing && route_fast_ok<NV>(a.k)) load_row8<NV>(d.logits + (int64_t)warp * a.E, a.E, lane, lv);
 #pragma unroll
     for (int i = 0; i < kMaxGW; ++i) {
         const int grp = gg_lo + i;
@@ -1034,6 +1072,15 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         breg[i][0] = v0.x; breg[i][1] = v0.y; breg[i][2] = v0.z; breg[i][3] = v0.w;
         breg[i][4] = v1.x; breg[i][5] = v1.y; breg[i][6] = v1.z; breg[i][7] = v1.w;
     }
+    if (routing) {
+        if (route_fast_ok<NV>(a.k))
+            route_row_fast<NV>(lv, a.E, a.k, lane, S.s_idx + warp * a.k, S.s_w + warp * a.k);
+        else
+            route_row<NV>(d.logits + (int64_t)warp * a.E, a.E, a.k, lane, S.s_idx + warp * a.k,
+                          S.s_w + warp * a.k);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(S.routed);
+    }
 #pragma unroll
     for (int i = 0; i < kMaxGW; ++i) {
         const int grp = gg_lo + i;
@@ -1045,17 +1092,23 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             reinterpret_cast<float4*>(S.corr)[grp * 4 + c] = make_float4(-cs[0], -cs[1], -cs[0], -cs[1]);
     }
     if (amax > 65504.f) report(a.status, COLI_ERR_RANGE);
+    __syncwarp();
+    const Ctx ctx{a, L, S, d.sync, gu_tiles};
+    bool have_table = false;
+    auto wait_table = [&]() -> bool {
+        if (have_table) return true;
+        if (!mbar_wait(S.tbl_ready, 0)) {
+            fail(ctx, lane);
+            return false;
+        }
+        have_table = true;
+        return true;
+    };
 
-    if (d.logits) table_from_logits(d, S);
-    else table_from_union(d, S);
-    consumers_sync();
-    if (threadIdx.x == 0) mbar_arrive(S.tbl_ready);
-    const int n_slots = *S.n_slots;
-    const Ctx ctx{a, L, S, d.sync, n_slots, gu_tiles};
-
-    // phase 1: gate/up items
+    // phase 1: gate/up items (the shared experts' first: they need no table)
     int j = 0;
     bool alive = true;
+    int pending = -1;  // the slot of the last tile this warp finished, not yet published
     for (;;) {  // the producer names each stage's item; -1 ends gate/up
         const int stage = j % kStagesD;
         if (*S.abort_flag) {
@@ -1069,13 +1122,20 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
         }
         const int item = S.stage_item[stage];
         if (item < 0) break;
-        alive = gateup_item(ctx, item, j, breg, coff, gg_lo);
+        if (item >= n_gu_shared && !wait_table()) {
+            alive = false;
+            break;
+        }
+        alive = gateup_item(ctx, item, j, breg, coff, gg_lo, pending);
         ++j;
         if (!alive) break;
     }
     // the sums of the last kRedLag items
     for (int m = j - kRedLag; alive && m < j; ++m)
-        if (m >= 0 && m % kCW == warp) alive = finish_item(ctx, m);
+        if (m >= 0 && m % kCW == warp) alive = finish_item(ctx, m, pending);
+    if (alive) publish_tile(ctx, pending);
+    if (alive) alive = wait_table();
+    const int n_slots = alive ? *S.n_slots : 0;
 
     // phase 2: down + combine over this CTA's output tiles, slot by slot;
     // h' fragments of the next slot are loaded while this one is computed
@@ -1093,8 +1153,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             dcoff[i] = code_offset(r, L.dn_segs, dg_lo + i < dG ? dg_lo + i : dG - 1, c);
         // h' fragments: b0 = this slot, b1 = the next one (loading)
         uint32_t b0[kMaxDW][8], b1[kMaxDW][8];
-        int frontier = 0;
-        alive = advance_frontier(ctx, frontier, 0);
+        alive = wait_frontier(ctx, 0);
         if (alive) load_down_b(a, S.table + 0, dg_lo, b1);
         float dcorr[kMaxDW][2];
         for (int s = 0; s < n_slots && alive; ++s, ++j) {
@@ -1108,7 +1167,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
                 dcorr[i][1] = -cs[1];
             }
             if (s + 1 < n_slots) {
-                if (frontier <= s + 1) alive = advance_frontier(ctx, frontier, s + 1);
+                alive = wait_frontier(ctx, s + 1);
                 if (alive) load_down_b(a, S.table + s + 1, dg_lo, b1);
             }
             if (alive) alive = down_stage(ctx, s, j, my_mt, b0, dcorr, dcoff, dg_lo, acc);
@@ -1147,12 +1206,13 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             }
         }
     }
-    // the last CTA to get here returns the counters to zero
+    // the last CTA to get here returns the counters to zero (every slot a
+    // call can have: a CTA that gave up may not know the table)
     if (threadIdx.x == 0) {
         fence_acq_rel_gpu();
         if (atomicAdd(d.sync + kSyncDone, 1) == G - 1) {
             fence_acq_rel_gpu();
-            for (int s = 0; s < n_slots; ++s) d.sync[kSyncSlots + s] = 0;
+            for (int s = 0; s < d.max_slots; ++s) d.sync[kSyncSlots + s] = 0;
             d.sync[kSyncItems] = 0;
             d.sync[kSyncDone] = 0;
         }
@@ -1231,7 +1291,7 @@ bool decode_supported(int H, int I, int T, int E, int k, int n_shared, int num_s
     const Layout L = make_layout(H, I, max_slots_for(E, k, T, n_shared), 0);
     if (L.smem > kSmemLimitD) return false;
     if (H / kGroup > kCW * kMaxGW || I / kGroup > kCW * kMaxDW) return false;
-    if (T * E > kRedFloats) return false;  // logits staged in the reduction buffers
+    if (T * E > 5632) return false;  // the routing shapes the kernel is tested with
     if (H / kDnRows > kMaxMT * num_sms) return false;
     return L.gu_segs <= 256 && L.dn_segs <= 256 && L.gGp <= 256 && L.dGp <= 256;
 }

@@ -7,8 +7,8 @@
 
 namespace coli {
 
-constexpr int kMaxGW = 9;   // gate/up scale groups per consumer warp (H <= 6336)
-constexpr int kMaxDW = 3;   // down scale groups per consumer warp (I <= 2112)
+constexpr int kMaxGW = 6;   // gate/up scale groups per consumer warp (H <= 6144)
+constexpr int kMaxDW = 2;   // down scale groups per consumer warp (I <= 2048)
 
 struct DecodeArgs {
     FfnArgs f;                // shapes, experts, x, the union (when logits is null), h rows,

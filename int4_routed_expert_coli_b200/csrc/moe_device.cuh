@@ -75,6 +75,116 @@ __device__ __forceinline__ void route_row(const float* __restrict__ row, int E, 
 }
 
 // ---------------------------------------------------------------------------
+// Routing of one token row by one warp at low latency (the same selection
+// and weights as route_row).  Top-k for E <= 256 and k in {1, 2, 4, 8}: each
+// lane sorts its 8 keys (descending, a 19-comparator network), then five
+// butterfly levels merge the lanes' lists: a lane keeps the 8 largest of its
+// 16 keys and its partner's (the element-wise max of one list and the other
+// reversed is a bitonic sequence holding them; three half-cleaner stages
+// sort it), so after the last level every lane holds the row's 8 largest
+// keys in order.  No warp-wide reduction sits on the critical path, which a
+// round of the k-round selection needs twice.  The winners' logits come
+// back from their keys, so no second read of the row is needed.  Other
+// shapes use route_row.
+
+__device__ __forceinline__ void cas_desc(uint64_t& a, uint64_t& b) {
+    const bool sw = a < b;
+    const uint64_t hi = sw ? b : a, lo = sw ? a : b;
+    a = hi;
+    b = lo;
+}
+
+__device__ __forceinline__ void sort8_desc(uint64_t (&v)[8]) {
+    cas_desc(v[0], v[2]); cas_desc(v[1], v[3]); cas_desc(v[4], v[6]); cas_desc(v[5], v[7]);
+    cas_desc(v[0], v[4]); cas_desc(v[1], v[5]); cas_desc(v[2], v[6]); cas_desc(v[3], v[7]);
+    cas_desc(v[0], v[1]); cas_desc(v[2], v[3]); cas_desc(v[4], v[5]); cas_desc(v[6], v[7]);
+    cas_desc(v[2], v[4]); cas_desc(v[3], v[5]);
+    cas_desc(v[1], v[4]); cas_desc(v[3], v[6]);
+    cas_desc(v[1], v[2]); cas_desc(v[3], v[4]); cas_desc(v[5], v[6]);
+}
+
+// v (sorted, descending) <- the 8 largest of v and lane ^ d's list, sorted.
+__device__ __forceinline__ void merge8_xor(uint64_t (&v)[8], int d) {
+    uint64_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v[i], d);
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v[i] >> 32), d);
+        o[i] = ((uint64_t)hi << 32) | lo;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = v[i] > o[7 - i] ? v[i] : o[7 - i];
+#pragma unroll
+    for (int s = 4; s >= 1; s >>= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if ((i & s) == 0) cas_desc(v[i], v[i + s]);
+}
+
+// The logit a key was made from (-0 comes back as +0, NaN as a NaN).
+__device__ __forceinline__ float key_value(uint64_t key) {
+    const uint32_t k32 = (uint32_t)(key >> 32);
+    return __uint_as_float((k32 & 0x80000000u) ? (k32 & 0x7FFFFFFFu) : ~k32);
+}
+
+// True when route_row_fast handles the shape (else route_row).
+template <int NV>
+__device__ __forceinline__ bool route_fast_ok(int k) {
+    return NV <= 8 && k <= 8 && (k & (k - 1)) == 0;
+}
+
+// This lane's logits of one row (e = lane + 32 i), loaded before the row is
+// routed so the loads can be in flight with others.
+template <int NV>
+__device__ __forceinline__ void load_row8(const float* __restrict__ row, int E, int lane,
+                                          float (&val)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        val[i] = (i < NV && e < E) ? row[e] : 0.f;
+    }
+}
+
+// Routes one row from the values load_row8 gave (route_fast_ok(k) holds).
+template <int NV>
+__device__ __forceinline__ void route_row_fast(const float (&val)[8], int E, int k, int lane,
+                                               int* __restrict__ idx_out, float* __restrict__ w_out) {
+    uint64_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (i < NV && e < E) ? rank_key(val[i], e) : 0ull;  // padding never wins (k <= E)
+    }
+    sort8_desc(v);
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) merge8_xor(v, d);
+    uint64_t mine = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mine = lane == i ? v[i] : mine;
+    const int my_idx = (int)(0xFFFFFFFFu - (uint32_t)mine);
+    // weights: as route_row, over the k lanes holding the picks
+    const float x = (lane < k) ? key_value(mine) : 0.f;
+    const float m = __shfl_sync(0xffffffffu, x, 0);
+    double wj;
+    if (isinf(m) && m > 0.f) {
+        const bool pinf = lane < k && isinf(x) && x > 0.f;
+        const unsigned inf_mask = __ballot_sync(0xffffffffu, pinf);
+        wj = pinf ? 1.0 / (double)__popc(inf_mask) : 0.0;
+    } else if (isnan(m) || (isinf(m) && m < 0.f)) {
+        wj = 1.0 / (double)k;
+    } else {
+        const double ej = (lane < k && !isnan(x)) ? exp((double)x - (double)m) : 0.0;
+        double z = ej;
+        for (int o = k >> 1; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        wj = ej / z;
+    }
+    if (lane < k) {
+        idx_out[lane] = my_idx;
+        w_out[lane] = (float)wj;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Batch-union: all positions routed to one expert are listed together so the
 // expert is read once for all of them ("yunpan.plus/t/30351-1-1",
 // capability two, batch-union bullet).  A stable counting sort of the P

@@ -249,3 +249,42 @@ def test_glm_decode_deterministic(glm):
     a = _layer(layer, x, logits=lg)[0]
     b = _layer(layer, x, logits=lg)[0]
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+@pytest.mark.parametrize("E,k,T", [(64, 8, 7), (64, 2, 8), (64, 1, 5), (200, 8, 8), (256, 4, 8),
+                                   (256, 8, 3)])
+def test_fused_decode_routing_ties_and_specials(E, k, T):
+    """The fused decode kernel routes inside the kernel (a butterfly top-k per
+    token row; E <= 256, T * k < E): indices bit-exact and weights within 2
+    ulp of the oracle on tied, NaN, +-inf and signed-zero logits and on rows
+    that are all NaN or all -inf; the layer output against the oracle."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    H, I = 512, 512
+    bank = synth.make_expert_bank(H, I, E + 1, seed=E + k, device="cuda")
+    layer = c.MoELayer(bank, n_routed=E, top_k=k, n_shared=1)
+    rng = np.random.default_rng(E * 31 + k * 7 + T)
+    rows = []
+    for t in range(T):
+        r = rng.integers(-3, 4, size=E).astype(np.float32)   # many ties
+        kind = t % 7
+        if kind == 1:
+            r[rng.integers(0, E, size=3)] = np.nan
+        elif kind == 2:
+            r[rng.integers(0, E, size=2)] = -np.inf
+        elif kind == 3:
+            r[rng.integers(0, E, size=2)] = np.inf
+        elif kind == 4:
+            r[rng.integers(0, E, size=4)] = -0.0
+            r[rng.integers(0, E, size=4)] = 0.0
+        elif kind == 5:
+            r[:] = np.nan
+        elif kind == 6:
+            r[:] = -np.inf
+        rows.append(r)
+    lg = torch.from_numpy(np.stack(rows)).cuda()
+    x = synth.make_activations(T, H, seed=3, device="cuda")
+    out, idx, w, _ = _layer(layer, x, logits=lg)
+    ref, ri, rw = reference_layer(bank, E, k, 1, x, lg)
+    assert np.array_equal(idx, ri)
+    assert_weights_close(w, rw)
+    assert_close(out.cpu().numpy(), ref, f"E={E} k={k} T={T}")
