@@ -512,8 +512,9 @@ __device__ __forceinline__ void publish_tile(const Ctx& x, int pending) {
 // depend on timing) and its epilogue h' = w * silu(g) * u for the slot's
 // tokens, by warp m % kCW kRedLag items later: off the critical path of the
 // warp that finished item m last.  The tile this warp finished before is
-// published first; this one becomes `pending`.  false: timeout or abort.
-__device__ bool finish_item(const Ctx& x, int m, int& pending) {
+// published first; this one becomes `pending`, stored at item `at`.
+// false: timeout or abort.
+__device__ bool finish_item(const Ctx& x, int m, int& pending, int& pending_at, int at) {
     const FfnArgs& a = x.a;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int rb = m % kRedBufs;
@@ -551,6 +552,7 @@ __device__ bool finish_item(const Ctx& x, int m, int& pending) {
     if (en->e < 0) return true;
     publish_tile(x, pending);
     pending = slot;
+    pending_at = at;
     const float v[4] = {sum.x, sum.y, sum.z, sum.w};
     const int n = tile * kGuRows + r;
     const int hcol = (n / kGroup) * kGroup + perm64(n % kGroup);
@@ -580,7 +582,8 @@ __device__ bool finish_item(const Ctx& x, int m, int& pending) {
 // Returns false when the kernel must wind down.
 __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
                                             const uint32_t (&breg)[kMaxGW][8],
-                                            const int (&coff)[kMaxGW], int g_lo, int& pending) {
+                                            const int (&coff)[kMaxGW], int g_lo, int& pending,
+                                            int& pending_at) {
     const int slot = item / x.gu_tiles;
     const Layout& L = x.L;
     const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
@@ -647,7 +650,8 @@ __device__ __forceinline__ bool gateup_item(const Ctx& x, int item, int j,
         return false;
     }
     const int m = j - kRedLag;
-    if (m >= 0 && m % kCW == (int)(threadIdx.x >> 5)) return finish_item(x, m, pending);
+    if (m >= 0 && m % kCW == (int)(threadIdx.x >> 5))
+        return finish_item(x, m, pending, pending_at, j);
     return true;
 }
 
@@ -1109,6 +1113,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
     int j = 0;
     bool alive = true;
     int pending = -1;  // the slot of the last tile this warp finished, not yet published
+    int pending_at = 0;  // the item this warp was at when it stored that tile
     for (;;) {  // the producer names each stage's item; -1 ends gate/up
         const int stage = j % kStagesD;
         if (*S.abort_flag) {
@@ -1126,13 +1131,18 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_fused_kernel(const Decode
             alive = false;
             break;
         }
-        alive = gateup_item(ctx, item, j, breg, coff, gg_lo, pending);
+        // a tile stored two items ago goes out now (its stores are complete)
+        if (pending >= 0 && j >= pending_at + 2) {
+            publish_tile(ctx, pending);
+            pending = -1;
+        }
+        alive = gateup_item(ctx, item, j, breg, coff, gg_lo, pending, pending_at);
         ++j;
         if (!alive) break;
     }
     // the sums of the last kRedLag items
     for (int m = j - kRedLag; alive && m < j; ++m)
-        if (m >= 0 && m % kCW == warp) alive = finish_item(ctx, m, pending);
+        if (m >= 0 && m % kCW == warp) alive = finish_item(ctx, m, pending, pending_at, j);
     if (alive) publish_tile(ctx, pending);
     if (alive) alive = wait_table();
     const int n_slots = alive ? *S.n_slots : 0;
