@@ -162,12 +162,20 @@ coli_status coli_moe_route(int32_t T, int32_t E, int32_t k, const float *logits,
  * Deterministic: positions come from scans, never from atomic tickets.
  * `ws` may be NULL; if given (at least COLI_WS_HEADER_BYTES), an index
  * outside [0, E) is recorded in its status word (the pair is dropped from
- * the lists).
+ * the lists).  With at least coli_moe_union_workspace_size(T, E, k) bytes,
+ * a batch of 4096 or more pairs is split over several CTAs (per-CTA counts
+ * past the header); the lists are the same, bit for bit.
  * Errors: INVALID_ARG, SHAPE (as coli_moe_route; T*k > 2^24). */
 coli_status coli_moe_union(int32_t T, int32_t E, int32_t k, const int32_t *topk_idx,
                            int32_t *counts, int32_t *offsets, int32_t *pairs,
                            int32_t *active, int32_t *n_active, void *ws, size_t ws_bytes,
                            void *stream);
+
+/* Workspace bytes with which coli_moe_union splits a large batch over
+ * several CTAs (COLI_WS_HEADER_BYTES when the batch is not split); 0 for
+ * T < 0, E < 1 or k < 1.  A library addition, not an operation of the
+ * pages. */
+size_t coli_moe_union_workspace_size(int32_t T, int32_t E, int32_t k);
 
 /* Expert FFN over a prepared batch-union (steps 3-5): every active expert's
  * weights are streamed once for all tokens on its list; the shared experts

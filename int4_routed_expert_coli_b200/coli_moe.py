@@ -35,7 +35,8 @@ COLI_OUT_BF16 = 1
 COLI_GROUP_PER_ROW = 0  # coli_moe_desc.group_size of the per-row int4 format
 
 EXPORTS = ("coli_moe_create", "coli_moe_destroy", "coli_moe_workspace_size",
-           "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union", "coli_moe_ffn",
+           "coli_moe_workspace_clear", "coli_moe_route", "coli_moe_union",
+           "coli_moe_union_workspace_size", "coli_moe_ffn",
            "coli_moe_layer", "coli_moe_layer_noalloc", "coli_moe_combine_rows",
            "coli_moe_prefetch",
            "coli_moe_get_status",
@@ -81,6 +82,8 @@ def _load():
     L.coli_moe_route.restype = ctypes.c_int
     L.coli_moe_union.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, sz, P]
     L.coli_moe_union.restype = ctypes.c_int
+    L.coli_moe_union_workspace_size.argtypes = [i32, i32, i32]
+    L.coli_moe_union_workspace_size.restype = sz
     L.coli_moe_ffn.argtypes = [P, i32, P, P, P, P, P, P, P, P, P, ctypes.c_int, P, sz, P]
     L.coli_moe_ffn.restype = ctypes.c_int
     L.coli_moe_layer.argtypes = [P, i32, P, P, P, P, P, ctypes.c_int, P, P, P, sz, P]
@@ -150,6 +153,10 @@ def coli_moe_union(T, E, k, topk_idx, counts, offsets, pairs, active, n_active, 
     s = lib.coli_moe_union(T, E, k, _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(pairs),
                            _ptr(active), _ptr(n_active), _ptr(ws), ws_bytes, _stream(stream))
     return _check(s, "coli_moe_union", raise_on_error)
+
+
+def coli_moe_union_workspace_size(T, E, k):
+    return int(lib.coli_moe_union_workspace_size(T, E, k))
 
 
 def coli_moe_ffn(handle, T, x, topk_w, counts, offsets, pairs, active, n_active, residual, out,

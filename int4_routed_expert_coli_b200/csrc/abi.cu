@@ -337,6 +337,11 @@ coli_status coli_moe_workspace_clear(void* ws, size_t ws_bytes, void* stream) {
     return from_cuda(cudaMemsetAsync(ws, 0, coli::kHeaderBytes, static_cast<cudaStream_t>(stream)));
 }
 
+size_t coli_moe_union_workspace_size(int32_t T, int32_t E, int32_t k) {
+    if (T < 0 || E < 1 || k < 1) return 0;
+    return coli::kHeaderBytes + coli::union_scratch_bytes((int64_t)T * k, E);
+}
+
 coli_status coli_moe_route(int32_t T, int32_t E, int32_t k, const float* logits,
                            int32_t* topk_idx, float* topk_w, void* stream) {
     coli_status s = check_route_dims(T, E, k);
@@ -358,10 +363,16 @@ coli_status coli_moe_union(int32_t T, int32_t E, int32_t k, const int32_t* topk_
     for (const void* p : ptrs)
         if (p && !aligned(p, 4)) return COLI_ERR_ALIGN;
     if (ws && (ws_bytes < coli::kHeaderBytes || !aligned(ws, 256))) return COLI_ERR_WORKSPACE;
+    // a workspace with room for the per-CTA counts past its header lets a
+    // large batch split over several CTAs
+    const size_t need = coli::union_scratch_bytes((int64_t)T * k, E);
+    int* scratch = (ws && need > 0 && ws_bytes >= coli::kHeaderBytes + need)
+                       ? reinterpret_cast<int*>(static_cast<char*>(ws) + coli::kHeaderBytes)
+                       : nullptr;
     // T == 0 still writes empty lists (counts 0, offsets 0, no active experts).
     return from_cuda(coli::launch_union(T, E, k, topk_idx, counts, offsets, pairs, active,
                                         n_active, nullptr, ws ? static_cast<int*>(ws) : nullptr,
-                                        static_cast<cudaStream_t>(stream)));
+                                        scratch, static_cast<cudaStream_t>(stream)));
 }
 
 coli_status coli_moe_ffn(const coli_moe* h, int32_t T, const void* x_bf16, const float* topk_w,
@@ -438,7 +449,7 @@ coli_status coli_moe_layer(const coli_moe* h, int32_t T, const void* x_bf16, con
         if (err == cudaSuccess) err = coli::launch_route(T, h->E, h->k, lg, idx, w, st);
         if (err == cudaSuccess)
             err = coli::launch_union(T, h->E, h->k, idx, counts, offsets, pairs, active, n_active,
-                                     a.inv, a.status, st);
+                                     a.inv, a.status, at<int>(ws, L.ucnt), st);
     }
     if (err == cudaSuccess) err = run_ffn(h, T, a, ws, st, T <= coli::kSmallT && !prefill);
     profile_end_call();

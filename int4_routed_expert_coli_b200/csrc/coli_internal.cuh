@@ -56,8 +56,23 @@ struct WsLayout {
     size_t y;        // [S][H] f32, per-(pair) expert outputs
     size_t xg;       // [T*k + T][H] f16, expert-sorted activations (tensor-core path)
     size_t ntile;    // [E + n_shared + 1] i32, token-tile prefix (tensor-core path)
+    size_t ucnt;     // [C][E] i32, per-CTA expert counts of the split batch-union
     size_t total;
 };
+
+// The batch-union of T*k >= kUnionSplitPairs pairs runs on C CTAs of
+// union_chunk(P) pairs each (a multiple of 1024, at most kUnionMaxCtas CTAs).
+constexpr int64_t kUnionSplitPairs = 4096;
+constexpr int64_t kUnionMaxCtas = 256;
+inline int64_t union_chunk(int64_t P) {
+    int64_t c = (P + kUnionMaxCtas - 1) / kUnionMaxCtas;
+    c = (c + 1023) / 1024 * 1024;
+    return c < 1024 ? 1024 : c;
+}
+inline int union_ctas(int64_t P) { return (int)((P + union_chunk(P) - 1) / union_chunk(P)); }
+inline size_t union_scratch_bytes(int64_t P, int E) {
+    return P >= kUnionSplitPairs ? sizeof(int) * (size_t)union_ctas(P) * (size_t)E : 0;
+}
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -85,6 +100,7 @@ inline WsLayout ws_layout(int64_t T, int E, int k, int H, int I, int n_shared) {
     L.y = take(sizeof(float) * S * H);
     L.xg = take(sizeof(uint16_t) * (P + T) * H);
     L.ntile = take(sizeof(int) * (E + n_shared + 2));
+    L.ucnt = take(union_scratch_bytes(P, E));
     L.total = o;
     return L;
 }
@@ -146,9 +162,11 @@ cudaError_t launch_router_logits(int T, int E, int H, const __nv_bfloat16* x, co
                                  float* logits, cudaStream_t st);
 cudaError_t launch_route(int T, int E, int k, const float* logits, int* idx, float* w,
                          cudaStream_t st);
+// `scratch` (nullable, union_scratch_bytes): with it, T*k >= kUnionSplitPairs
+// pairs are split over several CTAs (two launches); the lists are the same.
 cudaError_t launch_union(int T, int E, int k, const int* idx, int* counts, int* offsets,
                          int* pairs, int* active, int* n_active, int* inv, int* status,
-                         cudaStream_t st);
+                         int* scratch, cudaStream_t st);
 cudaError_t launch_prep_small(const PrepArgs& p, cudaStream_t st);
 cudaError_t launch_ffn_stream(const FfnArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_prepare_x(int T, int H, const __nv_bfloat16* x, __half* xp, float* corr,

@@ -1,6 +1,14 @@
-// Batch-union kernel (device body in moe_device.cuh) and the fused
+// Batch-union kernels (device body in moe_device.cuh) and the fused
 // preparation kernel for small batches: routing, batch-union, the inverse
 // pair map and the activation permutation in a single launch.
+//
+// Large batches (T*k >= kUnionSplitPairs) split the union over C CTAs of a
+// contiguous pair range each, in two launches: every CTA counts its pairs
+// per expert (per-warp histograms, one leader per distinct expert in a
+// 32-pair slice); then every CTA reads all CTAs' counts, scans them
+// (expert-major, then CTA, then warp) and writes its pairs at
+// base + rank-among-equal-keys.  The lists are those of the one-CTA union:
+// inside an expert, pairs ascend.
 #include "moe_device.cuh"
 #include "ptx.cuh"
 
@@ -51,21 +59,151 @@ prep_small_kernel(PrepArgs p) {
     }
 }
 
+// Per-warp histograms of pairs [lo, hi) of this warp (hist[warp][E], zeroed
+// by the caller); invalid indices count nowhere and, with `status`, are
+// reported.
+__device__ __forceinline__ void warp_hist(int lo, int hi, int E, const int* __restrict__ idx,
+                                          int* my_hist, int* status) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int p0 = lo; p0 < hi; p0 += 32) {
+        const int p = p0 + lane;
+        int e = p < hi ? idx[p] : -1;
+        if (p < hi && (e < 0 || e >= E)) {
+            if (status) report(status, COLI_ERR_BAD_INDEX);
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (peers & lt_mask) == 0) my_hist[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// Split union, launch 1: cta_cnt[c][e] = pairs of CTA c's range routed to e.
+__global__ void __launch_bounds__(kUnionThreads)
+union_count_kernel(int P, int E, int chunk, const int* __restrict__ idx, int* __restrict__ cta_cnt,
+                   int* status) {
+    extern __shared__ int hist[];
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kUnionWarps * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int wchunk = chunk / kUnionWarps;
+    const int lo = blockIdx.x * chunk + warp * wchunk;
+    warp_hist(lo, min(P, lo + wchunk), E, idx, hist + warp * E, status);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int n = 0;
+        for (int w = 0; w < kUnionWarps; ++w) n += hist[w * E + e];
+        cta_cnt[(int64_t)blockIdx.x * E + e] = n;
+    }
+}
+
+// Split union, launch 2: every CTA scans all CTAs' counts and writes its
+// pairs; CTA 0 also writes counts, offsets, active and n_active.
+__global__ void __launch_bounds__(kUnionThreads)
+union_write_kernel(int P, int E, int chunk, int n_cta, const int* __restrict__ idx,
+                   const int* __restrict__ cta_cnt, int* __restrict__ counts,
+                   int* __restrict__ offsets, int* __restrict__ pairs, int* __restrict__ active,
+                   int* __restrict__ n_active, int* __restrict__ inv) {
+    extern __shared__ int hist[];
+    __shared__ int scan_tmp[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < kUnionWarps * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int wchunk = chunk / kUnionWarps;
+    const int lo = blockIdx.x * chunk + warp * wchunk;
+    const int hi = min(P, lo + wchunk);
+    int* my_hist = hist + warp * E;
+    warp_hist(lo, hi, E, idx, my_hist, nullptr);
+    __syncthreads();
+
+    const int e_self = threadIdx.x;  // E <= kUnionThreads
+    int total = 0, before = 0;
+    if (e_self < E) {
+        for (int c = 0; c < n_cta; ++c) {
+            const int n = cta_cnt[(int64_t)c * E + e_self];
+            total += n;
+            before += c < (int)blockIdx.x ? n : 0;
+        }
+    }
+    int all;
+    const int off = block_exclusive_scan(e_self < E ? total : 0, scan_tmp, &all);
+    int act_total;
+    const int act_pos =
+        block_exclusive_scan((e_self < E && total > 0) ? 1 : 0, scan_tmp, &act_total);
+    if (e_self < E) {
+        int run = off + before;  // this CTA's first position of expert e_self
+        for (int w = 0; w < kUnionWarps; ++w) {
+            const int n = hist[w * E + e_self];
+            hist[w * E + e_self] = run;
+            run += n;
+        }
+        if (blockIdx.x == 0) {
+            counts[e_self] = total;
+            offsets[e_self] = off;
+            if (total > 0) active[act_pos] = e_self;
+        }
+    }
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) {
+            offsets[E] = all;
+            *n_active = act_total;
+        }
+        for (int e = act_total + threadIdx.x; e < E; e += blockDim.x) active[e] = -1;
+    }
+    __syncthreads();
+
+    for (int p0 = lo; p0 < hi; p0 += 32) {
+        const int p = p0 + lane;
+        int e = p < hi ? idx[p] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0) {
+            const int pos = my_hist[e] + __popc(peers & lt_mask);
+            pairs[pos] = p;
+            if (inv) inv[p] = pos;
+        } else if (p < hi && inv) {
+            inv[p] = -1;
+        }
+        __syncwarp();
+        if (e >= 0 && (peers & lt_mask) == 0) my_hist[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_union(int T, int E, int k, const int* idx, int* counts, int* offsets,
                          int* pairs, int* active, int* n_active, int* inv, int* status,
-                         cudaStream_t st) {
+                         int* scratch, cudaStream_t st) {
     const int P = T * k;
     const size_t smem = union_smem_bytes(E);
+    const bool split = scratch != nullptr && P >= kUnionSplitPairs && E <= kUnionThreads;
     if (smem > 48 * 1024) {
-        cudaError_t err = cudaFuncSetAttribute(union_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)smem);
+        cudaError_t err = split ? cudaFuncSetAttribute(union_count_kernel,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)smem)
+                                : cudaFuncSetAttribute(union_kernel,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)smem);
+        if (err == cudaSuccess && split)
+            err = cudaFuncSetAttribute(union_write_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
     }
-    union_kernel<<<1, kUnionThreads, smem, st>>>(P, E, idx, counts, offsets, pairs, active,
-                                                 n_active, inv, status);
+    if (!split) {
+        union_kernel<<<1, kUnionThreads, smem, st>>>(P, E, idx, counts, offsets, pairs, active,
+                                                     n_active, inv, status);
+        return cudaGetLastError();
+    }
+    const int chunk = (int)union_chunk(P), n_cta = union_ctas(P);
+    union_count_kernel<<<n_cta, kUnionThreads, smem, st>>>(P, E, chunk, idx, scratch, status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    union_write_kernel<<<n_cta, kUnionThreads, smem, st>>>(P, E, chunk, n_cta, idx, scratch,
+                                                           counts, offsets, pairs, active,
+                                                           n_active, inv);
     return cudaGetLastError();
 }
 

@@ -28,8 +28,14 @@ def _run(idx: np.ndarray, E: int, ws=None):
                 n_active=int(na.item()))
 
 
-def _check(idx, E):
-    got = _run(idx, E)
+def _check(idx, E, split=False):
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    ws = None
+    if split:  # a workspace with room for the per-CTA counts: large batches split
+        T, k = idx.shape
+        ws = torch.zeros(c.coli_moe_union_workspace_size(T, E, k), dtype=torch.uint8,
+                         device="cuda")
+    got = _run(idx, E, ws)
     ref = oracle.union(idx, E)
     for key in ("counts", "offsets", "pairs", "active"):
         assert np.array_equal(got[key], ref[key]), key
@@ -74,3 +80,51 @@ def test_union_deterministic():
     b = _run(idx, 256)
     for key in ("counts", "offsets", "pairs", "active"):
         assert np.array_equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("T,E,k", [(4096, 256, 8), (512, 256, 8), (4097, 256, 8), (20000, 1000, 8),
+                                   (70000, 1024, 32), (2048, 3, 2)])
+def test_union_split_over_ctas(T, E, k):
+    """Batches of 4096 or more pairs with a workspace for the per-CTA counts
+    take the split union (several CTAs, two launches): the same lists, bit for
+    bit, including ragged last CTAs and CTAs with many pair slices."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    assert c.coli_moe_union_workspace_size(T, E, k) > c.COLI_WS_HEADER_BYTES or T * k < 4096
+    lg = np.random.default_rng(T * 3 + E).random((T, E), dtype=np.float32)
+    idx, _ = oracle.route(lg, k)
+    _check(idx, E, split=True)
+
+
+def test_union_split_zipf_and_all_to_one():
+    sets, logits = synth.zipf_routing(1024, 256, 8, steps=2, seed=9)
+    for lg in logits:
+        idx, _ = oracle.route(lg, 8)
+        _check(idx, 256, split=True)
+    _check(np.tile(np.arange(8, dtype=np.int32), (4096, 1)), 256, split=True)
+
+
+def test_union_split_bad_index_reported():
+    """An index outside [0, E) in a split batch: reported in the status word
+    and the pair dropped; the lists are the definition's (a stable sort of
+    the valid pairs by expert), computed here by brute force."""
+    from int4_routed_expert_coli_b200 import coli_moe as c
+    T, E, k = 1024, 256, 8
+    lg = np.random.default_rng(11).random((T, E), dtype=np.float32)
+    idx, _ = oracle.route(lg, k)
+    idx = idx.copy()
+    idx[700, 3] = 5000
+    idx[1000, 0] = -2
+    ws = torch.zeros(c.coli_moe_union_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
+    got = _run(idx, E, ws)
+    assert c.coli_moe_get_status(ws) == c.COLI_ERR_BAD_INDEX
+    flat = idx.ravel()
+    valid = (flat >= 0) & (flat < E)
+    counts = np.bincount(flat[valid], minlength=E)
+    n = int(valid.sum())
+    assert np.array_equal(got["counts"], counts)
+    assert np.array_equal(got["offsets"], np.concatenate([[0], np.cumsum(counts)]))
+    order = np.argsort(np.where(valid, flat, E), kind="stable")
+    assert np.array_equal(got["pairs"][:n], order[:n])
+    act = np.nonzero(counts)[0]
+    assert got["n_active"] == len(act)
+    assert np.array_equal(got["active"], np.concatenate([act, -np.ones(E - len(act), np.int64)]))
