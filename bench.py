@@ -78,19 +78,12 @@ PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 # workload -> (source file, sha256, bytes per unit, unit, how it was measured)
 _DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
                "fe5733e351aa296cfbdb8fe7dbcff3d1c947ef884e1702defe6aad80d9300fee")
-_GEMM_SRC = ("int4_routed_expert_coli_b200/csrc/prefill.cu",
-             "896bf7fc35acc8db8115674e96ccda327433d88f3880fd31f647173a8a1185f3")
-_GEMM_SMALL = (*_GEMM_SRC, 13_692_332, "streamed expert",
-               "ncu launch list, 12 launches of the small-tile gate/up GEMM on a 64-expert "
-               "bank at T=32: bytes per streamed expert (unique routed + shared)")
 DRAM_TRAFFIC = {
     "decode": (*_DECODE_SRC, 184_230_741, "launch",
                "ncu launch list, 18 launches of the fused decode kernel on a 64-expert bank "
                "(a T=1 step streams 8 + 1 experts on any bank)"),
     "verify4": (*_DECODE_SRC, 184_230_741 // 9, "streamed expert",
                 "the T=1 fused-kernel capture, bytes per streamed expert"),
-    "batch32": _GEMM_SMALL,
-    "stack": _GEMM_SMALL,
 }
 
 
@@ -550,7 +543,8 @@ def run_stack(args, rank, world, local, with_cpu=True):
                    "parallelism": f"replicas x{world}"},
         "achieved_gbs_step": step_bytes / (total_ms / args.steps / 1e3) / 1e9,
         "roofline": {"bound": "hbm",
-                     "kernel": "gateup_kernel" if T * k < E else "prefill_gemm_kernel<gate/up>",
+                     "kernel": "decode_fused_kernel" if T <= 8 and T * k < E
+                     else "batch_ffn_kernel<gate/up>" if T <= 64 else "prefill_gemm_kernel<gate/up>",
                      "achieved": achieved,
                      "peak": P["hbm"], "unit": "GB/s", "frac": achieved / P["hbm"],
                      "peak_source": P["src"], "traffic": traffic, "traffic_source": traffic_src,
@@ -566,8 +560,8 @@ def run_stack(args, rank, world, local, with_cpu=True):
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
-        "gpu_launches": (1 if T <= 8 and T * k < E else 7 if T * k >= 4096 else 6)
-        * L * args.steps,
+        "gpu_launches": (1 if T <= 8 and T * k < E else 4 if T <= 64 else 7 if T * k >= 4096
+                         else 6) * L * args.steps,
         "clocks": clocks,
     }
     return line
@@ -699,9 +693,11 @@ def run_ours(args, rank, world, local, name, with_cpu=True):
     step_bytes = (n_uniq + n_sh) * expert_bytes(H, I)
     # dominant kernel: up to 8 tokens with T*k < E the fused decode kernel
     # (routing, gate/up, down and combine; it streams every active expert
-    # whole), otherwise the gate/up kernel of the tensor-core grouped GEMM (the
-    # library's default for every call the fused kernel does not take)
+    # whole), other calls of up to 64 tokens the small-batch gate/up kernel,
+    # larger ones the gate/up kernel of the tensor-core grouped GEMM (the
+    # library's default paths)
     fused = T <= 8 and T * k < E
+    small = not fused and T <= 64
     tensor = kind == "uniform"  # prefill: tensor-bound
     k_ms = phase_ms[1] / max(n_calls, 1)
     traffic, traffic_src = traffic_for(name, n_uniq + n_sh)
@@ -718,7 +714,8 @@ def run_ours(args, rank, world, local, name, with_cpu=True):
         k_bytes = step_bytes if fused else (n_uniq + n_sh) * gateup_bytes(H, I)
         achieved = k_bytes / (k_ms / 1e3) / 1e9
         roof = {"bound": "hbm",
-                "kernel": "decode_fused_kernel" if fused else "prefill_gemm_kernel<gate/up>",
+                "kernel": "decode_fused_kernel" if fused else "batch_ffn_kernel<gate/up>" if small
+                else "prefill_gemm_kernel<gate/up>",
                 "achieved": achieved, "peak": P["hbm"], "unit": "GB/s",
                 "frac": achieved / P["hbm"], "peak_source": P["src"],
                 "traffic": traffic, "traffic_source": traffic_src,
@@ -740,9 +737,11 @@ def run_ours(args, rank, world, local, name, with_cpu=True):
         "cpu_baseline": cpu,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 4},
-        # grouped-GEMM path: route, union (two launches from 4096 pairs on),
-        # gather, gate/up, down, combine
-        "gpu_launches": (1 if fused else 7 if T * k >= 4096 else 6) * args.steps,
+        # small-batch path: preparation (routing, union, activation operand),
+        # gate/up, down, combine; grouped-GEMM path: route, union (two launches
+        # from 4096 pairs on), gather, gate/up, down, combine
+        "gpu_launches": (1 if fused else 4 if small else 7 if T * k >= 4096 else 6)
+        * args.steps,
         "clocks": clocks,
     }
     return line

@@ -110,12 +110,13 @@ typedef struct {
     const coli_expert *experts; /* host array, n_routed + n_shared entries */
     int32_t prefill_min_tokens; /* T*k/E at or above which the tensor-core
                                    grouped GEMM is used; 0 = library default:
-                                   the grouped GEMM for every call the fused
-                                   decode kernel does not take (more than 8
-                                   tokens, T*k >= E, or a shape it does not
-                                   support); a positive value: calls with
-                                   T*k >= value * E, the streaming kernels for
-                                   the rest the fused kernel does not take */
+                                   the fused decode kernel where it applies
+                                   (T <= 8, T*k < E), the small-batch kernels
+                                   for the other calls of up to 64 tokens, the
+                                   grouped GEMM above; a positive value: calls
+                                   with T*k >= value * E, the streaming kernels
+                                   for the rest the fused kernel does not
+                                   take */
 } coli_moe_desc;
 
 #define COLI_GROUP_PER_ROW 0 /* group_size of the per-row int4 format */

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "coli_internal.cuh"
+#include "batch.cuh"
 #include "decode.cuh"
 #include "handle.cuh"
 #include "prefill.cuh"
@@ -125,11 +126,18 @@ bool fused_ok(const coli_moe* h, int64_t T) {
            coli::decode_supported(h->H, h->I, (int)T, h->E, h->k, h->n_shared, h->num_sms);
 }
 
+// True when a call with T tokens runs the small-batch kernels (the default
+// for calls of up to 64 tokens the fused decode kernel does not take).
+bool use_batch(const coli_moe* h, int64_t T) {
+    return h->d_wmaps != nullptr && h->prefill_min == 0 && !fused_ok(h, T) &&
+           coli::batch_supported(h->H, h->I, (int)T);
+}
+
 // True when a call with T tokens runs the tensor-core grouped GEMM.
 bool use_prefill(const coli_moe* h, int64_t T) {
     if (h->d_wmaps == nullptr) return false;
     if (h->prefill_min > 0) return T * h->k >= (int64_t)h->prefill_min * h->E;
-    return !fused_ok(h, T);
+    return !fused_ok(h, T) && !use_batch(h, T);
 }
 
 // True when a call with T tokens runs the fused decode kernel.
@@ -162,6 +170,13 @@ cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* 
     if (use_prefill(h, T)) {
         err = coli::launch_prefill(a, h->d_wmaps, at<__half>(ws, L.xg), at<int>(ws, L.ntile),
                                    h->num_sms, st);
+        if (err == cudaSuccess) err = coli::launch_combine(a, h->num_sms, st);
+        coli::profile_mark(4, st);
+        return err;
+    }
+    if (use_batch(h, T)) {
+        if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
+        if (err == cudaSuccess) err = coli::launch_batch_ffn(a, h->d_wmaps, h->num_sms, st);
         if (err == cudaSuccess) err = coli::launch_combine(a, h->num_sms, st);
         coli::profile_mark(4, st);
         return err;

@@ -1,0 +1,465 @@
+// Small-batch expert FFN: every call with up to 64 tokens that the fused
+// decode kernel does not take (more than 8 tokens, or T*k >= E).
+//
+// With a few tokens per expert, each active expert's weights are streamed
+// once for its token list (the batch-union, "yunpan.plus/t/30351-1-1",
+// capability two), and the arithmetic is the fused decode kernel's: codes
+// unpacked raw in registers (1032 + q at even k, 1152 + 16 q at odd k, whose
+// activations enter divided by 16), m16n8k16 MMAs with the activation
+// fragments as 8-token column tiles, the unpack's offset sums from an MMA of
+// its constant part with the same fragments as each chain's initial value,
+// fp32 accumulation, each group's bf16 scale applied to the group's partial.
+// The weights never pass through shared-memory operands of the tensor cores
+// or tensor memory: at a few tokens per expert the grouped GEMM's fp16
+// operand costs more on-chip traffic than HBM delivers.
+//
+// Tiles.  A tile is 256 weight rows of one expert over the whole reduction
+// dimension and up to 32 entries of its token list: for gate/up the gate and
+// the up rows of 128 features, for down 256 rows of W_d.  Each of 16
+// consumer warps owns 16 rows (gate/up: 8 gate and the 8 up rows of the same
+// features, so SwiGLU happens in registers) and runs the whole K loop: no
+// partial sums cross warps.  A list of more than 32 tokens (calls with more
+// than 32 tokens: the shared experts, popular routed ones) is split into two
+// column chunks, each a tile of its own that reads the rows again.  Tiles are
+// dealt to the CTAs (one per SM) round-robin, slot-major (shared experts
+// first).
+//
+// Data movement.  A producer warp stages four 64-element K-blocks at a time
+// in a ring of 4 stages of 49 KB: the codes of the tile's rows by 2-D tensor
+// copies (128 rows x 32 bytes each), each token's 256 activations (fragment
+// order, 512 bytes) by a 1-D bulk copy into a row of 528 bytes (the padding
+// spreads the fragment reads over the banks), and for gate/up each token's 4
+// precomputed offset sums (16 bytes).  The activations are, for gate/up, the
+// prepared x rows of the list's tokens, whose offset sums the preparation
+// computed; for down, the h' rows that the gate/up kernel wrote (odd features
+// / 16), whose offset sums an MMA computes from the fragments.  Scales are
+// read by the consumers from global memory, eight K-blocks at a time, a chunk
+// ahead.
+//
+// Every wait is bounded (COLI_ERR_TIMEOUT).
+#include <cuda.h>
+
+#include "batch.cuh"
+#include "mma_frag.cuh"
+#include "moe_device.cuh"
+#include "ptx.cuh"
+
+namespace coli {
+namespace {
+
+constexpr int kBW = 16;                               // consumer warps
+constexpr int kBThreads = (kBW + 1) * 32;             // + producer warp
+constexpr int kTileRows = 16 * kBW;                   // weight rows per tile
+constexpr int kBoxRows = 128;                         // rows per tensor copy
+constexpr int kChunkTok = 32;                         // list entries per tile
+constexpr int kMaxNT = kChunkTok / 8;                 // 8-token column tiles
+constexpr int kChunks = kBatchMaxTokens / kChunkTok;  // column chunks of a list
+constexpr int kKBS = 4;                               // K-blocks (scale groups) per stage
+constexpr int kBlockBytes = kTileRows * 32;           // codes of one K-block (two boxes)
+constexpr int kCodeBytes = kKBS * kBlockBytes;
+constexpr int kActRow = kKBS * 128 + 16;              // staged activation row (bytes)
+constexpr int kCorrOff = kCodeBytes + kChunkTok * kActRow;  // offset sums, 16 B per token
+constexpr int kStageB = kCorrOff + kChunkTok * 16;
+constexpr int kHdrB = 1024;
+constexpr int kSmemLimitB = 227 * 1024;
+constexpr int kStagesB = 4;
+constexpr int kSmemB = kHdrB + kStagesB * kStageB + 1024;  // 1024: alignment slack
+constexpr unsigned kAllB = 0xffffffffu;
+static_assert(kSmemB <= kSmemLimitB, "stage ring");
+static_assert(kChunkTok <= 32, "one activation row per producer lane");
+static_assert(kActRow % 16 == 0 && kStageB % 16 == 0 && kCorrOff % 16 == 0, "bulk copy alignment");
+// a staged activation row of 33 16-byte units: the 8 lanes of a quarter-warp
+// (rows r, r + 1; units 2c .. 2c + 1) fall on distinct bank groups
+static_assert((kActRow / 16) % 8 == 1, "activation row stride");
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ void tma_2d_hint(void* dst, const void* tmap, int c0, int c1,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// One expert slot of the call: shared experts first (every token, weight 1),
+// then the active routed experts in the union's order.
+struct BSlot {
+    int e;           // expert row in the device table
+    int list_begin;  // first h / y row of the slot's token list
+    int ntok;        // tokens on the list
+    bool shared;
+    bool valid;      // false: an inconsistent union entry (reported, skipped)
+};
+
+__device__ __forceinline__ BSlot batch_slot(const FfnArgs& a, int slot) {
+    BSlot s;
+    const int P = a.T * a.k;
+    if (slot < a.n_shared) {
+        s.e = a.E + slot;
+        s.list_begin = P + slot * a.T;
+        s.ntok = a.T;
+        s.shared = true;
+        s.valid = a.T <= kBatchMaxTokens;
+        return s;
+    }
+    s.shared = false;
+    const int e = a.active[slot - a.n_shared];
+    int b = 0, en = 0;
+    if (e >= 0 && e < a.E) {
+        b = a.offsets[e];
+        en = a.offsets[e + 1];
+    }
+    s.valid = e >= 0 && e < a.E && b >= 0 && en > b && en <= P && en - b <= kBatchMaxTokens;
+    s.e = s.valid ? e : 0;
+    s.list_begin = s.valid ? b : 0;
+    s.ntok = s.valid ? en - b : 0;
+    return s;
+}
+
+// kGU: gate/up + SwiGLU -> h' rows; otherwise down -> y rows.
+template <bool kGU>
+__global__ void __launch_bounds__(kBThreads, 1)
+batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kStagesB;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 512);
+    uint8_t* stage0 = smem + kHdrB;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesB; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kBW);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();  // the union lists and the activation rows come from the previous kernels
+
+    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
+    if (n_act < 0 || n_act > a.E) {
+        if (threadIdx.x == 0) report(a.status, COLI_ERR_BAD_INDEX);
+        n_act = 0;
+    }
+    const int n_slots = n_act + a.n_shared;
+    const int K = kGU ? a.H : a.I;
+    const int KB = K / kGroup;
+    const int m_tiles = kGU ? a.I / kBoxRows : (a.H + kTileRows - 1) / kTileRows;
+    const int n_chunks = a.T > kChunkTok ? kChunks : 1;  // column chunks per list
+    const int64_t n_tiles = (int64_t)n_slots * n_chunks * m_tiles;
+    const int P = a.T * a.k;
+    // tile -> slot, column chunk (entries 32 ch ..), row tile
+    auto split = [&](int64_t tile, int& slot, int& ch, int& mt) {
+        slot = (int)(tile / (n_chunks * m_tiles));
+        const int rem = (int)(tile - (int64_t)slot * n_chunks * m_tiles);
+        ch = rem / m_tiles;
+        mt = rem - ch * m_tiles;
+    };
+
+    if (warp == kBW) {
+        // ------------------------------ producer ------------------------------
+        const uint64_t policy = policy_evict_first();
+        int j = 0;
+        bool stop = false;
+        for (int64_t tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
+            int slot, ch, mt;
+            split(tile, slot, ch, mt);
+            const BSlot sl = batch_slot(a, slot);
+            const int n_base = ch * kChunkTok;
+            const int ntok = sl.valid ? min(kChunkTok, sl.ntok - n_base) : 0;
+            if (ntok <= 0) continue;
+            // this lane's activation row: list entry n_base + lane (a pair id
+            // out of range reads token 0's row and is reported; the combine
+            // skips it)
+            const __half* src = nullptr;
+            const float* csrc = nullptr;  // gate/up: the token's offset sums
+            if (lane < ntok) {
+                const int n = n_base + lane;
+                if constexpr (kGU) {
+                    int t = n;
+                    if (!sl.shared) {
+                        const int p = a.pairs[sl.list_begin + n];
+                        if (p < 0 || p >= P) report(a.status, COLI_ERR_BAD_INDEX);
+                        t = (p >= 0 && p < P) ? p / a.k : 0;
+                    }
+                    src = a.xp + (int64_t)t * a.H;
+                    csrc = a.corr + (int64_t)t * KB;
+                } else {
+                    src = a.hp + (int64_t)(sl.list_begin + n) * a.I;
+                }
+            }
+            const CUtensorMap* map0 = wmaps + (size_t)sl.e * 3 + (kGU ? 0 : 2);
+            const CUtensorMap* map1 = wmaps + (size_t)sl.e * 3 + (kGU ? 1 : 2);
+            const int row0 = kGU ? mt * kBoxRows : mt * kTileRows;
+            const int row1 = kGU ? row0 : row0 + kBoxRows;  // down rows past H read as zeros
+            for (int kb0 = 0; kb0 < KB; kb0 += kKBS) {
+                const int nkb = min(kKBS, KB - kb0);
+                const uint32_t tx = (uint32_t)(nkb * kBlockBytes + ntok * nkb * 128) +
+                                    (kGU ? (uint32_t)ntok * 16u : 0u);
+                const int s = j & (kStagesB - 1), use = j / kStagesB;
+                int ok = 1;
+                if (lane == 0) {
+                    if (*abort_flag) ok = 0;
+                    else if (use > 0) ok = (int)mbar_wait(&empty[s], (uint32_t)(use - 1) & 1);
+                    if (!ok && !*abort_flag) {
+                        report(a.status, COLI_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                }
+                if (!__shfl_sync(kAllB, ok, 0)) {
+                    stop = true;
+                    break;
+                }
+                uint8_t* st = stage0 + (size_t)s * kStageB;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], tx);
+                    for (int q = 0; q < nkb; ++q) {
+                        const int xk = (kb0 + q) * (kGroup / 2);
+                        uint8_t* blk = st + q * kBlockBytes;
+                        tma_2d_hint(blk, map0, xk, row0, &full[s], policy);
+                        tma_2d_hint(blk + kBoxRows * 32, map1, xk, row1, &full[s], policy);
+                    }
+                }
+                __syncwarp();
+                if (lane < ntok) {
+                    bulk_g2s(st + kCodeBytes + lane * kActRow, src + kb0 * kGroup,
+                             (uint32_t)nkb * 128u, &full[s]);
+                    // 4 offset sums: within the row, as KB % 4 == 0 for gate/up
+                    if constexpr (kGU) bulk_g2s(st + kCorrOff + lane * 16, csrc + kb0, 16u, &full[s]);
+                }
+                ++j;
+            }
+        }
+        if (stop && lane == 0) {
+            // let the copies already issued land before the CTA goes away
+            for (int back = 1; back <= kStagesB && back <= j; ++back) {
+                const int jj = j - back;
+                (void)mbar_wait(&full[jj & (kStagesB - 1)], (uint32_t)(jj / kStagesB) & 1);
+            }
+        }
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    const int r = lane >> 2, c = lane & 3;
+    const Magic mg = magic();
+    // staged rows of this warp's A fragment rows 0-7 and 8-15
+    const int rtop = kGU ? 8 * warp + r : 16 * warp + r;
+    const uint32_t off_a = (uint32_t)(rtop * 32 + c * 8);
+    const uint32_t off_b = kGU ? off_a + (uint32_t)(kBoxRows * 32) : off_a + 8u * 32u;
+    const int SG = scale_cols(K, a.per_row);
+    const bool vec = !a.per_row && (KB & 7) == 0;
+    int j = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        int slot, ch, mt;
+        split(tile, slot, ch, mt);
+        const BSlot sl = batch_slot(a, slot);
+        if (!sl.valid) {
+            if (warp == 0 && lane == 0 && ch == 0) report(a.status, COLI_ERR_BAD_INDEX);
+            continue;
+        }
+        const int n_base = ch * kChunkTok;
+        const int ntok = min(kChunkTok, sl.ntok - n_base);
+        if (ntok <= 0) continue;
+        const int nt = (ntok + 7) >> 3;
+        const DevExpert ex = a.experts[sl.e];
+        // this lane's two weight rows and their scale rows
+        int ra, rb;
+        bool live_a = true, live_b = true;
+        const uint16_t* sa;
+        const uint16_t* sb;
+        if constexpr (kGU) {
+            ra = rb = mt * kBoxRows + 8 * warp + r;  // gate row and up row of one feature
+            sa = ex.gate_s + (int64_t)ra * SG;
+            sb = ex.up_s + (int64_t)rb * SG;
+        } else {
+            ra = mt * kTileRows + 16 * warp + r;
+            rb = ra + 8;
+            live_a = ra < a.H;
+            live_b = rb < a.H;
+            sa = ex.down_s + (int64_t)(live_a ? ra : 0) * SG;
+            sb = ex.down_s + (int64_t)(live_b ? rb : 0) * SG;
+        }
+        // scales: eight K-blocks per 16-byte load, a chunk ahead (gs64 rows of
+        // whole 16-byte chunks), else one per K-block, one ahead; per-row: one
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        uint4 cha = z4, chb = z4;
+        uint4 cha_n = (vec && live_a) ? __ldg(reinterpret_cast<const uint4*>(sa)) : z4;
+        uint4 chb_n = (vec && live_b) ? __ldg(reinterpret_cast<const uint4*>(sb)) : z4;
+        uint16_t na = (!vec && live_a) ? __ldg(sa) : (uint16_t)0;
+        uint16_t nb = (!vec && live_b) ? __ldg(sb) : (uint16_t)0;
+
+        float acc[kMaxNT][4];
+#pragma unroll
+        for (int jn = 0; jn < kMaxNT; ++jn)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[jn][q] = 0.f;
+
+        for (int kb0 = 0; kb0 < KB; kb0 += kKBS, ++j) {
+            const int s = j & (kStagesB - 1);
+            if (!mbar_wait(&full[s], (uint32_t)(j / kStagesB) & 1)) {
+                if (lane == 0) {
+                    report(a.status, COLI_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                return;
+            }
+            const uint32_t st = smem_addr(stage0) + (uint32_t)(s * kStageB);
+#pragma unroll 1
+            for (int q = 0; q < kKBS; ++q) {
+                const int kb = kb0 + q;
+                if (kb >= KB) break;
+                uint16_t ca, cb;
+                if (vec) {
+                    const int sub = kb & 7;
+                    if (sub == 0) {
+                        cha = cha_n;
+                        chb = chb_n;
+                        if (kb + 8 < KB) {
+                            if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa + kb + 8));
+                            if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb + kb + 8));
+                        }
+                    }
+                    const uint32_t wa2 = sub < 4 ? (sub < 2 ? cha.x : cha.y) : (sub < 6 ? cha.z : cha.w);
+                    const uint32_t wb2 = sub < 4 ? (sub < 2 ? chb.x : chb.y) : (sub < 6 ? chb.z : chb.w);
+                    ca = (uint16_t)((sub & 1) ? (wa2 >> 16) : (wa2 & 0xFFFFu));
+                    cb = (uint16_t)((sub & 1) ? (wb2 >> 16) : (wb2 & 0xFFFFu));
+                } else {
+                    ca = na;
+                    cb = nb;
+                    if (!a.per_row && kb + 1 < KB) {
+                        if (live_a) na = __ldg(sa + kb + 1);
+                        if (live_b) nb = __ldg(sb + kb + 1);
+                    }
+                }
+                const float fa = __uint_as_float((uint32_t)ca << 16);
+                const float fb = __uint_as_float((uint32_t)cb << 16);
+                const uint32_t blk = st + (uint32_t)(q * kBlockBytes);
+                const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
+                uint32_t A[4][4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
+                    unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
+                }
+                const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
+                const uint32_t cbase = st + (uint32_t)(kCorrOff + 2 * c * 16 + q * 4);
+#pragma unroll
+                for (int jn = 0; jn < kMaxNT; ++jn) {
+                    if (jn < nt) {
+                        const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
+                        const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
+                        const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        float part[4];
+                        if constexpr (kGU) {
+                            // the preparation's offset sums of columns 2c, 2c + 1
+                            const float c0 = lds_f(cbase + (uint32_t)(jn * 8 * 16));
+                            const float c1 = lds_f(cbase + (uint32_t)(jn * 8 * 16) + 16u);
+                            part[0] = -c0;
+                            part[1] = -c1;
+                            part[2] = -c0;
+                            part[3] = -c1;
+                        } else {
+                            float cs[4];
+                            offset_sums(bw, cs);  // the unpack offsets' contribution
+                            part[0] = -cs[0];
+                            part[1] = -cs[1];
+                            part[2] = -cs[0];
+                            part[3] = -cs[1];
+                        }
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bw[2 * ks],
+                                     bw[2 * ks + 1]);
+                        acc[jn][0] = fmaf(fa, part[0], acc[jn][0]);
+                        acc[jn][1] = fmaf(fa, part[1], acc[jn][1]);
+                        acc[jn][2] = fmaf(fb, part[2], acc[jn][2]);
+                        acc[jn][3] = fmaf(fb, part[3], acc[jn][3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+
+        // epilogue: column 8 jn + 2c + e2 is list entry n_base + that; rows
+        // ra (acc 0, 1) and rb (acc 2, 3)
+#pragma unroll
+        for (int jn = 0; jn < kMaxNT; ++jn) {
+            if (jn >= nt) continue;
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int nl = 8 * jn + 2 * c + e2;
+                if (nl >= ntok) continue;
+                const int64_t orow = sl.list_begin + n_base + nl;
+                if constexpr (kGU) {
+                    // h = silu(g) * u; the gate weight is applied by the combine
+                    const float gv = acc[jn][e2], uv = acc[jn][2 + e2];
+                    float h = gv / (1.f + expf(-gv)) * uv;
+                    if (fabsf(h) > 65504.f) {
+                        report(a.status, COLI_ERR_RANGE);
+                        h = copysignf(65504.f, h);
+                    }
+                    // h' in the down operand's fragment order; odd features
+                    // are the down projection's odd-K elements: stored / 16
+                    const int fe = ra;
+                    const int hcol = (fe / kGroup) * kGroup + perm64(fe % kGroup);
+                    a.hp[orow * a.I + hcol] = __float2half_rn((fe & 1) ? h * 0.0625f : h);
+                } else {
+                    if (live_a) a.y[orow * a.H + ra] = acc[jn][e2];
+                    if (live_b) a.y[orow * a.H + rb] = acc[jn][2 + e2];
+                }
+            }
+        }
+    }
+}
+
+template <bool kGU>
+cudaError_t launch_one(const FfnArgs& a, const CUtensorMap* wmaps, int blocks, cudaStream_t st) {
+    auto kern = batch_ffn_kernel<kGU>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemB);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(kBThreads);
+    cfg.dynamicSmemBytes = kSmemB;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, wmaps);
+}
+
+}  // namespace
+
+bool batch_supported(int H, int I, int T) {
+    return T >= 1 && T <= kBatchMaxTokens && H >= kKBS * kGroup && H % (kKBS * kGroup) == 0 &&
+           I >= kBoxRows && I % kBoxRows == 0;
+}
+
+cudaError_t launch_batch_ffn(const FfnArgs& a, const CUtensorMap* wmaps, int num_sms,
+                             cudaStream_t st) {
+    profile_mark(1, st);
+    cudaError_t err = launch_one<true>(a, wmaps, num_sms, st);
+    if (err != cudaSuccess) return err;
+    profile_mark(2, st);
+    err = launch_one<false>(a, wmaps, num_sms, st);
+    profile_mark(3, st);
+    return err;
+}
+
+}  // namespace coli
