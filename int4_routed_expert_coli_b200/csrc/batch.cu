@@ -124,8 +124,10 @@ __device__ __forceinline__ BSlot batch_slot(const FfnArgs& a, int slot) {
     return s;
 }
 
-// kGU: gate/up + SwiGLU -> h' rows; otherwise down -> y rows.
-template <bool kGU>
+// kGU: gate/up + SwiGLU -> h' rows; otherwise down -> y rows.  kVec: gs64
+// scale rows of whole 16-byte chunks (K / 64 a multiple of 8), read eight at a
+// time; otherwise one scale per K-block (per-row: the row's one scale).
+template <bool kGU, bool kVec>
 __global__ void __launch_bounds__(kBThreads, 1)
 batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
     extern __shared__ uint8_t smem_raw[];
@@ -260,7 +262,6 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
     const uint32_t off_a = (uint32_t)(rtop * 32 + c * 8);
     const uint32_t off_b = kGU ? off_a + (uint32_t)(kBoxRows * 32) : off_a + 8u * 32u;
     const int SG = scale_cols(K, a.per_row);
-    const bool vec = !a.per_row && (KB & 7) == 0;
     int j = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         int slot, ch, mt;
@@ -292,14 +293,19 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
             sa = ex.down_s + (int64_t)(live_a ? ra : 0) * SG;
             sb = ex.down_s + (int64_t)(live_b ? rb : 0) * SG;
         }
-        // scales: eight K-blocks per 16-byte load, a chunk ahead (gs64 rows of
-        // whole 16-byte chunks), else one per K-block, one ahead; per-row: one
+        // scales: eight K-blocks per 16-byte load, a chunk ahead (kVec), else
+        // one per K-block, one ahead; per-row: the row's one scale
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-        uint4 cha = z4, chb = z4;
-        uint4 cha_n = (vec && live_a) ? __ldg(reinterpret_cast<const uint4*>(sa)) : z4;
-        uint4 chb_n = (vec && live_b) ? __ldg(reinterpret_cast<const uint4*>(sb)) : z4;
-        uint16_t na = (!vec && live_a) ? __ldg(sa) : (uint16_t)0;
-        uint16_t nb = (!vec && live_b) ? __ldg(sb) : (uint16_t)0;
+        uint4 cha_n = z4, chb_n = z4;  // the next chunk
+        uint32_t ha0 = 0u, ha1 = 0u, hb0 = 0u, hb1 = 0u;  // the current chunk's second half
+        uint16_t na = 0, nb = 0;
+        if constexpr (kVec) {
+            if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa));
+            if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb));
+        } else {
+            if (live_a) na = __ldg(sa);
+            if (live_b) nb = __ldg(sb);
+        }
 
         float acc[kMaxNT][4];
 #pragma unroll
@@ -317,35 +323,47 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                 return;
             }
             const uint32_t st = smem_addr(stage0) + (uint32_t)(s * kStageB);
+            // the stage's four scales of both rows, as bf16 pairs: the first
+            // or the second half of the current chunk
+            uint32_t spa0 = 0u, spa1 = 0u, spb0 = 0u, spb1 = 0u;
+            if constexpr (kVec) {
+                if ((kb0 & 7) == 0) {
+                    spa0 = cha_n.x;
+                    spa1 = cha_n.y;
+                    spb0 = chb_n.x;
+                    spb1 = chb_n.y;
+                    ha0 = cha_n.z;
+                    ha1 = cha_n.w;
+                    hb0 = chb_n.z;
+                    hb1 = chb_n.w;
+                    if (kb0 + 8 < KB) {
+                        if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa + kb0 + 8));
+                        if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb + kb0 + 8));
+                    }
+                } else {
+                    spa0 = ha0;
+                    spa1 = ha1;
+                    spb0 = hb0;
+                    spb1 = hb1;
+                }
+            }
 #pragma unroll 1
             for (int q = 0; q < kKBS; ++q) {
                 const int kb = kb0 + q;
                 if (kb >= KB) break;
-                uint16_t ca, cb;
-                if (vec) {
-                    const int sub = kb & 7;
-                    if (sub == 0) {
-                        cha = cha_n;
-                        chb = chb_n;
-                        if (kb + 8 < KB) {
-                            if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa + kb + 8));
-                            if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb + kb + 8));
-                        }
-                    }
-                    const uint32_t wa2 = sub < 4 ? (sub < 2 ? cha.x : cha.y) : (sub < 6 ? cha.z : cha.w);
-                    const uint32_t wb2 = sub < 4 ? (sub < 2 ? chb.x : chb.y) : (sub < 6 ? chb.z : chb.w);
-                    ca = (uint16_t)((sub & 1) ? (wa2 >> 16) : (wa2 & 0xFFFFu));
-                    cb = (uint16_t)((sub & 1) ? (wb2 >> 16) : (wb2 & 0xFFFFu));
+                float fa, fb;
+                if constexpr (kVec) {
+                    const uint32_t wa2 = q < 2 ? spa0 : spa1, wb2 = q < 2 ? spb0 : spb1;
+                    fa = __uint_as_float((q & 1) ? (wa2 & 0xFFFF0000u) : (wa2 << 16));
+                    fb = __uint_as_float((q & 1) ? (wb2 & 0xFFFF0000u) : (wb2 << 16));
                 } else {
-                    ca = na;
-                    cb = nb;
+                    fa = __uint_as_float((uint32_t)na << 16);
+                    fb = __uint_as_float((uint32_t)nb << 16);
                     if (!a.per_row && kb + 1 < KB) {
                         if (live_a) na = __ldg(sa + kb + 1);
                         if (live_b) nb = __ldg(sb + kb + 1);
                     }
                 }
-                const float fa = __uint_as_float((uint32_t)ca << 16);
-                const float fb = __uint_as_float((uint32_t)cb << 16);
                 const uint32_t blk = st + (uint32_t)(q * kBlockBytes);
                 const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
                 uint32_t A[4][4];
@@ -426,9 +444,9 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
     }
 }
 
-template <bool kGU>
+template <bool kGU, bool kVec>
 cudaError_t launch_one(const FfnArgs& a, const CUtensorMap* wmaps, int blocks, cudaStream_t st) {
-    auto kern = batch_ffn_kernel<kGU>;
+    auto kern = batch_ffn_kernel<kGU, kVec>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemB);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -453,11 +471,16 @@ bool batch_supported(int H, int I, int T) {
 
 cudaError_t launch_batch_ffn(const FfnArgs& a, const CUtensorMap* wmaps, int num_sms,
                              cudaStream_t st) {
+    // gs64 rows of whole 16-byte chunks: scales read eight K-blocks at a time
+    const bool vec_gu = !a.per_row && (a.H / kGroup) % 8 == 0;
+    const bool vec_dn = !a.per_row && (a.I / kGroup) % 8 == 0;
     profile_mark(1, st);
-    cudaError_t err = launch_one<true>(a, wmaps, num_sms, st);
+    cudaError_t err = vec_gu ? launch_one<true, true>(a, wmaps, num_sms, st)
+                             : launch_one<true, false>(a, wmaps, num_sms, st);
     if (err != cudaSuccess) return err;
     profile_mark(2, st);
-    err = launch_one<false>(a, wmaps, num_sms, st);
+    err = vec_dn ? launch_one<false, true>(a, wmaps, num_sms, st)
+                 : launch_one<false, false>(a, wmaps, num_sms, st);
     profile_mark(3, st);
     return err;
 }
