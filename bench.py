@@ -77,13 +77,19 @@ PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 # changed since, the bench reports traffic as null.
 # workload -> (source file, sha256, bytes per unit, unit, how it was measured)
 _DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
-               "fe5733e351aa296cfbdb8fe7dbcff3d1c947ef884e1702defe6aad80d9300fee")
+               "4b2566a371c85094c21a668a748004e16efadabc12e262cffc246356d1698882")
+_BATCH_SRC = ("int4_routed_expert_coli_b200/csrc/batch.cu",
+              "3f171ea60eeaf3249b7e85bed6d7723e08e7a59fd1cc17841215096c71592069")
+_BATCH = (*_BATCH_SRC, 13_327_027, "streamed expert",
+          "ncu launch list, 12 launches of the small-batch gate/up kernel on a 64-expert bank "
+          "at T=32: bytes per streamed expert (unique routed + shared)")
 DRAM_TRAFFIC = {
-    "decode": (*_DECODE_SRC, 184_230_741, "launch",
+    "decode": (*_DECODE_SRC, 183_850_410, "launch",
                "ncu launch list, 18 launches of the fused decode kernel on a 64-expert bank "
                "(a T=1 step streams 8 + 1 experts on any bank)"),
-    "verify4": (*_DECODE_SRC, 184_230_741 // 9, "streamed expert",
+    "verify4": (*_DECODE_SRC, 183_850_410 // 9, "streamed expert",
                 "the T=1 fused-kernel capture, bytes per streamed expert"),
+    "batch32": _BATCH,
 }
 
 
