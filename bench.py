@@ -79,8 +79,8 @@ PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 _DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
                "4b2566a371c85094c21a668a748004e16efadabc12e262cffc246356d1698882")
 _BATCH_SRC = ("int4_routed_expert_coli_b200/csrc/batch.cu",
-              "3f171ea60eeaf3249b7e85bed6d7723e08e7a59fd1cc17841215096c71592069")
-_BATCH = (*_BATCH_SRC, 13_327_027, "streamed expert",
+              "ecd0e0f3e5e8123c3033fef1e8b8685872cda2a39c03012815fe0775d54c8348")
+_BATCH = (*_BATCH_SRC, 13_325_395, "streamed expert",
           "ncu launch list, 12 launches of the small-batch gate/up kernel on a 64-expert bank "
           "at T=32: bytes per streamed expert (unique routed + shared)")
 DRAM_TRAFFIC = {

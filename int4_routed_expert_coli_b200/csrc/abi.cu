@@ -129,7 +129,7 @@ bool fused_ok(const coli_moe* h, int64_t T) {
 // True when a call with T tokens runs the small-batch kernels (the default
 // for calls of up to 64 tokens the fused decode kernel does not take).
 bool use_batch(const coli_moe* h, int64_t T) {
-    return h->d_wmaps != nullptr && h->prefill_min == 0 && !fused_ok(h, T) &&
+    return h->d_bmaps != nullptr && h->prefill_min == 0 && !fused_ok(h, T) &&
            coli::batch_supported(h->H, h->I, (int)T);
 }
 
@@ -176,7 +176,7 @@ cudaError_t run_ffn(const coli_moe* h, int32_t T, const coli::FfnArgs& a, void* 
     }
     if (use_batch(h, T)) {
         if (!x_prepared) err = coli::launch_prepare_x(T, h->H, a.x, a.xp, a.corr, a.status, st);
-        if (err == cudaSuccess) err = coli::launch_batch_ffn(a, h->d_wmaps, h->num_sms, st);
+        if (err == cudaSuccess) err = coli::launch_batch_ffn(a, h->d_bmaps, h->num_sms, st);
         if (err == cudaSuccess) err = coli::launch_combine(a, h->num_sms, st);
         coli::profile_mark(4, st);
         return err;
@@ -294,6 +294,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     h->num_sms = sms;
     h->d_experts = nullptr;
     h->d_wmaps = nullptr;
+    h->d_bmaps = nullptr;
     h->d_dmaps = nullptr;
     coli::DevExpert* host = static_cast<coli::DevExpert*>(std::malloc(sizeof(coli::DevExpert) * n));
     if (!host) {
@@ -312,7 +313,9 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (err == cudaSuccess)
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
     if (err == cudaSuccess && coli::prefill_available())
-        err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
+        err = coli::build_weight_maps(host, n, h->H, h->I, false, &h->d_wmaps);
+    if (err == cudaSuccess && h->d_wmaps)
+        err = coli::build_weight_maps(host, n, h->H, h->I, true, &h->d_bmaps);
     // the fused decode kernel only where one CTA per SM can be resident at once
     if (err == cudaSuccess && h->d_wmaps &&
         coli::decode_supported(h->H, h->I, 1, h->E, h->k, h->n_shared, h->num_sms) &&
@@ -325,6 +328,7 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (err != cudaSuccess) {
         if (h->d_experts) cudaFree(h->d_experts);
         if (h->d_wmaps) cudaFree(h->d_wmaps);
+        if (h->d_bmaps) cudaFree(h->d_bmaps);
         if (h->d_dmaps) cudaFree(h->d_dmaps);
         delete h;
         return COLI_ERR_CUDA;
@@ -337,6 +341,7 @@ void coli_moe_destroy(coli_moe* h) {
     if (!h) return;
     cudaFree(h->d_experts);
     if (h->d_wmaps) cudaFree(h->d_wmaps);
+    if (h->d_bmaps) cudaFree(h->d_bmaps);
     if (h->d_dmaps) cudaFree(h->d_dmaps);
     delete h;
 }

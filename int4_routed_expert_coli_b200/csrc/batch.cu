@@ -25,8 +25,10 @@
 // first).
 //
 // Data movement.  A producer warp stages four 64-element K-blocks at a time
-// in a ring of 4 stages of 49 KB: the codes of the tile's rows by 2-D tensor
-// copies (128 rows x 32 bytes each), each token's 256 activations (fragment
+// in a ring of 4 stages of 49 KB: the codes of the tile's rows by two 2-D
+// tensor copies (128 rows x 128 bytes each, 128-byte swizzle: a narrow box of
+// one K-block per row moves a quarter of the bytes per copied row, and the
+// copy engine's row rate then limits the stream), each token's 256 activations (fragment
 // order, 512 bytes) by a 1-D bulk copy into a row of 528 bytes (the padding
 // spreads the fragment reads over the banks), and for gate/up each token's 4
 // precomputed offset sums (16 bytes).  The activations are, for gate/up, the
@@ -55,8 +57,8 @@ constexpr int kChunkTok = 32;                         // list entries per tile
 constexpr int kMaxNT = kChunkTok / 8;                 // 8-token column tiles
 constexpr int kChunks = kBatchMaxTokens / kChunkTok;  // column chunks of a list
 constexpr int kKBS = 4;                               // K-blocks (scale groups) per stage
-constexpr int kBlockBytes = kTileRows * 32;           // codes of one K-block (two boxes)
-constexpr int kCodeBytes = kKBS * kBlockBytes;
+constexpr int kBoxBytes = kBoxRows * kKBS * 32;       // one tensor copy: 128 rows x 128 bytes
+constexpr int kCodeBytes = 2 * kBoxBytes;             // a stage's codes (two copies)
 constexpr int kActRow = kKBS * 128 + 16;              // staged activation row (bytes)
 constexpr int kCorrOff = kCodeBytes + kChunkTok * kActRow;  // offset sums, 16 B per token
 constexpr int kStageB = kCorrOff + kChunkTok * 16;
@@ -68,6 +70,8 @@ constexpr unsigned kAllB = 0xffffffffu;
 static_assert(kSmemB <= kSmemLimitB, "stage ring");
 static_assert(kChunkTok <= 32, "one activation row per producer lane");
 static_assert(kActRow % 16 == 0 && kStageB % 16 == 0 && kCorrOff % 16 == 0, "bulk copy alignment");
+// the 128-byte swizzle repeats every 8 rows of 128 bytes: stages stay 1 KB aligned
+static_assert(kStageB % 1024 == 0 && kHdrB % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzle atoms");
 // a staged activation row of 33 16-byte units: the 8 lanes of a quarter-warp
 // (rows r, r + 1; units 2c .. 2c + 1) fall on distinct bank groups
 static_assert((kActRow / 16) % 8 == 1, "activation row stride");
@@ -208,7 +212,8 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
             const int row1 = kGU ? row0 : row0 + kBoxRows;  // down rows past H read as zeros
             for (int kb0 = 0; kb0 < KB; kb0 += kKBS) {
                 const int nkb = min(kKBS, KB - kb0);
-                const uint32_t tx = (uint32_t)(nkb * kBlockBytes + ntok * nkb * 128) +
+                // a box past the end of K is filled with zeros and counts whole
+                const uint32_t tx = (uint32_t)(kCodeBytes + ntok * nkb * 128) +
                                     (kGU ? (uint32_t)ntok * 16u : 0u);
                 const int s = j & (kStagesB - 1), use = j / kStagesB;
                 int ok = 1;
@@ -227,12 +232,9 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                 uint8_t* st = stage0 + (size_t)s * kStageB;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[s], tx);
-                    for (int q = 0; q < nkb; ++q) {
-                        const int xk = (kb0 + q) * (kGroup / 2);
-                        uint8_t* blk = st + q * kBlockBytes;
-                        tma_2d_hint(blk, map0, xk, row0, &full[s], policy);
-                        tma_2d_hint(blk + kBoxRows * 32, map1, xk, row1, &full[s], policy);
-                    }
+                    const int xk = kb0 * (kGroup / 2);  // a multiple of 128 bytes
+                    tma_2d_hint(st, map0, xk, row0, &full[s], policy);
+                    tma_2d_hint(st + kBoxBytes, map1, xk, row1, &full[s], policy);
                 }
                 __syncwarp();
                 if (lane < ntok) {
@@ -257,10 +259,17 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
     // -------------------------------- consumers --------------------------------
     const int r = lane >> 2, c = lane & 3;
     const Magic mg = magic();
-    // staged rows of this warp's A fragment rows 0-7 and 8-15
+    // staged rows of this warp's A fragment rows 0-7 and 8-15: gate/up, row
+    // 8 warp + r of the gate box and of the up box; down, rows 16 warp + r and
+    // + 8 of the tile (box warp / 8).  Every such row is r modulo 8, so the
+    // swizzle puts logical 16-byte unit u of a row at u ^ r: K-block q's 8
+    // bytes for this lane (unit 2q + c / 2, half c % 2) sit at
+    // ((q ^ (r / 2)) * 32) + ((c / 2) ^ (r % 2)) * 16 + (c % 2) * 8.
     const int rtop = kGU ? 8 * warp + r : 16 * warp + r;
-    const uint32_t off_a = (uint32_t)(rtop * 32 + c * 8);
-    const uint32_t off_b = kGU ? off_a + (uint32_t)(kBoxRows * 32) : off_a + 8u * 32u;
+    const uint32_t off_a = (uint32_t)((rtop / kBoxRows) * kBoxBytes + (rtop % kBoxRows) * 128 +
+                                      (((c >> 1) ^ (r & 1)) << 4) + ((c & 1) << 3));
+    const uint32_t off_b = kGU ? off_a + (uint32_t)kBoxBytes : off_a + 8u * 128u;
+    const uint32_t rq = (uint32_t)(r >> 1);
     const int SG = scale_cols(K, a.per_row);
     int j = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -364,7 +373,7 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                         if (live_b) nb = __ldg(sb + kb + 1);
                     }
                 }
-                const uint32_t blk = st + (uint32_t)(q * kBlockBytes);
+                const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
                 const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
                 uint32_t A[4][4];
 #pragma unroll

@@ -15,8 +15,8 @@ constexpr int kBatchMaxTokens = 64;
 bool batch_supported(int H, int I, int T);
 // gate/up + SwiGLU (h rows), then down (y rows), over the union lists of a
 // call; the activation operand (xp, fragment order) must be ready; the caller
-// runs the combine.  wmaps: the grouped GEMM's per-expert code tensor maps
-// (3 per expert, 128-row boxes of 32 bytes).
+// runs the combine.  wmaps: per-expert code tensor maps (3 per expert,
+// 128-row boxes of 128 bytes, 128-byte swizzle).
 cudaError_t launch_batch_ffn(const FfnArgs& a, const CUtensorMap* wmaps, int num_sms,
                              cudaStream_t st);
 

@@ -13,5 +13,6 @@ struct coli_moe {
     int num_sms;
     coli::DevExpert* d_experts;  // device table, E + n_shared entries
     CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)
+    CUtensorMap* d_bmaps;        // 128-byte-wide swizzled code maps, 3 per expert (small batches)
     CUtensorMap* d_dmaps;        // swizzled 3-D code maps, 3 per expert (fused decode path)
 };

@@ -145,6 +145,7 @@ extern "C" coli_status coli_moe_layer_noalloc(const coli_moe_desc* d, int32_t T,
     h.num_sms = s->num_sms;
     h.d_experts = reinterpret_cast<coli::DevExpert*>(base);
     h.d_wmaps = nullptr;
+    h.d_bmaps = nullptr;
     h.d_dmaps = nullptr;
     st = coli_moe_layer(&h, T, x_bf16, logits, nullptr, residual, out, out_dtype, nullptr, nullptr,
                         ws, kScratchBytes, stream);

@@ -35,8 +35,11 @@ struct GatherArgs {
 };
 
 // Tensor maps of every expert's packed code matrices (device array, 3 per
-// expert: gate, up, down).  Returns an error if the driver lacks tensor maps.
-cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I,
+// expert: gate, up, down), boxes of 128 rows: one 64-code K-block (32 bytes,
+// unswizzled; the grouped GEMM) or, `wide`, four K-blocks (128 bytes, 128-byte
+// swizzle; the small-batch kernels).  Returns an error if the driver lacks
+// tensor maps.
+cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I, bool wide,
                               CUtensorMap** d_maps);
 // gather -> gate/up GEMM -> down GEMM (writes y); the caller runs the combine.
 cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* xg,
