@@ -313,9 +313,9 @@ coli_status coli_moe_create(const coli_moe_desc* d, coli_moe** out) {
     if (err == cudaSuccess)
         err = cudaMemcpy(h->d_experts, host, sizeof(coli::DevExpert) * n, cudaMemcpyHostToDevice);
     if (err == cudaSuccess && coli::prefill_available())
-        err = coli::build_weight_maps(host, n, h->H, h->I, false, &h->d_wmaps);
+        err = coli::build_weight_maps(host, n, h->H, h->I, &h->d_wmaps);
     if (err == cudaSuccess && h->d_wmaps)
-        err = coli::build_weight_maps(host, n, h->H, h->I, true, &h->d_bmaps);
+        err = coli::build_batch_maps(host, n, h->H, h->I, h->per_row, &h->d_bmaps);
     // the fused decode kernel only where one CTA per SM can be resident at once
     if (err == cudaSuccess && h->d_wmaps &&
         coli::decode_supported(h->H, h->I, 1, h->E, h->k, h->n_shared, h->num_sms) &&

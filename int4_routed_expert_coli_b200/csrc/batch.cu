@@ -41,7 +41,12 @@
 // Every wait is bounded (COLI_ERR_TIMEOUT).
 #include <cuda.h>
 
+#include <cstring>
+#include <new>
+
 #include "batch.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
 #include "mma_frag.cuh"
 #include "moe_device.cuh"
 #include "ptx.cuh"
@@ -61,7 +66,10 @@ constexpr int kBoxBytes = kBoxRows * kKBS * 32;       // one tensor copy: 128 ro
 constexpr int kCodeBytes = 2 * kBoxBytes;             // a stage's codes (two copies)
 constexpr int kActRow = kKBS * 128 + 16;              // staged activation row (bytes)
 constexpr int kCorrOff = kCodeBytes + kChunkTok * kActRow;  // offset sums, 16 B per token
-constexpr int kStageB = kCorrOff + kChunkTok * 16;
+constexpr int kScaleOff = kCorrOff + kChunkTok * 16;        // scale chunks (kVec)
+constexpr int kScaleBox = kBoxRows * 16;                     // 128 rows x 8 scales
+constexpr int kScaleBytes = 2 * kScaleBox;
+constexpr int kStageB = kScaleOff + kScaleBytes;
 constexpr int kHdrB = 1024;
 constexpr int kSmemLimitB = 227 * 1024;
 constexpr int kStagesB = 4;
@@ -90,6 +98,14 @@ __device__ __forceinline__ void tma_2d_hint(void* dst, const void* tmap, int c0,
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
         "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
         "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(void* dst, const void* tmap, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar))
         : "memory");
 }
 
@@ -128,16 +144,29 @@ __device__ __forceinline__ BSlot batch_slot(const FfnArgs& a, int slot) {
     return s;
 }
 
+// What a staged stage holds, written by the producer before it arms the
+// stage (the arming arrive releases it to the consumers' waits).
+struct StageMeta {
+    int mt;          // row tile
+    int row_begin;   // first h / y row of the tile's list entries (0 .. ntok - 1)
+    int ntok;        // list entries; 0: the CTA's tile sequence is over
+    int kb0;         // first K-block of the stage
+    int last;        // the tile's last stage
+    int e;           // expert row in the device table
+};
+
 // kGU: gate/up + SwiGLU -> h' rows; otherwise down -> y rows.  kVec: gs64
-// scale rows of whole 16-byte chunks (K / 64 a multiple of 8), read eight at a
-// time; otherwise one scale per K-block (per-row: the row's one scale).
+// scale rows of whole 16-byte chunks (K / 64 a multiple of 8), staged with
+// the codes; otherwise read from global memory one per K-block (per-row: the
+// row's one scale).
 template <bool kGU, bool kVec>
 __global__ void __launch_bounds__(kBThreads, 1)
-batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
+batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kStagesB;
+    volatile StageMeta* meta = reinterpret_cast<volatile StageMeta*>(smem + 128);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 512);
     uint8_t* stage0 = smem + kHdrB;
 
@@ -154,37 +183,50 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
     pdl_launch_dependents();
     pdl_wait();  // the union lists and the activation rows come from the previous kernels
 
-    int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
-    if (n_act < 0 || n_act > a.E) {
-        if (threadIdx.x == 0) report(a.status, COLI_ERR_BAD_INDEX);
-        n_act = 0;
-    }
-    const int n_slots = n_act + a.n_shared;
     const int K = kGU ? a.H : a.I;
     const int KB = K / kGroup;
-    const int m_tiles = kGU ? a.I / kBoxRows : (a.H + kTileRows - 1) / kTileRows;
-    const int n_chunks = a.T > kChunkTok ? kChunks : 1;  // column chunks per list
-    const int64_t n_tiles = (int64_t)n_slots * n_chunks * m_tiles;
-    const int P = a.T * a.k;
-    // tile -> slot, column chunk (entries 32 ch ..), row tile
-    auto split = [&](int64_t tile, int& slot, int& ch, int& mt) {
-        slot = (int)(tile / (n_chunks * m_tiles));
-        const int rem = (int)(tile - (int64_t)slot * n_chunks * m_tiles);
-        ch = rem / m_tiles;
-        mt = rem - ch * m_tiles;
-    };
 
     if (warp == kBW) {
         // ------------------------------ producer ------------------------------
+        int n_act = *reinterpret_cast<const volatile int*>(a.n_active);
+        if (n_act < 0 || n_act > a.E) {
+            if (lane == 0) report(a.status, COLI_ERR_BAD_INDEX);
+            n_act = 0;
+        }
+        const int n_slots = n_act + a.n_shared;
+        const int m_tiles = kGU ? a.I / kBoxRows : (a.H + kTileRows - 1) / kTileRows;
+        const int n_chunks = a.T > kChunkTok ? kChunks : 1;  // column chunks per list
+        const int64_t n_tiles = (int64_t)n_slots * n_chunks * m_tiles;
+        const int P = a.T * a.k;
         const uint64_t policy = policy_evict_first();
         int j = 0;
         bool stop = false;
+        // waits for stage j's slot to be free; false: wind down
+        auto acquire = [&](int jj) {
+            const int use = jj / kStagesB;
+            int ok = 1;
+            if (lane == 0) {
+                if (*abort_flag) ok = 0;
+                else if (use > 0) ok = (int)mbar_wait(&empty[jj & (kStagesB - 1)], (uint32_t)(use - 1) & 1);
+                if (!ok && !*abort_flag) {
+                    report(a.status, COLI_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+            }
+            return __shfl_sync(kAllB, ok, 0) != 0;
+        };
         for (int64_t tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
-            int slot, ch, mt;
-            split(tile, slot, ch, mt);
+            // tile -> slot (shared experts first), column chunk, row tile
+            const int slot = (int)(tile / (n_chunks * m_tiles));
+            const int rem = (int)(tile - (int64_t)slot * n_chunks * m_tiles);
+            const int ch = rem / m_tiles, mt = rem - ch * m_tiles;
             const BSlot sl = batch_slot(a, slot);
+            if (!sl.valid) {
+                if (lane == 0 && ch == 0 && mt == 0) report(a.status, COLI_ERR_BAD_INDEX);
+                continue;
+            }
             const int n_base = ch * kChunkTok;
-            const int ntok = sl.valid ? min(kChunkTok, sl.ntok - n_base) : 0;
+            const int ntok = min(kChunkTok, sl.ntok - n_base);
             if (ntok <= 0) continue;
             // this lane's activation row: list entry n_base + lane (a pair id
             // out of range reads token 0's row and is reported; the combine
@@ -206,35 +248,41 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                     src = a.hp + (int64_t)(sl.list_begin + n) * a.I;
                 }
             }
-            const CUtensorMap* map0 = wmaps + (size_t)sl.e * 3 + (kGU ? 0 : 2);
-            const CUtensorMap* map1 = wmaps + (size_t)sl.e * 3 + (kGU ? 1 : 2);
+            const CUtensorMap* maps = bmaps + (size_t)sl.e * 6;
+            const CUtensorMap* map0 = maps + (kGU ? 0 : 2);
+            const CUtensorMap* map1 = maps + (kGU ? 1 : 2);
             const int row0 = kGU ? mt * kBoxRows : mt * kTileRows;
             const int row1 = kGU ? row0 : row0 + kBoxRows;  // down rows past H read as zeros
             for (int kb0 = 0; kb0 < KB; kb0 += kKBS) {
                 const int nkb = min(kKBS, KB - kb0);
-                // a box past the end of K is filled with zeros and counts whole
+                // a box past the end of K (or of the rows) is filled with zeros
+                // and counts whole
                 const uint32_t tx = (uint32_t)(kCodeBytes + ntok * nkb * 128) +
-                                    (kGU ? (uint32_t)ntok * 16u : 0u);
-                const int s = j & (kStagesB - 1), use = j / kStagesB;
-                int ok = 1;
-                if (lane == 0) {
-                    if (*abort_flag) ok = 0;
-                    else if (use > 0) ok = (int)mbar_wait(&empty[s], (uint32_t)(use - 1) & 1);
-                    if (!ok && !*abort_flag) {
-                        report(a.status, COLI_ERR_TIMEOUT);
-                        *abort_flag = 1;
-                    }
-                }
-                if (!__shfl_sync(kAllB, ok, 0)) {
+                                    (kGU ? (uint32_t)ntok * 16u : 0u) +
+                                    (kVec ? (uint32_t)kScaleBytes : 0u);
+                if (!acquire(j)) {
                     stop = true;
                     break;
                 }
+                const int s = j & (kStagesB - 1);
                 uint8_t* st = stage0 + (size_t)s * kStageB;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], tx);
-                    const int xk = kb0 * (kGroup / 2);  // a multiple of 128 bytes
+                    meta[s].mt = mt;
+                    meta[s].row_begin = sl.list_begin + n_base;
+                    meta[s].ntok = ntok;
+                    meta[s].kb0 = kb0;
+                    meta[s].last = kb0 + kKBS >= KB;
+                    meta[s].e = sl.e;
+                    mbar_arrive_expect_tx(&full[s], tx);  // releases the record
+                    const int xk = kb0 * (kGroup / 2);     // a multiple of 128 bytes
                     tma_2d_hint(st, map0, xk, row0, &full[s], policy);
                     tma_2d_hint(st + kBoxBytes, map1, xk, row1, &full[s], policy);
+                    if constexpr (kVec) {
+                        // the 8-scale chunk holding the stage's 4 (x: a multiple of 8 scales)
+                        const int xs = kb0 & ~7;
+                        tma_2d(st + kScaleOff, maps + (kGU ? 3 : 5), xs, row0, &full[s]);
+                        tma_2d(st + kScaleOff + kScaleBox, maps + (kGU ? 4 : 5), xs, row1, &full[s]);
+                    }
                 }
                 __syncwarp();
                 if (lane < ntok) {
@@ -245,6 +293,17 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                 }
                 ++j;
             }
+        }
+        if (!stop && acquire(j)) {
+            // the end of the sequence: a stage with no entries, armed by a plain arrive
+            const int s = j & (kStagesB - 1);
+            if (lane == 0) {
+                meta[s].ntok = 0;
+                mbar_arrive(&full[s]);
+            }
+            ++j;
+        } else {
+            stop = true;
         }
         if (stop && lane == 0) {
             // let the copies already issued land before the CTA goes away
@@ -270,158 +329,136 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
                                       (((c >> 1) ^ (r & 1)) << 4) + ((c & 1) << 3));
     const uint32_t off_b = kGU ? off_a + (uint32_t)kBoxBytes : off_a + 8u * 128u;
     const uint32_t rq = (uint32_t)(r >> 1);
+    // staged scale chunks of the two rows (16 bytes a row in 128-row boxes)
+    const uint32_t soff_a = (uint32_t)(kScaleOff + (rtop / kBoxRows) * kScaleBox + (rtop % kBoxRows) * 16);
+    const uint32_t soff_b = kGU ? soff_a + (uint32_t)kScaleBox : soff_a + 8u * 16u;
     const int SG = scale_cols(K, a.per_row);
-    int j = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        int slot, ch, mt;
-        split(tile, slot, ch, mt);
-        const BSlot sl = batch_slot(a, slot);
-        if (!sl.valid) {
-            if (warp == 0 && lane == 0 && ch == 0) report(a.status, COLI_ERR_BAD_INDEX);
-            continue;
+
+    float acc[kMaxNT][4];
+    int ra = 0, rb = 0, nt = 0;
+    bool live_a = true, live_b = true;
+    const uint16_t* sa = nullptr;  // global scale rows (not kVec)
+    const uint16_t* sb = nullptr;
+    uint16_t na = 0, nb = 0;
+    for (int j = 0;; ++j) {
+        const int s = j & (kStagesB - 1);
+        if (*abort_flag || !mbar_wait(&full[s], (uint32_t)(j / kStagesB) & 1)) {
+            if (lane == 0 && !*abort_flag) {
+                report(a.status, COLI_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            return;
         }
-        const int n_base = ch * kChunkTok;
-        const int ntok = min(kChunkTok, sl.ntok - n_base);
-        if (ntok <= 0) continue;
-        const int nt = (ntok + 7) >> 3;
-        const DevExpert ex = a.experts[sl.e];
-        // this lane's two weight rows and their scale rows
-        int ra, rb;
-        bool live_a = true, live_b = true;
-        const uint16_t* sa;
-        const uint16_t* sb;
-        if constexpr (kGU) {
-            ra = rb = mt * kBoxRows + 8 * warp + r;  // gate row and up row of one feature
-            sa = ex.gate_s + (int64_t)ra * SG;
-            sb = ex.up_s + (int64_t)rb * SG;
-        } else {
-            ra = mt * kTileRows + 16 * warp + r;
-            rb = ra + 8;
-            live_a = ra < a.H;
-            live_b = rb < a.H;
-            sa = ex.down_s + (int64_t)(live_a ? ra : 0) * SG;
-            sb = ex.down_s + (int64_t)(live_b ? rb : 0) * SG;
+        const int ntok = meta[s].ntok;
+        if (ntok <= 0) return;  // the sequence is over
+        const int mt = meta[s].mt, kb0 = meta[s].kb0, row_begin = meta[s].row_begin;
+        const bool last = meta[s].last != 0;
+        if (kb0 == 0) {
+            // a new tile: this lane's two weight rows
+            nt = (ntok + 7) >> 3;
+            if constexpr (kGU) {
+                ra = rb = mt * kBoxRows + 8 * warp + r;  // gate row and up row of one feature
+            } else {
+                ra = mt * kTileRows + 16 * warp + r;
+                rb = ra + 8;
+                live_a = ra < a.H;
+                live_b = rb < a.H;
+            }
+            if constexpr (!kVec) {
+                const DevExpert ex = a.experts[meta[s].e];
+                if constexpr (kGU) {
+                    sa = ex.gate_s + (int64_t)ra * SG;
+                    sb = ex.up_s + (int64_t)rb * SG;
+                } else {
+                    sa = ex.down_s + (int64_t)(live_a ? ra : 0) * SG;
+                    sb = ex.down_s + (int64_t)(live_b ? rb : 0) * SG;
+                }
+                na = live_a ? __ldg(sa) : (uint16_t)0;
+                nb = live_b ? __ldg(sb) : (uint16_t)0;
+            }
+#pragma unroll
+            for (int jn = 0; jn < kMaxNT; ++jn)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[jn][q] = 0.f;
         }
-        // scales: eight K-blocks per 16-byte load, a chunk ahead (kVec), else
-        // one per K-block, one ahead; per-row: the row's one scale
-        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-        uint4 cha_n = z4, chb_n = z4;  // the next chunk
-        uint32_t ha0 = 0u, ha1 = 0u, hb0 = 0u, hb1 = 0u;  // the current chunk's second half
-        uint16_t na = 0, nb = 0;
+        const uint32_t st = smem_addr(stage0) + (uint32_t)(s * kStageB);
+        // the stage's four scales of both rows, as bf16 pairs: the first or
+        // the second half of the staged chunk
+        uint32_t spa0 = 0u, spa1 = 0u, spb0 = 0u, spb1 = 0u;
         if constexpr (kVec) {
-            if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa));
-            if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb));
-        } else {
-            if (live_a) na = __ldg(sa);
-            if (live_b) nb = __ldg(sb);
+            const uint32_t half = (kb0 & 4) ? 8u : 0u;
+            const uint2 va = lds_u2(st + soff_a + half), vb = lds_u2(st + soff_b + half);
+            spa0 = va.x;
+            spa1 = va.y;
+            spb0 = vb.x;
+            spb1 = vb.y;
         }
-
-        float acc[kMaxNT][4];
-#pragma unroll
-        for (int jn = 0; jn < kMaxNT; ++jn)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[jn][q] = 0.f;
-
-        for (int kb0 = 0; kb0 < KB; kb0 += kKBS, ++j) {
-            const int s = j & (kStagesB - 1);
-            if (!mbar_wait(&full[s], (uint32_t)(j / kStagesB) & 1)) {
-                if (lane == 0) {
-                    report(a.status, COLI_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                return;
-            }
-            const uint32_t st = smem_addr(stage0) + (uint32_t)(s * kStageB);
-            // the stage's four scales of both rows, as bf16 pairs: the first
-            // or the second half of the current chunk
-            uint32_t spa0 = 0u, spa1 = 0u, spb0 = 0u, spb1 = 0u;
-            if constexpr (kVec) {
-                if ((kb0 & 7) == 0) {
-                    spa0 = cha_n.x;
-                    spa1 = cha_n.y;
-                    spb0 = chb_n.x;
-                    spb1 = chb_n.y;
-                    ha0 = cha_n.z;
-                    ha1 = cha_n.w;
-                    hb0 = chb_n.z;
-                    hb1 = chb_n.w;
-                    if (kb0 + 8 < KB) {
-                        if (live_a) cha_n = __ldg(reinterpret_cast<const uint4*>(sa + kb0 + 8));
-                        if (live_b) chb_n = __ldg(reinterpret_cast<const uint4*>(sb + kb0 + 8));
-                    }
-                } else {
-                    spa0 = ha0;
-                    spa1 = ha1;
-                    spb0 = hb0;
-                    spb1 = hb1;
-                }
-            }
 #pragma unroll 1
-            for (int q = 0; q < kKBS; ++q) {
-                const int kb = kb0 + q;
-                if (kb >= KB) break;
-                float fa, fb;
-                if constexpr (kVec) {
-                    const uint32_t wa2 = q < 2 ? spa0 : spa1, wb2 = q < 2 ? spb0 : spb1;
-                    fa = __uint_as_float((q & 1) ? (wa2 & 0xFFFF0000u) : (wa2 << 16));
-                    fb = __uint_as_float((q & 1) ? (wb2 & 0xFFFF0000u) : (wb2 << 16));
-                } else {
-                    fa = __uint_as_float((uint32_t)na << 16);
-                    fb = __uint_as_float((uint32_t)nb << 16);
-                    if (!a.per_row && kb + 1 < KB) {
-                        if (live_a) na = __ldg(sa + kb + 1);
-                        if (live_b) nb = __ldg(sb + kb + 1);
-                    }
-                }
-                const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
-                const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
-                uint32_t A[4][4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
-                    unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
-                }
-                const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
-                const uint32_t cbase = st + (uint32_t)(kCorrOff + 2 * c * 16 + q * 4);
-#pragma unroll
-                for (int jn = 0; jn < kMaxNT; ++jn) {
-                    if (jn < nt) {
-                        const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
-                        const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
-                        const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                        float part[4];
-                        if constexpr (kGU) {
-                            // the preparation's offset sums of columns 2c, 2c + 1
-                            const float c0 = lds_f(cbase + (uint32_t)(jn * 8 * 16));
-                            const float c1 = lds_f(cbase + (uint32_t)(jn * 8 * 16) + 16u);
-                            part[0] = -c0;
-                            part[1] = -c1;
-                            part[2] = -c0;
-                            part[3] = -c1;
-                        } else {
-                            float cs[4];
-                            offset_sums(bw, cs);  // the unpack offsets' contribution
-                            part[0] = -cs[0];
-                            part[1] = -cs[1];
-                            part[2] = -cs[0];
-                            part[3] = -cs[1];
-                        }
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bw[2 * ks],
-                                     bw[2 * ks + 1]);
-                        acc[jn][0] = fmaf(fa, part[0], acc[jn][0]);
-                        acc[jn][1] = fmaf(fa, part[1], acc[jn][1]);
-                        acc[jn][2] = fmaf(fb, part[2], acc[jn][2]);
-                        acc[jn][3] = fmaf(fb, part[3], acc[jn][3]);
-                    }
+        for (int q = 0; q < kKBS; ++q) {
+            const int kb = kb0 + q;
+            if (kb >= KB) break;
+            float fa, fb;
+            if constexpr (kVec) {
+                const uint32_t wa2 = q < 2 ? spa0 : spa1, wb2 = q < 2 ? spb0 : spb1;
+                fa = __uint_as_float((q & 1) ? (wa2 & 0xFFFF0000u) : (wa2 << 16));
+                fb = __uint_as_float((q & 1) ? (wb2 & 0xFFFF0000u) : (wb2 << 16));
+            } else {
+                fa = __uint_as_float((uint32_t)na << 16);
+                fb = __uint_as_float((uint32_t)nb << 16);
+                if (!a.per_row && kb + 1 < KB) {
+                    if (live_a) na = __ldg(sa + kb + 1);
+                    if (live_b) nb = __ldg(sb + kb + 1);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
+            const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
+            uint32_t A[4][4];
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
+                unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
+            }
+            const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
+            const uint32_t cbase = st + (uint32_t)(kCorrOff + 2 * c * 16 + q * 4);
+#pragma unroll
+            for (int jn = 0; jn < kMaxNT; ++jn) {
+                if (jn < nt) {
+                    const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
+                    const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
+                    const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    float part[4];
+                    if constexpr (kGU) {
+                        // the preparation's offset sums of columns 2c, 2c + 1
+                        const float c0 = lds_f(cbase + (uint32_t)(jn * 8 * 16));
+                        const float c1 = lds_f(cbase + (uint32_t)(jn * 8 * 16) + 16u);
+                        part[0] = -c0;
+                        part[1] = -c1;
+                        part[2] = -c0;
+                        part[3] = -c1;
+                    } else {
+                        float cs[4];
+                        offset_sums(bw, cs);  // the unpack offsets' contribution
+                        part[0] = -cs[0];
+                        part[1] = -cs[1];
+                        part[2] = -cs[0];
+                        part[3] = -cs[1];
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bw[2 * ks],
+                                 bw[2 * ks + 1]);
+                    acc[jn][0] = fmaf(fa, part[0], acc[jn][0]);
+                    acc[jn][1] = fmaf(fa, part[1], acc[jn][1]);
+                    acc[jn][2] = fmaf(fb, part[2], acc[jn][2]);
+                    acc[jn][3] = fmaf(fb, part[3], acc[jn][3]);
+                }
+            }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (!last) continue;
 
-        // epilogue: column 8 jn + 2c + e2 is list entry n_base + that; rows
+        // epilogue: column 8 jn + 2c + e2 is list entry that of the tile; rows
         // ra (acc 0, 1) and rb (acc 2, 3)
 #pragma unroll
         for (int jn = 0; jn < kMaxNT; ++jn) {
@@ -430,7 +467,7 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
             for (int e2 = 0; e2 < 2; ++e2) {
                 const int nl = 8 * jn + 2 * c + e2;
                 if (nl >= ntok) continue;
-                const int64_t orow = sl.list_begin + n_base + nl;
+                const int64_t orow = row_begin + nl;
                 if constexpr (kGU) {
                     // h = silu(g) * u; the gate weight is applied by the combine
                     const float gv = acc[jn][e2], uv = acc[jn][2 + e2];
@@ -454,7 +491,7 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ wmaps) {
 }
 
 template <bool kGU, bool kVec>
-cudaError_t launch_one(const FfnArgs& a, const CUtensorMap* wmaps, int blocks, cudaStream_t st) {
+cudaError_t launch_one(const FfnArgs& a, const CUtensorMap* bmaps, int blocks, cudaStream_t st) {
     auto kern = batch_ffn_kernel<kGU, kVec>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemB);
     if (err != cudaSuccess) return err;
@@ -468,7 +505,7 @@ cudaError_t launch_one(const FfnArgs& a, const CUtensorMap* wmaps, int blocks, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, wmaps);
+    return cudaLaunchKernelEx(&cfg, kern, a, bmaps);
 }
 
 }  // namespace
@@ -478,19 +515,55 @@ bool batch_supported(int H, int I, int T) {
            I >= kBoxRows && I % kBoxRows == 0;
 }
 
-cudaError_t launch_batch_ffn(const FfnArgs& a, const CUtensorMap* wmaps, int num_sms,
+cudaError_t launch_batch_ffn(const FfnArgs& a, const CUtensorMap* bmaps, int num_sms,
                              cudaStream_t st) {
-    // gs64 rows of whole 16-byte chunks: scales read eight K-blocks at a time
+    // gs64 rows of whole 16-byte chunks: scales staged with the codes
     const bool vec_gu = !a.per_row && (a.H / kGroup) % 8 == 0;
     const bool vec_dn = !a.per_row && (a.I / kGroup) % 8 == 0;
     profile_mark(1, st);
-    cudaError_t err = vec_gu ? launch_one<true, true>(a, wmaps, num_sms, st)
-                             : launch_one<true, false>(a, wmaps, num_sms, st);
+    cudaError_t err = vec_gu ? launch_one<true, true>(a, bmaps, num_sms, st)
+                             : launch_one<true, false>(a, bmaps, num_sms, st);
     if (err != cudaSuccess) return err;
     profile_mark(2, st);
-    err = vec_dn ? launch_one<false, true>(a, wmaps, num_sms, st)
-                 : launch_one<false, false>(a, wmaps, num_sms, st);
+    err = vec_dn ? launch_one<false, true>(a, bmaps, num_sms, st)
+                 : launch_one<false, false>(a, bmaps, num_sms, st);
     profile_mark(3, st);
+    return err;
+}
+
+cudaError_t build_batch_maps(const DevExpert* host_experts, int n, int H, int I, bool per_row,
+                             CUtensorMap** d_maps) {
+    *d_maps = nullptr;
+    CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * 6];
+    if (!maps) return cudaErrorMemoryAllocation;
+    std::memset(maps, 0, sizeof(CUtensorMap) * (size_t)n * 6);
+    const int GH = H / kGroup, GI = I / kGroup;
+    const bool vec_gu = !per_row && GH % 8 == 0, vec_dn = !per_row && GI % 8 == 0;
+    bool ok = true;
+    for (int e = 0; e < n && ok; ++e) {
+        const DevExpert& x = host_experts[e];
+        CUtensorMap* m = maps + (size_t)e * 6;
+        const uint32_t box = kKBS * 32;  // four K-blocks of a row
+        ok = encode_codes_2d(&m[0], x.gate_q, H / 2, I, box, kBoxRows, true) &&
+             encode_codes_2d(&m[1], x.up_q, H / 2, I, box, kBoxRows, true) &&
+             encode_codes_2d(&m[2], x.down_q, I / 2, H, box, kBoxRows, true);
+        if (ok && vec_gu)
+            ok = encode_tma_rows_u16(&m[3], x.gate_s, I, GH, 8, kBoxRows) &&
+                 encode_tma_rows_u16(&m[4], x.up_s, I, GH, 8, kBoxRows);
+        if (ok && vec_dn) ok = encode_tma_rows_u16(&m[5], x.down_s, H, GI, 8, kBoxRows);
+    }
+    if (!ok) {
+        delete[] maps;
+        return cudaErrorInvalidValue;
+    }
+    cudaError_t err = cudaMalloc(d_maps, sizeof(CUtensorMap) * (size_t)n * 6);
+    if (err == cudaSuccess)
+        err = cudaMemcpy(*d_maps, maps, sizeof(CUtensorMap) * (size_t)n * 6, cudaMemcpyHostToDevice);
+    delete[] maps;
+    if (err != cudaSuccess && *d_maps) {
+        cudaFree(*d_maps);
+        *d_maps = nullptr;
+    }
     return err;
 }
 

@@ -13,6 +13,7 @@ struct coli_moe {
     int num_sms;
     coli::DevExpert* d_experts;  // device table, E + n_shared entries
     CUtensorMap* d_wmaps;        // packed-code tensor maps, 3 per expert (tensor-core path)
-    CUtensorMap* d_bmaps;        // 128-byte-wide swizzled code maps, 3 per expert (small batches)
+    CUtensorMap* d_bmaps;        // small-batch maps, 6 per expert: codes (128-byte swizzled
+                                 // boxes) and scales (8 x 128 boxes; zero where not used)
     CUtensorMap* d_dmaps;        // swizzled 3-D code maps, 3 per expert (fused decode path)
 };

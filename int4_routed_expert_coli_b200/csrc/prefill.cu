@@ -746,23 +746,20 @@ cudaError_t launch_gemm(const CUtensorMap (&bmap)[3], const GemmArgs& a, int num
 
 }  // namespace
 
-cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I, bool wide,
+cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I,
                               CUtensorMap** d_maps) {
     *d_maps = nullptr;
     CUtensorMap* maps = new (std::nothrow) CUtensorMap[(size_t)n * 3];
     if (!maps) return cudaErrorMemoryAllocation;
-    // one K-block (32 bytes) per row, or four with the 128-byte swizzle
-    const uint32_t box_bytes = wide ? 4 * (BK / 2) : BK / 2;
-    const CUtensorMapSwizzle sw = wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
     for (int e = 0; e < n; ++e) {
         const DevExpert& x = host_experts[e];
         const bool ok =
             encode_2d(&maps[e * 3 + 0], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.gate_q, H / 2, I, H / 2,
-                      box_bytes, BM, sw) &&
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.up_q, H / 2, I, H / 2,
-                      box_bytes, BM, sw) &&
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&maps[e * 3 + 2], CU_TENSOR_MAP_DATA_TYPE_UINT8, x.down_q, I / 2, H, I / 2,
-                      box_bytes, BM, sw);
+                      BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (!ok) {
             delete[] maps;
             return cudaErrorInvalidValue;
@@ -855,6 +852,12 @@ cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* x
 }
 
 bool prefill_available() { return get_encode() != nullptr; }
+
+bool encode_codes_2d(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_bytes, uint32_t box_rows, bool swizzle128) {
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, row_bytes, rows, row_bytes, box_bytes,
+                     box_rows, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
 
 bool encode_tma(CUtensorMap* m, const void* base, int rank, int rows, int row_bytes, int segs,
                 int box_rows) {

@@ -35,12 +35,14 @@ struct GatherArgs {
 };
 
 // Tensor maps of every expert's packed code matrices (device array, 3 per
-// expert: gate, up, down), boxes of 128 rows: one 64-code K-block (32 bytes,
-// unswizzled; the grouped GEMM) or, `wide`, four K-blocks (128 bytes, 128-byte
-// swizzle; the small-batch kernels).  Returns an error if the driver lacks
-// tensor maps.
-cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I, bool wide,
+// expert: gate, up, down), boxes of one 64-code K-block (32 bytes) x 128 rows.
+// Returns an error if the driver lacks tensor maps.
+cudaError_t build_weight_maps(const DevExpert* host_experts, int n, int H, int I,
                               CUtensorMap** d_maps);
+// A 2-D map of a row-major byte matrix (rows of row_bytes), boxes of
+// box_bytes x box_rows, optionally with the 128-byte swizzle.
+bool encode_codes_2d(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_bytes, uint32_t box_rows, bool swizzle128);
 // gather -> gate/up GEMM -> down GEMM (writes y); the caller runs the combine.
 cudaError_t launch_prefill(const FfnArgs& f, const CUtensorMap* wmaps, __half* xg,
                            int* ntile_start, int num_sms, cudaStream_t st);
