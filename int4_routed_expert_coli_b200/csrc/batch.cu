@@ -393,7 +393,7 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             spb0 = vb.x;
             spb1 = vb.y;
         }
-#pragma unroll 1
+#pragma unroll
         for (int q = 0; q < kKBS; ++q) {
             const int kb = kb0 + q;
             if (kb >= KB) break;
