@@ -3,12 +3,15 @@
 //
 // With a few tokens per expert, each active expert's weights are streamed
 // once for its token list (the batch-union, "yunpan.plus/t/30351-1-1",
-// capability two), and the arithmetic is the fused decode kernel's: codes
-// unpacked raw in registers (1032 + q at even k, 1152 + 16 q at odd k, whose
-// activations enter divided by 16), m16n8k16 MMAs with the activation
-// fragments as 8-token column tiles, the unpack's offset sums from an MMA of
-// its constant part with the same fragments as each chain's initial value,
-// fp32 accumulation, each group's bf16 scale applied to the group's partial.
+// capability two).  Codes are unpacked in registers by the fused decode
+// kernel's raw unpack (1032 + q at even k, 1152 + 16 q at odd k, whose
+// activations enter divided by 16) and one fp16 add takes the offsets off
+// (q, 16 q: exact), so each group's chain of m16n8k16 MMAs (the activation
+// fragments as 8-token column tiles) starts from zero; fp32 accumulation,
+// each group's bf16 scale applied to the group's partial.  (Offset sums as
+// the chains' initial values, loaded or from an MMA of the unpack's constant
+// part, put a dependent load or four MMAs in front of every chain, and were
+// slower.)
 // The weights never pass through shared-memory operands of the tensor cores
 // or tensor memory: at a few tokens per expert the grouped GEMM's fp16
 // operand costs more on-chip traffic than HBM delivers.
@@ -25,18 +28,20 @@
 // first).
 //
 // Data movement.  A producer warp stages four 64-element K-blocks at a time
-// in a ring of 4 stages of 49 KB: the codes of the tile's rows by two 2-D
-// tensor copies (128 rows x 128 bytes each, 128-byte swizzle: a narrow box of
-// one K-block per row moves a quarter of the bytes per copied row, and the
-// copy engine's row rate then limits the stream), each token's 256 activations (fragment
-// order, 512 bytes) by a 1-D bulk copy into a row of 528 bytes (the padding
-// spreads the fragment reads over the banks), and for gate/up each token's 4
-// precomputed offset sums (16 bytes).  The activations are, for gate/up, the
-// prepared x rows of the list's tokens, whose offset sums the preparation
-// computed; for down, the h' rows that the gate/up kernel wrote (odd features
-// / 16), whose offset sums an MMA computes from the fragments.  Scales are
-// read by the consumers from global memory, eight K-blocks at a time, a chunk
-// ahead.
+// in a ring of 4 stages of 53 KB: the codes of the tile's rows by two 2-D
+// tensor copies (128 rows x 128 bytes each, 128-byte swizzle: a box of one
+// K-block per row moves a quarter of the bytes per copied row, and the copy
+// engine's row rate then limits the stream); each token's 256 activations
+// (fragment order, 512 bytes) by a 1-D bulk copy into a row of 528 bytes (the
+// padding spreads the fragment reads over the banks): for gate/up the
+// prepared x rows of the list's tokens, for down the h' rows that the gate/up
+// kernel wrote (odd features / 16); and, for gs64 rows of whole 16-byte scale
+// chunks, the 8-scale chunk of each row holding the stage's four scales (two
+// 128-row tensor copies).  Other scale layouts (per-row, or K / 64 not a
+// multiple of 8) are read by the consumers from global memory.  With each
+// stage the producer writes a record of its tile (row tile, list, K-block,
+// whether it ends the tile), so the consumers run stage by stage without
+// global loads; a record with no entries ends the sequence.
 //
 // Every wait is bounded (COLI_ERR_TIMEOUT).
 #include <cuda.h>
@@ -65,11 +70,10 @@ constexpr int kKBS = 4;                               // K-blocks (scale groups)
 constexpr int kBoxBytes = kBoxRows * kKBS * 32;       // one tensor copy: 128 rows x 128 bytes
 constexpr int kCodeBytes = 2 * kBoxBytes;             // a stage's codes (two copies)
 constexpr int kActRow = kKBS * 128 + 16;              // staged activation row (bytes)
-constexpr int kCorrOff = kCodeBytes + kChunkTok * kActRow;  // offset sums, 16 B per token
-constexpr int kScaleOff = kCorrOff + kChunkTok * 16;        // scale chunks (kVec)
-constexpr int kScaleBox = kBoxRows * 16;                     // 128 rows x 8 scales
+constexpr int kScaleOff = kCodeBytes + kChunkTok * kActRow;  // scale chunks (kVec)
+constexpr int kScaleBox = kBoxRows * 16;                      // 128 rows x 8 scales
 constexpr int kScaleBytes = 2 * kScaleBox;
-constexpr int kStageB = kScaleOff + kScaleBytes;
+constexpr int kStageB = (kScaleOff + kScaleBytes + 1023) / 1024 * 1024;
 constexpr int kHdrB = 1024;
 constexpr int kSmemLimitB = 227 * 1024;
 constexpr int kStagesB = 4;
@@ -77,7 +81,7 @@ constexpr int kSmemB = kHdrB + kStagesB * kStageB + 1024;  // 1024: alignment sl
 constexpr unsigned kAllB = 0xffffffffu;
 static_assert(kSmemB <= kSmemLimitB, "stage ring");
 static_assert(kChunkTok <= 32, "one activation row per producer lane");
-static_assert(kActRow % 16 == 0 && kStageB % 16 == 0 && kCorrOff % 16 == 0, "bulk copy alignment");
+static_assert(kActRow % 16 == 0 && kScaleOff % 128 == 0, "copy destinations");
 // the 128-byte swizzle repeats every 8 rows of 128 bytes: stages stay 1 KB aligned
 static_assert(kStageB % 1024 == 0 && kHdrB % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzle atoms");
 // a staged activation row of 33 16-byte units: the 8 lanes of a quarter-warp
@@ -107,6 +111,15 @@ __device__ __forceinline__ void tma_2d(void* dst, const void* tmap, int c0, int 
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar))
         : "memory");
+}
+
+// A raw-unpacked pair less its offset: 1032 + q -> q (even k), 1152 + 16 q ->
+// 16 q (odd k); fp16 represents both sides exactly, so the sum is exact.
+__device__ __forceinline__ uint32_t strip_offset(uint32_t v, bool odd) {
+    const uint32_t neg = odd ? 0xE480E480u : 0xE408E408u;  // (-1152, -1152), (-1032, -1032)
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(neg));
+    return d;
 }
 
 // One expert slot of the call: shared experts first (every token, weight 1),
@@ -232,7 +245,6 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             // out of range reads token 0's row and is reported; the combine
             // skips it)
             const __half* src = nullptr;
-            const float* csrc = nullptr;  // gate/up: the token's offset sums
             if (lane < ntok) {
                 const int n = n_base + lane;
                 if constexpr (kGU) {
@@ -243,7 +255,6 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
                         t = (p >= 0 && p < P) ? p / a.k : 0;
                     }
                     src = a.xp + (int64_t)t * a.H;
-                    csrc = a.corr + (int64_t)t * KB;
                 } else {
                     src = a.hp + (int64_t)(sl.list_begin + n) * a.I;
                 }
@@ -258,7 +269,6 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
                 // a box past the end of K (or of the rows) is filled with zeros
                 // and counts whole
                 const uint32_t tx = (uint32_t)(kCodeBytes + ntok * nkb * 128) +
-                                    (kGU ? (uint32_t)ntok * 16u : 0u) +
                                     (kVec ? (uint32_t)kScaleBytes : 0u);
                 if (!acquire(j)) {
                     stop = true;
@@ -285,12 +295,9 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
                     }
                 }
                 __syncwarp();
-                if (lane < ntok) {
+                if (lane < ntok)
                     bulk_g2s(st + kCodeBytes + lane * kActRow, src + kb0 * kGroup,
                              (uint32_t)nkb * 128u, &full[s]);
-                    // 4 offset sums: within the row, as KB % 4 == 0 for gate/up
-                    if constexpr (kGU) bulk_g2s(st + kCorrOff + lane * 16, csrc + kb0, 16u, &full[s]);
-                }
                 ++j;
             }
         }
@@ -412,37 +419,24 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             }
             const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
             const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
+            // exact codes: q at even k, 16 q at odd k (the raw unpack less
+            // its offsets, exact in fp16), so every chain starts from zero
             uint32_t A[4][4];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
                 unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) A[ks][u] = strip_offset(A[ks][u], u >= 2);
             }
             const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
-            const uint32_t cbase = st + (uint32_t)(kCorrOff + 2 * c * 16 + q * 4);
 #pragma unroll
             for (int jn = 0; jn < kMaxNT; ++jn) {
                 if (jn < nt) {
                     const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
                     const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
                     const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                    float part[4];
-                    if constexpr (kGU) {
-                        // the preparation's offset sums of columns 2c, 2c + 1
-                        const float c0 = lds_f(cbase + (uint32_t)(jn * 8 * 16));
-                        const float c1 = lds_f(cbase + (uint32_t)(jn * 8 * 16) + 16u);
-                        part[0] = -c0;
-                        part[1] = -c1;
-                        part[2] = -c0;
-                        part[3] = -c1;
-                    } else {
-                        float cs[4];
-                        offset_sums(bw, cs);  // the unpack offsets' contribution
-                        part[0] = -cs[0];
-                        part[1] = -cs[1];
-                        part[2] = -cs[0];
-                        part[3] = -cs[1];
-                    }
+                    float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bw[2 * ks],
