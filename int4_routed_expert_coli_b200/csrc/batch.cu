@@ -47,6 +47,7 @@
 #include <cuda.h>
 
 #include <cstring>
+#include <type_traits>
 #include <new>
 
 #include "batch.cuh"
@@ -111,15 +112,6 @@ __device__ __forceinline__ void tma_2d(void* dst, const void* tmap, int c0, int 
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar))
         : "memory");
-}
-
-// A raw-unpacked pair less its offset: 1032 + q -> q (even k), 1152 + 16 q ->
-// 16 q (odd k); fp16 represents both sides exactly, so the sum is exact.
-__device__ __forceinline__ uint32_t strip_offset(uint32_t v, bool odd) {
-    const uint32_t neg = odd ? 0xE480E480u : 0xE408E408u;  // (-1152, -1152), (-1032, -1032)
-    uint32_t d;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(neg));
-    return d;
 }
 
 // One expert slot of the call: shared experts first (every token, weight 1),
@@ -400,6 +392,9 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             spb0 = vb.x;
             spb1 = vb.y;
         }
+        // the stage's MMAs with the tile's column-tile count fixed
+        auto stage_math = [&](auto ntc) {
+            constexpr int NT = decltype(ntc)::value;
 #pragma unroll
         for (int q = 0; q < kKBS; ++q) {
             const int kb = kb0 + q;
@@ -431,8 +426,8 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             }
             const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
 #pragma unroll
-            for (int jn = 0; jn < kMaxNT; ++jn) {
-                if (jn < nt) {
+            for (int jn = 0; jn < NT; ++jn) {
+                {
                     const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
                     const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
                     const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
@@ -448,6 +443,11 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
                 }
             }
         }
+        };
+        if (nt == 1) stage_math(std::integral_constant<int, 1>{});
+        else if (nt == 2) stage_math(std::integral_constant<int, 2>{});
+        else if (nt == 3) stage_math(std::integral_constant<int, 3>{});
+        else stage_math(std::integral_constant<int, 4>{});
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         if (!last) continue;

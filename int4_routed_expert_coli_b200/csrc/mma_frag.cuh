@@ -32,6 +32,15 @@ __device__ __forceinline__ void unpack_raw_step(uint32_t w, int step, uint32_t& 
     o = and_xor(v, mg.hi_mask, mg.hi_bias);
 }
 
+// A raw-unpacked pair less its offset: 1032 + q -> q (even k), 1152 + 16 q ->
+// 16 q (odd k); fp16 represents both sides exactly, so the sum is exact.
+__device__ __forceinline__ uint32_t strip_offset(uint32_t v, bool odd) {
+    const uint32_t neg = odd ? 0xE480E480u : 0xE408E408u;  // (-1152, -1152), (-1032, -1032)
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(neg));
+    return d;
+}
+
 __device__ __forceinline__ void mma16816(float d[4], const float c[4], uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
