@@ -44,9 +44,16 @@ prep_small_kernel(PrepArgs p) {
         for (int i = threadIdx.x; i < p.E + p.n_shared; i += blockDim.x) slot_cnt[i] = 0;
         for (int i = threadIdx.x; i < p.H / 32; i += blockDim.x) tile_cnt[i] = 0;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        for (int t = warp; t < p.T; t += kUnionWarps)
-            route_row<NV>(p.logits + (int64_t)t * p.E, p.E, p.k, lane, p.idx + (int64_t)t * p.k,
-                          p.w + (int64_t)t * p.k);
+        for (int t = warp; t < p.T; t += kUnionWarps) {
+            const float* row = p.logits + (int64_t)t * p.E;
+            if (route_fast_ok<NV>(p.k)) {
+                float v[8];
+                load_row8<NV>(row, p.E, lane, v);
+                route_row_fast<NV>(v, p.E, p.k, lane, p.idx + (int64_t)t * p.k, p.w + (int64_t)t * p.k);
+            } else {
+                route_row<NV>(row, p.E, p.k, lane, p.idx + (int64_t)t * p.k, p.w + (int64_t)t * p.k);
+            }
+        }
         __syncthreads();
         union_block(p.T * p.k, p.E, p.idx, p.counts, p.offsets, p.pairs, p.active, p.n_active,
                     p.inv, p.status, hist, scan_tmp);
