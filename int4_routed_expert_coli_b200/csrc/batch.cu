@@ -24,8 +24,8 @@
 // partial sums cross warps.  A list of more than 32 tokens (calls with more
 // than 32 tokens: the shared experts, popular routed ones) is split into two
 // column chunks, each a tile of its own that reads the rows again.  Tiles are
-// dealt to the CTAs (one per SM) round-robin, slot-major (shared experts
-// first).
+// numbered slot-major (shared experts first) and handed out one at a time
+// through a counter in the workspace to the CTAs (one per SM).
 //
 // Data movement.  A producer warp stages four 64-element K-blocks at a time
 // in a ring of 4 stages of 53 KB: the codes of the tile's rows by two 2-D
@@ -220,7 +220,16 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
             }
             return __shfl_sync(kAllB, ok, 0) != 0;
         };
-        for (int64_t tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
+        // tiles are handed out one at a time (the next one grabbed while the
+        // current one streams): the shared experts' and the long lists'
+        // column tiles cost more than one-token tiles, so a fixed deal leaves
+        // the CTAs that drew them behind
+        int* tile_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(a.status) + kBatchCntOffset) +
+                        (kGU ? 0 : 1);
+        int grabbed = lane == 0 ? atomicAdd(tile_cnt, 1) : 0;  // lane 0's claim, read late
+        for (int64_t tile = __shfl_sync(kAllB, grabbed, 0); tile < n_tiles && !stop;
+             tile = __shfl_sync(kAllB, grabbed, 0)) {
+            if (lane == 0) grabbed = atomicAdd(tile_cnt, 1);
             // tile -> slot (shared experts first), column chunk, row tile
             const int slot = (int)(tile / (n_chunks * m_tiles));
             const int rem = (int)(tile - (int64_t)slot * n_chunks * m_tiles);

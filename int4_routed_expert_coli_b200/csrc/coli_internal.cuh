@@ -18,6 +18,8 @@ constexpr int kMaxShared = 4;
 constexpr size_t kHeaderBytes = 16384; // status word + tile counters at the start of ws
 constexpr size_t kSlotCntOffset = 1024; // int counters: finished gate/up items per expert slot
 constexpr size_t kTileCntOffset = 8192; // int counters: finished down items per 32-row tile
+constexpr size_t kBatchCntOffset = 64;  // 2 int counters: tiles handed out by the small-batch
+                                        // gate/up and down kernels (zeroed by the preparation)
 constexpr int kSmallT = 64;            // calls with T <= kSmallT use the fused prep kernel
 
 // Device status codes live in the first word of the workspace.

@@ -626,6 +626,12 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(const FfnArgs a) {
 __global__ void prepare_x_kernel(int T, int H, const __nv_bfloat16* __restrict__ x,
                                  __half* __restrict__ xp, float* __restrict__ corr, int* status) {
     const int64_t grp = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (grp == 0) {
+        // the small-batch kernels' tile counters start at zero
+        int* cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(status) + kBatchCntOffset);
+        cnt[0] = 0;
+        cnt[1] = 0;
+    }
     if (grp >= (int64_t)T * H / kGroup) return;
     corr[grp] = prepare_group64(reinterpret_cast<const uint16_t*>(x) + grp * kGroup,
                                 xp + grp * kGroup, status);

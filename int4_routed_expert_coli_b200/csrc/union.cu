@@ -41,6 +41,8 @@ prep_small_kernel(PrepArgs p) {
         // per-call counters of the fused decode kernel start at zero
         int* slot_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(p.status) + kSlotCntOffset);
         int* tile_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(p.status) + kTileCntOffset);
+        int* batch_cnt = reinterpret_cast<int*>(reinterpret_cast<char*>(p.status) + kBatchCntOffset);
+        if (threadIdx.x < 2) batch_cnt[threadIdx.x] = 0;  // the small-batch kernels' tile counters
         for (int i = threadIdx.x; i < p.E + p.n_shared; i += blockDim.x) slot_cnt[i] = 0;
         for (int i = threadIdx.x; i < p.H / 32; i += blockDim.x) tile_cnt[i] = 0;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
