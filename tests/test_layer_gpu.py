@@ -116,15 +116,17 @@ def test_glm_decode_steps(glm):
         assert_close(out.cpu().numpy(), ref, f"decode step {s}")
 
 
-@pytest.mark.parametrize("T,n_sample,stream", [(4, 4, False), (32, 32, False), (32, 32, True)])
-def test_glm_small_batch_zipf(glm, T, n_sample, stream):
+@pytest.mark.parametrize("T,n_sample,path", [(4, 4, "default"), (32, 32, "default"),
+                                              (32, 32, "gemm"), (32, 32, "stream")])
+def test_glm_small_batch_zipf(glm, T, n_sample, path):
     """Speculative-verify / small batch: Zipf-1.1 routing, 71.6 % repeats
-    (T = 32 on the default tensor-core path and on the streaming path)."""
+    (T = 32 on the default small-batch kernels, on the tensor-core grouped
+    GEMM with small token tiles, and on the streaming path)."""
     from int4_routed_expert_coli_b200 import coli_moe as c
     bank, layer = glm
-    if stream:
+    if path != "default":
         layer = c.MoELayer(bank, n_routed=GLM["E"], top_k=GLM["k"], n_shared=1,
-                           prefill_min_tokens=10 ** 6)
+                           prefill_min_tokens=1 if path == "gemm" else 10 ** 6)
     _, logits = synth.zipf_routing(T, 256, 8, steps=2, seed=T)
     for s, lg_np in enumerate(logits):
         x = synth.make_activations(T, 6144, seed=3000 + s, device="cuda")

@@ -2,9 +2,10 @@
 COLI_GROUP_PER_ROW: "ssnai.com/JustVugg_colibri.html", decision guide, the
 older GLM-5.2 mirror) on every kernel path, against the oracle's per-row
 reading: the fused decode kernel (GLM-5.2 shape, T = 1 and 4), the
-tensor-core grouped GEMM with small token tiles (T = 32) and large ones
-(T = 512), the streaming dequant-GEMV (forced, and the tiny shape), and the
-entry point without allocation.  Same tolerance as every layer test."""
+small-batch kernels (T = 32, scales from global memory), the tensor-core
+grouped GEMM with small token tiles (T = 32) and large ones (T = 512), the
+streaming dequant-GEMV (forced, and the tiny shape), and the entry point
+without allocation.  Same tolerance as every layer test."""
 import numpy as np
 import pytest
 import torch
@@ -44,12 +45,13 @@ def test_per_row_fused_decode(glm_rows, T):
     assert_close(out.cpu().numpy(), ref, f"per-row fused decode T={T}")
 
 
-@pytest.mark.parametrize("stream", [False, True])
-def test_per_row_small_batch(glm_rows, stream):
+@pytest.mark.parametrize("path", ["default", "gemm", "stream"])
+def test_per_row_small_batch(glm_rows, path):
     from int4_routed_expert_coli_b200 import coli_moe as c
     bank, layer = glm_rows
-    if stream:
-        layer = c.MoELayer(bank, n_routed=256, top_k=8, n_shared=1, prefill_min_tokens=10 ** 6)
+    if path != "default":
+        layer = c.MoELayer(bank, n_routed=256, top_k=8, n_shared=1,
+                           prefill_min_tokens=1 if path == "gemm" else 10 ** 6)
     T = 32
     _, logits = synth.zipf_routing(T, 256, 8, steps=1, seed=84)
     x = synth.make_activations(T, 6144, seed=85, device="cuda")
@@ -57,7 +59,7 @@ def test_per_row_small_batch(glm_rows, stream):
     out, idx = _run(layer, x, lg)
     ref, ri, _ = reference_layer(bank, 256, 8, 1, x, lg)
     assert np.array_equal(idx, ri)
-    assert_close(out.cpu().numpy(), ref, f"per-row T=32 stream={stream}")
+    assert_close(out.cpu().numpy(), ref, f"per-row T=32 path={path}")
 
 
 def test_per_row_large_tiles(glm_rows):
