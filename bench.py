@@ -79,8 +79,8 @@ PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 _DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
                "4b2566a371c85094c21a668a748004e16efadabc12e262cffc246356d1698882")
 _BATCH_SRC = ("int4_routed_expert_coli_b200/csrc/batch.cu",
-              "ecd0e0f3e5e8123c3033fef1e8b8685872cda2a39c03012815fe0775d54c8348")
-_BATCH = (*_BATCH_SRC, 13_325_395, "streamed expert",
+              "b751a9116bb55d68d0e55d3f2303e77ecd0515fd6bdddd4f934c1521fe95fc3e")
+_BATCH = (*_BATCH_SRC, 13_331_461, "streamed expert",
           "ncu launch list, 12 launches of the small-batch gate/up kernel on a 64-expert bank "
           "at T=32: bytes per streamed expert (unique routed + shared)")
 DRAM_TRAFFIC = {
