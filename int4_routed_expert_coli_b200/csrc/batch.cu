@@ -405,53 +405,51 @@ batch_ffn_kernel(const FfnArgs a, const CUtensorMap* __restrict__ bmaps) {
         auto stage_math = [&](auto ntc) {
             constexpr int NT = decltype(ntc)::value;
 #pragma unroll
-        for (int q = 0; q < kKBS; ++q) {
-            const int kb = kb0 + q;
-            if (kb >= KB) break;
-            float fa, fb;
-            if constexpr (kVec) {
-                const uint32_t wa2 = q < 2 ? spa0 : spa1, wb2 = q < 2 ? spb0 : spb1;
-                fa = __uint_as_float((q & 1) ? (wa2 & 0xFFFF0000u) : (wa2 << 16));
-                fb = __uint_as_float((q & 1) ? (wb2 & 0xFFFF0000u) : (wb2 << 16));
-            } else {
-                fa = __uint_as_float((uint32_t)na << 16);
-                fb = __uint_as_float((uint32_t)nb << 16);
-                if (!a.per_row && kb + 1 < KB) {
-                    if (live_a) na = __ldg(sa + kb + 1);
-                    if (live_b) nb = __ldg(sb + kb + 1);
+            for (int q = 0; q < kKBS; ++q) {
+                const int kb = kb0 + q;
+                if (kb >= KB) break;
+                float fa, fb;
+                if constexpr (kVec) {
+                    const uint32_t wa2 = q < 2 ? spa0 : spa1, wb2 = q < 2 ? spb0 : spb1;
+                    fa = __uint_as_float((q & 1) ? (wa2 & 0xFFFF0000u) : (wa2 << 16));
+                    fb = __uint_as_float((q & 1) ? (wb2 & 0xFFFF0000u) : (wb2 << 16));
+                } else {
+                    fa = __uint_as_float((uint32_t)na << 16);
+                    fb = __uint_as_float((uint32_t)nb << 16);
+                    if (!a.per_row && kb + 1 < KB) {
+                        if (live_a) na = __ldg(sa + kb + 1);
+                        if (live_b) nb = __ldg(sb + kb + 1);
+                    }
                 }
-            }
-            const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
-            const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
-            // exact codes: q at even k, 16 q at odd k (the raw unpack less
-            // its offsets, exact in fp16), so every chain starts from zero
-            uint32_t A[4][4];
+                const uint32_t blk = st + ((((uint32_t)q) ^ rq) << 5);
+                const uint2 wa = lds_u2(blk + off_a), wb = lds_u2(blk + off_b);
+                // exact codes: q at even k, 16 q at odd k (the raw unpack less
+                // its offsets, exact in fp16), so every chain starts from zero
+                uint32_t A[4][4];
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
-                unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
+                for (int ks = 0; ks < 4; ++ks) {
+                    unpack_raw_step((ks >> 1) ? wa.y : wa.x, ks & 1, A[ks][0], A[ks][2], mg);
+                    unpack_raw_step((ks >> 1) ? wb.y : wb.x, ks & 1, A[ks][1], A[ks][3], mg);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) A[ks][u] = strip_offset(A[ks][u], u >= 2);
-            }
-            const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
+                    for (int u = 0; u < 4; ++u) A[ks][u] = strip_offset(A[ks][u], u >= 2);
+                }
+                const uint32_t bbase = st + (uint32_t)(kCodeBytes + r * kActRow + q * 128 + c * 32);
 #pragma unroll
-            for (int jn = 0; jn < NT; ++jn) {
-                {
+                for (int jn = 0; jn < NT; ++jn) {
                     const uint4 b0 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow));
                     const uint4 b1 = lds_u4(bbase + (uint32_t)(jn * 8 * kActRow) + 16u);
                     const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bw[2 * ks],
-                                 bw[2 * ks + 1]);
+                        mma16816(part, part, A[ks][0], A[ks][1], A[ks][2], A[ks][3],
+                                 bw[2 * ks], bw[2 * ks + 1]);
                     acc[jn][0] = fmaf(fa, part[0], acc[jn][0]);
                     acc[jn][1] = fmaf(fa, part[1], acc[jn][1]);
                     acc[jn][2] = fmaf(fb, part[2], acc[jn][2]);
                     acc[jn][3] = fmaf(fb, part[3], acc[jn][3]);
                 }
             }
-        }
         };
         if (nt == 1) stage_math(std::integral_constant<int, 1>{});
         else if (nt == 2) stage_math(std::integral_constant<int, 2>{});
