@@ -86,6 +86,21 @@ def test_tiny_layer_f32_residual_many_tokens(tiny):
     assert_close(out.cpu().numpy(), ref, "tiny T=203")
 
 
+@pytest.mark.parametrize("T", [19, 40])
+def test_tiny_layer_small_batch(tiny, T):
+    """Tiny layer on the small-batch kernels: H / 64 = 4 and I / 64 = 2 scale
+    groups (scales read from global memory, down's only stage half full);
+    T = 40 puts the shared expert's list in two column chunks."""
+    bank, layer = tiny
+    x = synth.make_activations(T, 256, seed=7 + T, device="cuda")
+    lg = synth.make_logits_normal(T, 16, seed=8 + T, device="cuda")
+    res = synth.make_residual(T, 256, seed=9 + T, device="cuda")
+    out, idx, w, _ = _layer(layer, x, logits=lg, residual=res)
+    ref, ri, _ = reference_layer(bank, 16, 2, 1, x, lg, residual=res)
+    assert np.array_equal(idx, ri)
+    assert_close(out.cpu().numpy(), ref, f"tiny small-batch T={T}")
+
+
 @pytest.mark.parametrize("prefill_min", [0, 10 ** 6])  # default path / streaming forced
 def test_ragged_dims_two_shared(prefill_min):
     """H, I multiples of 128 but not of 256; 12 experts top-3; 2 shared;

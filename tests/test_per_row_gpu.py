@@ -74,10 +74,12 @@ def test_per_row_large_tiles(glm_rows):
     assert_close(out.cpu().numpy()[sample], ref, "per-row T=512")
 
 
-@pytest.mark.parametrize("T", [4, 19, 203])
+@pytest.mark.parametrize("T", [4, 19, 40, 203])
 def test_per_row_tiny_all_paths(T):
-    """Tiny layer (H 256, I 128, 16 experts top-2 + 1 shared): T = 4 streams,
-    T = 19 and 203 take the tensor-core GEMM (small and large token tiles)."""
+    """Tiny layer (H 256, I 128, 16 experts top-2 + 1 shared; too small for
+    the fused decode kernel): T = 4, 19 and 40 run the small-batch kernels
+    (40: two column chunks for the shared expert), T = 203 the tensor-core
+    GEMM."""
     from int4_routed_expert_coli_b200 import coli_moe as c
     bank = synth.make_expert_bank(256, 128, 17, seed=88, device="cuda", per_row=True)
     layer = c.MoELayer(bank, n_routed=16, top_k=2, n_shared=1)
