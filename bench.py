@@ -79,7 +79,7 @@ PAIR_FLOP = 75_497_472  # 2 * 3 * H * I for the GLM-5.2 shape
 _DECODE_SRC = ("int4_routed_expert_coli_b200/csrc/decode.cu",
                "4b2566a371c85094c21a668a748004e16efadabc12e262cffc246356d1698882")
 _BATCH_SRC = ("int4_routed_expert_coli_b200/csrc/batch.cu",
-              "24f519a91e3cd8ab5209f6e3e9fe6a5cf0d67347c7ddb0052c750e7bc8055b70")
+              "915e7e0caeea9571397e94c19bb28624199bc941cf5f45f145b0d74d4e9cbbaa")
 _BATCH = (*_BATCH_SRC, 13_331_461, "streamed expert",
           "ncu launch list, 12 launches of the small-batch gate/up kernel on a 64-expert bank "
           "at T=32: bytes per streamed expert (unique routed + shared)")

@@ -1,5 +1,6 @@
 // Small-batch expert FFN: every call with up to 64 tokens that the fused
-// decode kernel does not take (more than 8 tokens, or T*k >= E).
+// decode kernel does not take (more than 8 tokens, T*k >= E, or a layer
+// shape outside the fused kernel's).
 //
 // With a few tokens per expert, each active expert's weights are streamed
 // once for its token list (the batch-union, "yunpan.plus/t/30351-1-1",
