@@ -82,7 +82,7 @@ typedef enum {
     COLI_ERR_WORKSPACE = 4,   /* workspace smaller than coli_moe_workspace_size */
     COLI_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, copy, allocation) */
     COLI_ERR_TIMEOUT = 6,     /* a bounded device wait gave up (status word) */
-    COLI_ERR_UNSUPPORTED = 7, /* no sm_100 device, or a feature this build lacks */
+    COLI_ERR_UNSUPPORTED = 7, /* no sm_100 device, or a feature the library lacks */
     COLI_ERR_BAD_INDEX = 8,   /* device saw an expert index outside [0, E) (status word) */
     COLI_ERR_RANGE = 9        /* a SwiGLU output exceeded the fp16 range and was clamped to
                                  +-65504 before the down projection (status word) */
